@@ -1,0 +1,350 @@
+// C-ABI entry points of libcosa.so: argument validation, workspace layout and
+// kernel launches.  All arithmetic of the method runs in the kernels included
+// below; this file only checks sizes and marshals pointers.
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+
+#include "common.cuh"
+#include "kap.cuh"
+#include "attn_mma.cuh"
+
+using namespace cosa;
+
+namespace {
+
+constexpr int kVersion = (0 << 16) | (1 << 8) | 0;
+
+bool is_pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
+
+cosa_status_t check_shape(const cosa_shape_t* s) {
+  if (!s) return COSA_ERR_INVALID_ARG;
+  if (s->batch <= 0 || s->num_q_heads <= 0 || s->num_kv_heads <= 0 || s->seq_len <= 0 ||
+      s->head_dim <= 0 || s->page_size <= 0 || s->q_block <= 0 || s->pages_per_seq <= 0 ||
+      s->num_phys_pages <= 0)
+    return COSA_ERR_INVALID_ARG;
+  if (!(s->softmax_scale > 0.f) || !std::isfinite(s->softmax_scale)) return COSA_ERR_INVALID_ARG;
+  if (s->num_q_heads % s->num_kv_heads) return COSA_ERR_INVALID_ARG;
+  if (s->seq_len % s->page_size || s->seq_len % s->q_block) return COSA_ERR_INVALID_ARG;
+  if (s->pages_per_seq < s->seq_len / s->page_size) return COSA_ERR_INVALID_ARG;
+  if (s->head_dim != 64 && s->head_dim != 128) return COSA_ERR_UNSUPPORTED;
+  if (s->page_size != 64 && s->page_size != 128) return COSA_ERR_UNSUPPORTED;
+  if (s->q_block != 64 && s->q_block != 128) return COSA_ERR_UNSUPPORTED;
+  // index arithmetic stays in 32 bits for token/page counts, 64 bits for offsets
+  if ((long long)s->seq_len > (1ll << 30)) return COSA_ERR_UNSUPPORTED;
+  return COSA_OK;
+}
+
+cosa_status_t check_kap(const cosa_shape_t* s, const cosa_kap_params_t* k) {
+  if (!k) return COSA_ERR_INVALID_ARG;
+  if (!(k->budget >= 0.f && k->budget <= 1.f)) return COSA_ERR_INVALID_ARG;
+  if (k->q_sub <= 0 || k->k_sub <= 0 || k->sink_pages < 0) return COSA_ERR_INVALID_ARG;
+  if (k->ascending != 0 && k->ascending != 1) return COSA_ERR_INVALID_ARG;
+  if (s->q_block % k->q_sub || s->page_size % k->k_sub) return COSA_ERR_INVALID_ARG;
+  int R = s->q_block / k->q_sub, T = s->page_size / k->k_sub;
+  if (!is_pow2(R) || R > 8 || !is_pow2(T) || T > 8) return COSA_ERR_UNSUPPORTED;
+  return COSA_OK;
+}
+
+struct KapLayout {
+  size_t qhat_off, khat_off, scores_off, hrm_off, total;
+};
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+KapLayout kap_layout(const cosa_shape_t* s, const cosa_kap_params_t* k) {
+  KapLayout L;
+  const size_t B = s->batch, Hq = s->num_q_heads, Hk = s->num_kv_heads, N = s->seq_len,
+               D = s->head_dim;
+  const size_t nP = N / s->page_size, nQB = N / s->q_block;
+  size_t off = 0;
+  L.qhat_off = off;
+  off = align256(off + B * Hq * (N / k->q_sub) * D * sizeof(float));
+  L.khat_off = off;
+  off = align256(off + B * Hk * (N / k->k_sub) * D * sizeof(float));
+  L.scores_off = off;
+  off = align256(off + B * Hq * nQB * nP * sizeof(float));
+  L.hrm_off = off;
+  off = align256(off + B * Hq * nQB * nP);
+  L.total = off;
+  return L;
+}
+
+int kcap_of(const cosa_shape_t* s, const cosa_kap_params_t* k) {
+  int best = 0;
+  const int nQB = s->seq_len / s->q_block;
+  for (int qb = 0; qb < nQB; ++qb) {
+    int v = budget_count(qb, s->q_block, s->page_size, k->sink_pages, k->budget);
+    best = v > best ? v : best;
+  }
+  return best;
+}
+
+cosa_status_t last_launch() {
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    return COSA_ERR_CUDA;
+  }
+  return COSA_OK;
+}
+
+// Score kernel: heads per CTA = largest divisor of G whose representatives and
+// score rows fit the shared-memory budget.
+constexpr size_t kScoreSmemLimit = 200 * 1024;
+
+template <int D>
+size_t score_smem(int hpc, int R, int nP) {
+  return (size_t)SCORE_MAXNR * 4 * (D / 4 + 4) * sizeof(float) + (size_t)hpc * R * nP * sizeof(float);
+}
+
+template <int D>
+cosa_status_t launch_kap(const cosa_shape_t* s, const cosa_kap_params_t* k, const void* q,
+                         const void* k_pool, const int32_t* page_table, int32_t* order,
+                         int32_t* count, float* scores, uint8_t* hrm, const KapLayout& L,
+                         uint8_t* ws, int k_cap, cudaStream_t st) {
+  const int B = s->batch, Hq = s->num_q_heads, Hk = s->num_kv_heads, N = s->seq_len;
+  const int P = s->page_size, Bq = s->q_block, nP = N / P, nQB = N / Bq;
+  const int R = Bq / k->q_sub, T = P / k->k_sub, G = Hq / Hk;
+  float* qhat = reinterpret_cast<float*>(ws + L.qhat_off);
+  float* khat = reinterpret_cast<float*>(ws + L.khat_off);
+  float* sc = scores ? scores : reinterpret_cast<float*>(ws + L.scores_off);
+  uint8_t* hr = hrm ? hrm : ws + L.hrm_off;
+
+  // K1
+  const long long n_qvec = (long long)B * Hq * (N / k->q_sub);
+  const long long n_kvec = (long long)B * Hk * nP * T;
+  const long long warps = n_qvec + n_kvec;
+  const long long blocks = (warps + 7) / 8;
+  if (blocks > 0x7fffffffll) return COSA_ERR_UNSUPPORTED;
+  kap_pool_kernel<D><<<(unsigned)blocks, 256, 0, st>>>(
+      reinterpret_cast<const __nv_bfloat16*>(q), reinterpret_cast<const __nv_bfloat16*>(k_pool),
+      page_table, qhat, khat, n_qvec, k->q_sub, n_kvec, k->k_sub, Hk, P, nP, s->pages_per_seq, T);
+  if (last_launch() != COSA_OK) return COSA_ERR_CUDA;
+
+  // K2
+  int hpc = 0;
+  for (int d = G; d >= 1; --d) {
+    if (G % d) continue;
+    if (d * R > SCORE_MAXNR) continue;
+    if (score_smem<D>(d, R, nP) > kScoreSmemLimit) continue;
+    hpc = d;
+    break;
+  }
+  if (hpc == 0) return COSA_ERR_UNSUPPORTED;
+  size_t smem2 = score_smem<D>(hpc, R, nP);
+  if (cudaFuncSetAttribute(kap_score_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)smem2) != cudaSuccess)
+    return COSA_ERR_CUDA;
+  dim3 g2(nQB, B * Hk * (G / hpc));
+  kap_score_kernel<D><<<g2, SCORE_THREADS, smem2, st>>>(qhat, khat, sc, hr, Hq, Hk, G, hpc, nQB,
+                                                       nP, R, T, k->q_sub, k->k_sub, P, Bq,
+                                                       s->softmax_scale);
+  if (last_launch() != COSA_OK) return COSA_ERR_CUDA;
+
+  // K3
+  int npow2 = 1;
+  while (npow2 < nP) npow2 <<= 1;
+  size_t smem3 = (size_t)npow2 * 8 + (size_t)nP * 4;
+  if (smem3 > 200 * 1024) return COSA_ERR_UNSUPPORTED;
+  if (cudaFuncSetAttribute(kap_order_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)smem3) != cudaSuccess)
+    return COSA_ERR_CUDA;
+  dim3 g3(nQB, B * Hq);
+  kap_order_kernel<<<g3, ORDER_THREADS, smem3, st>>>(sc, hr, order, count, nQB, nP, Bq, P,
+                                                     k->budget, k->sink_pages, k->ascending, k_cap);
+  return last_launch();
+}
+
+template <int D, int P, int BQ, bool DENSE>
+cosa_status_t launch_attn_t(const AttnParams& prm, int grid, cudaStream_t st) {
+  const size_t smem = (size_t)(BQ * D + 4 * P * D) * sizeof(__nv_bfloat16);
+  auto kern = attn_mma_kernel<D, P, BQ, DENSE>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+      cudaSuccess)
+    return COSA_ERR_CUDA;
+  kern<<<grid, BQ * 2, smem, st>>>(prm);
+  return last_launch();
+}
+
+template <bool DENSE>
+cosa_status_t launch_attn(const cosa_shape_t* s, const AttnParams& prm, int grid, cudaStream_t st) {
+  const int D = s->head_dim, P = s->page_size, BQ = s->q_block;
+#define COSA_ATTN_CASE(d, p, bq) \
+  if (D == d && P == p && BQ == bq) return launch_attn_t<d, p, bq, DENSE>(prm, grid, st);
+  COSA_ATTN_CASE(128, 64, 128)
+  COSA_ATTN_CASE(128, 128, 128)
+  COSA_ATTN_CASE(128, 64, 64)
+  COSA_ATTN_CASE(128, 128, 64)
+  COSA_ATTN_CASE(64, 64, 128)
+  COSA_ATTN_CASE(64, 128, 128)
+  COSA_ATTN_CASE(64, 64, 64)
+  COSA_ATTN_CASE(64, 128, 64)
+#undef COSA_ATTN_CASE
+  return COSA_ERR_UNSUPPORTED;
+}
+
+AttnParams make_params(const cosa_shape_t* s, const void* q, const void* k_pool,
+                       const void* v_pool, const int32_t* page_table, void* out, float* lse) {
+  AttnParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.q = reinterpret_cast<const __nv_bfloat16*>(q);
+  p.k_pool = reinterpret_cast<const __nv_bfloat16*>(k_pool);
+  p.v_pool = reinterpret_cast<const __nv_bfloat16*>(v_pool);
+  p.page_table = page_table;
+  p.out = reinterpret_cast<__nv_bfloat16*>(out);
+  p.lse = lse;
+  p.num_q_heads = s->num_q_heads;
+  p.num_kv_heads = s->num_kv_heads;
+  p.group = s->num_q_heads / s->num_kv_heads;
+  p.seq_len = s->seq_len;
+  p.num_q_blocks = s->seq_len / s->q_block;
+  p.pages_per_seq = s->pages_per_seq;
+  p.scale_log2 = s->softmax_scale * 1.4426950408889634f;
+  p.log2_eps = -INFINITY;
+  return p;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* cosa_status_string(cosa_status_t st) {
+  switch (st) {
+    case COSA_OK: return "ok";
+    case COSA_ERR_INVALID_ARG: return "invalid argument";
+    case COSA_ERR_UNSUPPORTED: return "unsupported shape or parameter";
+    case COSA_ERR_CUDA: return "CUDA error";
+    case COSA_ERR_TIMEOUT: return "kernel wait timed out";
+    case COSA_ERR_WORKSPACE: return "workspace missing or too small";
+  }
+  return "unknown status";
+}
+
+int32_t cosa_version(void) { return kVersion; }
+
+cosa_status_t cosa_kap_kcap(const cosa_shape_t* shape, const cosa_kap_params_t* kap,
+                            int32_t* k_cap) {
+  cosa_status_t e = check_shape(shape);
+  if (e != COSA_OK) return e;
+  if ((e = check_kap(shape, kap)) != COSA_OK) return e;
+  if (!k_cap) return COSA_ERR_INVALID_ARG;
+  *k_cap = kcap_of(shape, kap);
+  return COSA_OK;
+}
+
+cosa_status_t cosa_kap_workspace_size(const cosa_shape_t* shape, const cosa_kap_params_t* kap,
+                                      size_t* bytes) {
+  cosa_status_t e = check_shape(shape);
+  if (e != COSA_OK) return e;
+  if ((e = check_kap(shape, kap)) != COSA_OK) return e;
+  if (!bytes) return COSA_ERR_INVALID_ARG;
+  *bytes = kap_layout(shape, kap).total;
+  return COSA_OK;
+}
+
+cosa_status_t cosa_kap_select(const cosa_shape_t* shape, const cosa_kap_params_t* kap,
+                              const void* q, const void* k_pool, const int32_t* page_table,
+                              int32_t* order, int32_t* count, float* scores, uint8_t* hrm,
+                              void* workspace, size_t workspace_bytes, cosa_stream_t stream) {
+  cosa_status_t e = check_shape(shape);
+  if (e != COSA_OK) return e;
+  if ((e = check_kap(shape, kap)) != COSA_OK) return e;
+  if (!q || !k_pool || !page_table || !order || !count) return COSA_ERR_INVALID_ARG;
+  KapLayout L = kap_layout(shape, kap);
+  if (!workspace || workspace_bytes < L.total) return COSA_ERR_WORKSPACE;
+  if (reinterpret_cast<uintptr_t>(workspace) % 256) return COSA_ERR_WORKSPACE;
+  if (reinterpret_cast<uintptr_t>(q) % 16 || reinterpret_cast<uintptr_t>(k_pool) % 16)
+    return COSA_ERR_INVALID_ARG;
+  const int k_cap = kcap_of(shape, kap);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* ws = reinterpret_cast<uint8_t*>(workspace);
+  if (shape->head_dim == 128)
+    return launch_kap<128>(shape, kap, q, k_pool, page_table, order, count, scores, hrm, L, ws,
+                           k_cap, st);
+  return launch_kap<64>(shape, kap, q, k_pool, page_table, order, count, scores, hrm, L, ws, k_cap,
+                        st);
+}
+
+cosa_status_t cosa_kap_order(const cosa_shape_t* shape, const cosa_kap_params_t* kap,
+                             const float* scores, const uint8_t* hrm, int32_t* order,
+                             int32_t* count, cosa_stream_t stream) {
+  cosa_status_t e = check_shape(shape);
+  if (e != COSA_OK) return e;
+  if ((e = check_kap(shape, kap)) != COSA_OK) return e;
+  if (!scores || !hrm || !order || !count) return COSA_ERR_INVALID_ARG;
+  const int N = shape->seq_len, P = shape->page_size, Bq = shape->q_block;
+  const int nP = N / P, nQB = N / Bq;
+  int npow2 = 1;
+  while (npow2 < nP) npow2 <<= 1;
+  size_t smem3 = (size_t)npow2 * 8 + (size_t)nP * 4;
+  if (smem3 > 200 * 1024) return COSA_ERR_UNSUPPORTED;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaFuncSetAttribute(kap_order_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)smem3) != cudaSuccess)
+    return COSA_ERR_CUDA;
+  dim3 g3(nQB, shape->batch * shape->num_q_heads);
+  kap_order_kernel<<<g3, ORDER_THREADS, smem3, st>>>(scores, hrm, order, count, nQB, nP, Bq, P,
+                                                     kap->budget, kap->sink_pages, kap->ascending,
+                                                     kcap_of(shape, kap));
+  return last_launch();
+}
+
+cosa_status_t cosa_osk_attention(const cosa_shape_t* shape, const cosa_osk_params_t* osk,
+                                 const void* q, const void* k_pool, const void* v_pool,
+                                 const int32_t* page_table, const int32_t* order,
+                                 const int32_t* count, int32_t k_cap, void* out, float* lse,
+                                 int32_t* computed, uint8_t* skip_log, cosa_stream_t stream) {
+  cosa_status_t e = check_shape(shape);
+  if (e != COSA_OK) return e;
+  if (!osk || !(osk->eps >= 0.f)) return COSA_ERR_INVALID_ARG;
+  if (!q || !k_pool || !v_pool || !page_table || !order || !count || !out)
+    return COSA_ERR_INVALID_ARG;
+  if (k_cap <= 0 || k_cap > shape->seq_len / shape->page_size) return COSA_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(q) % 16 || reinterpret_cast<uintptr_t>(k_pool) % 16 ||
+      reinterpret_cast<uintptr_t>(v_pool) % 16 || reinterpret_cast<uintptr_t>(out) % 16)
+    return COSA_ERR_INVALID_ARG;
+  AttnParams p = make_params(shape, q, k_pool, v_pool, page_table, out, lse);
+  p.order = order;
+  p.count = count;
+  p.computed = computed;
+  p.skip_log = skip_log;
+  p.k_cap = k_cap;
+  p.log2_eps = osk->eps > 0.f ? log2f(osk->eps) : -INFINITY;
+  const long long grid = (long long)shape->batch * shape->num_q_heads * (shape->seq_len / shape->q_block);
+  if (grid > 0x7fffffffll) return COSA_ERR_UNSUPPORTED;
+  return launch_attn<false>(shape, p, (int)grid, reinterpret_cast<cudaStream_t>(stream));
+}
+
+cosa_status_t cosa_dense_attention(const cosa_shape_t* shape, const void* q, const void* k_pool,
+                                   const void* v_pool, const int32_t* page_table, void* out,
+                                   float* lse, cosa_stream_t stream) {
+  cosa_status_t e = check_shape(shape);
+  if (e != COSA_OK) return e;
+  if (!q || !k_pool || !v_pool || !page_table || !out) return COSA_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(q) % 16 || reinterpret_cast<uintptr_t>(k_pool) % 16 ||
+      reinterpret_cast<uintptr_t>(v_pool) % 16 || reinterpret_cast<uintptr_t>(out) % 16)
+    return COSA_ERR_INVALID_ARG;
+  AttnParams p = make_params(shape, q, k_pool, v_pool, page_table, out, lse);
+  const long long grid = (long long)shape->batch * shape->num_q_heads * (shape->seq_len / shape->q_block);
+  if (grid > 0x7fffffffll) return COSA_ERR_UNSUPPORTED;
+  return launch_attn<true>(shape, p, (int)grid, reinterpret_cast<cudaStream_t>(stream));
+}
+
+cosa_status_t cosa_get_status(cosa_stream_t stream) {
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  int v = 0;
+  if (cudaMemcpyFromSymbolAsync(&v, g_status, sizeof(int), 0, cudaMemcpyDeviceToHost, st) !=
+      cudaSuccess)
+    return COSA_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return COSA_ERR_CUDA;
+  if (v != 0) {
+    int zero = 0;
+    if (cudaMemcpyToSymbolAsync(g_status, &zero, sizeof(int), 0, cudaMemcpyHostToDevice, st) !=
+            cudaSuccess ||
+        cudaStreamSynchronize(st) != cudaSuccess)
+      return COSA_ERR_CUDA;
+  }
+  return static_cast<cosa_status_t>(v);
+}
+
+}  // extern "C"

@@ -1,0 +1,178 @@
+/*
+ * cosa.h — C interface of the CoSA block-sparse causal prefill attention library
+ * (libcosa.so, sm_100a).
+ *
+ * The method: "CoSA: Accelerating Long-Context Inference via Proxy-Kernel
+ * Co-Designed Sparse Attention".  Its abstract (insight.artgrammer.co.kr,
+ * fugumt.com) fixes two stages: a Kernel-Aware Proxy (KAP) that selects KV
+ * blocks under a moderate budget and emits an *ordered* mask, the order in
+ * which the kernel's inner loop visits KV pages; and an Ordered-Skipping Kernel
+ * (OSK) that applies the mask and skips further blocks from online-softmax
+ * statistics.  The technical summary on gist.science/pt gives the steps:
+ * §2.2 "Estágio 1: KAP" (downsampling, approximate scores, MaxPool over keys,
+ * MaxNorm, HRM flags, flag-group ordering) and §2.3 "Estágio 2: OSK" (mask-
+ * skipped pages via KV page remapping, in-kernel skip on local max vs running
+ * max, computed pages).
+ *
+ * Conventions for every entry point
+ *   - All tensor arguments are DEVICE pointers on the current CUDA device,
+ *     allocated and owned by the caller; the library allocates no device
+ *     memory per call and keeps no pointer after the call is enqueued.
+ *   - Layouts are dense, row-major (last index fastest):
+ *       q          bf16  [B][H_q][N][D]
+ *       k_pool     bf16  [num_phys_pages][H_kv][P][D]   (one page of one KV head
+ *                                                      is a contiguous P*D block)
+ *       v_pool     bf16  [num_phys_pages][H_kv][P][D]
+ *       page_table int32 [B][pages_per_seq]   logical page -> physical page
+ *       out        bf16  [B][H_q][N][D]
+ *       lse        fp32  [B][H_q][N]          natural-log softmax normaliser
+ *       order      int32 [B][H_q][nQB][k_cap] logical page ids, -1 past count
+ *       count      int32 [B][H_q][nQB]
+ *       scores     fp32  [B][H_q][nQB][nP]    proxy score S (0 past n_b)
+ *       hrm        uint8 [B][H_q][nQB][nP]    Have-RowMax flags (0 past n_b)
+ *     with N = seq_len, nP = N / P, nQB = N / Bq, and query head h reading KV
+ *     head h / (H_q / H_kv).  Query i attends to keys 0..i (causal prefill).
+ *   - Calls are asynchronous on `stream` (0 = legacy default stream).
+ *     Argument errors are detected on the host and returned before anything
+ *     is launched.  Launch failures return COSA_ERR_CUDA.  Errors detected
+ *     inside a kernel (a bounded wait that ran out) are recorded in a
+ *     per-device status word; read it with cosa_get_status().
+ *   - Supported shapes (COSA_ERR_UNSUPPORTED otherwise): D = 128 (all kernels)
+ *     or D = 64 (KAP and the attention kernels); P in {64, 128};
+ *     Bq in {64, 128}; N a multiple of P and of Bq; H_q a multiple of H_kv;
+ *     page_table entries in [0, num_phys_pages) (not checked: the caller's
+ *     contract, as for any index buffer).
+ */
+#ifndef COSA_H_
+#define COSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* cosa_stream_t; /* a cudaStream_t */
+
+typedef enum {
+  COSA_OK = 0,
+  COSA_ERR_INVALID_ARG = 1, /* null pointer, negative or inconsistent size       */
+  COSA_ERR_UNSUPPORTED = 2, /* valid but outside the supported shape set        */
+  COSA_ERR_CUDA = 3,        /* a CUDA runtime/driver call or a launch failed     */
+  COSA_ERR_TIMEOUT = 4,     /* a kernel's bounded wait ran out (status word)     */
+  COSA_ERR_WORKSPACE = 5    /* workspace missing or smaller than required        */
+} cosa_status_t;
+
+/* Problem shape shared by all entry points. */
+typedef struct {
+  int32_t batch;          /* B                                                  */
+  int32_t num_q_heads;    /* H_q                                                */
+  int32_t num_kv_heads;   /* H_kv, divides H_q                                  */
+  int32_t seq_len;        /* N (prefill length; queries and keys)               */
+  int32_t head_dim;       /* D                                                  */
+  int32_t page_size;      /* P tokens per KV page                               */
+  int32_t q_block;        /* Bq query rows per q-block (one OSK tile)           */
+  int32_t pages_per_seq;  /* row stride of page_table, >= N / P                 */
+  int32_t num_phys_pages; /* rows of k_pool / v_pool                            */
+  float softmax_scale;    /* multiplies q.k (usually 1/sqrt(D))                 */
+} cosa_shape_t;
+
+/* Kernel-Aware Proxy parameters (gist.science/pt §2.2). */
+typedef struct {
+  float budget;       /* fraction of a q-block's causal pages to keep, in [0,1]; the
+                         kept count is ceil(fl32(budget * n_b)), at least the forced
+                         pages, at most n_b                                           */
+  int32_t q_sub;      /* query rows pooled into one representative; divides Bq,
+                         Bq / q_sub in {1, 2, 4, 8}                                   */
+  int32_t k_sub;      /* keys pooled into one sub-key; divides P, P / k_sub in
+                         {1, 2, 4, 8}                                                 */
+  int32_t sink_pages; /* leading pages always kept (>= 0); the q-block's own pages
+                         are always kept too                                          */
+  int32_t ascending;  /* 0: list kept pages by rank (HRM first, then score
+                         descending, then lower page id) — the ordered mask;
+                         1: list them by page id (a binary mask's visit order)       */
+} cosa_kap_params_t;
+
+/* Ordered-Skipping Kernel parameters (gist.science/pt §2.3). */
+typedef struct {
+  float eps; /* >= 0.  A listed page other than the first is skipped when, for every
+                row of the q-block that sees a key in it, (page max logit - running
+                max) < ln(eps).  0 never skips; +inf skips every page after the
+                first unless some row meets its first visible key there.          */
+} cosa_osk_params_t;
+
+/* Status string for a status code (static storage, never NULL). */
+const char* cosa_status_string(cosa_status_t status);
+
+/* Library version as (major << 16) | (minor << 8) | patch. */
+int32_t cosa_version(void);
+
+/* Length of one ordered-page row: the largest per-q-block kept count k_b.
+ * Host-only; no CUDA call. */
+cosa_status_t cosa_kap_kcap(const cosa_shape_t* shape, const cosa_kap_params_t* kap,
+                            int32_t* k_cap);
+
+/* Bytes of device workspace cosa_kap_select needs (pooled queries and keys,
+ * scores and HRM flags).  Host-only; no CUDA call. */
+cosa_status_t cosa_kap_workspace_size(const cosa_shape_t* shape, const cosa_kap_params_t* kap,
+                                      size_t* bytes);
+
+/* Stage 1, all steps (gist.science/pt §2.2 "Ranking de Blocos", "Geração de
+ * Flag HRM", "Ordenação por Grupo de Flags"; abstract: "selects blocks under a
+ * moderate budget and produces an ordered mask"):
+ *   q^ = mean of q_sub consecutive rows, k^ = mean of k_sub consecutive keys;
+ *   a[r][p] = max over causally visible sub-keys of scale * <q^_r, k^_{p,t}>;
+ *   S[p] = mean_r exp(a[r][p] - max_p' a[r][p']); HRM[p] = page holding the row
+ *   max of some representative (lowest page on ties);
+ *   keep the forced pages (sink_pages leading pages + the q-block's own pages)
+ *   plus the best-ranked others up to k_b; list them by rank (or by page id).
+ * Writes order (k_cap entries per q-block, -1 padded) and count.  scores / hrm
+ * may be NULL; when given, the per-page S and flags are written there too.
+ * workspace: device buffer of at least cosa_kap_workspace_size bytes, 256-byte
+ * aligned; its contents on entry do not matter. */
+cosa_status_t cosa_kap_select(const cosa_shape_t* shape, const cosa_kap_params_t* kap,
+                              const void* q, const void* k_pool, const int32_t* page_table,
+                              int32_t* order, int32_t* count, float* scores, uint8_t* hrm,
+                              void* workspace, size_t workspace_bytes, cosa_stream_t stream);
+
+/* Stage 1, selection and ordering only (gist.science/pt §2.2 "Ordenação por
+ * Grupo de Flags"), from caller-given scores (fp32, >= 0) and HRM flags laid out
+ * as above; entries past each q-block's causal pages are ignored.  Given the
+ * same scores and flags, the result is fully determined (ties broken by page
+ * id), so it is bit-reproducible.  No workspace. */
+cosa_status_t cosa_kap_order(const cosa_shape_t* shape, const cosa_kap_params_t* kap,
+                             const float* scores, const uint8_t* hrm, int32_t* order,
+                             int32_t* count, cosa_stream_t stream);
+
+/* Stage 2 (gist.science/pt §2.3): for every (b, h_q, q-block) visit the listed
+ * pages order[0..count) in list order through the page table (unlisted pages are
+ * never read), accumulate online softmax, and skip a page per the eps rule above
+ * (one decision per q-block tile; skipped pages change nothing).
+ * order/count as written by cosa_kap_select (or any list of distinct causal
+ * pages per q-block, count >= 1, order[j] < n_b).  lse, computed (int32
+ * [B][H_q][nQB], pages actually computed) and skip_log (uint8
+ * [B][H_q][nQB][k_cap], 1 = skipped, entries past count untouched) may be NULL. */
+cosa_status_t cosa_osk_attention(const cosa_shape_t* shape, const cosa_osk_params_t* osk,
+                                 const void* q, const void* k_pool, const void* v_pool,
+                                 const int32_t* page_table, const int32_t* order,
+                                 const int32_t* count, int32_t k_cap, void* out, float* lse,
+                                 int32_t* computed, uint8_t* skip_log, cosa_stream_t stream);
+
+/* Dense causal attention over the same paged cache (every causal page in page
+ * order, no skipping): the comparison point for the sparse path's speedup.
+ * lse may be NULL. */
+cosa_status_t cosa_dense_attention(const cosa_shape_t* shape, const void* q, const void* k_pool,
+                                   const void* v_pool, const int32_t* page_table, void* out,
+                                   float* lse, cosa_stream_t stream);
+
+/* Read (and clear) the current device's status word: COSA_OK, or the first
+ * in-kernel error recorded since the last call (e.g. COSA_ERR_TIMEOUT).
+ * Synchronises `stream`. */
+cosa_status_t cosa_get_status(cosa_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* COSA_H_ */

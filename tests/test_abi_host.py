@@ -1,0 +1,114 @@
+"""Host-side checks of the C-ABI library (no GPU): it loads, exports every
+symbol include/cosa.h declares, and validates arguments on the host before any
+CUDA call."""
+import ctypes
+import math
+import os
+import re
+
+import pytest
+
+import block_sparse_long_kap_b200 as C
+import oracle as O
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_symbols():
+    text = open(os.path.join(ROOT, "include", "cosa.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(cosa_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_library_exports_every_declared_symbol():
+    lib = ctypes.CDLL(C.library_path)
+    declared = _declared_symbols()
+    assert declared, "no declarations parsed"
+    for name in declared:
+        assert hasattr(lib, name), f"{name} declared in cosa.h but not exported"
+    assert set(declared) == set(C.EXPORTED_SYMBOLS)
+
+
+def test_status_strings_and_version():
+    for code in range(6):
+        assert C.cosa_status_string(code)
+    assert C.cosa_status_string(99) == "unknown status"
+    assert C.cosa_version() > 0
+
+
+@pytest.mark.parametrize("N,P,Bq,budget,sink", [
+    (131072, 64, 128, 0.2, 1), (32768, 64, 128, 0.1, 1), (65536, 64, 128, 0.05, 1),
+    (131072, 128, 128, 0.15, 1), (2048, 64, 64, 0.25, 1), (4096, 128, 64, 0.5, 2),
+    (1024, 64, 128, 0.0, 0), (1024, 64, 128, 1.0, 1)])
+def test_kcap_matches_oracle(N, P, Bq, budget, sink):
+    s = C.Shape(1, 4, 2, N, 128, P, Bq)
+    k = C.KapParams(budget=budget, sink_pages=sink)
+    assert C.cosa_kap_kcap(s, k) == O.k_cap(N, Bq, P, sink, budget)
+
+
+def test_workspace_size_covers_pooled_vectors_and_scores():
+    s = C.Shape(1, 32, 8, 131072, 128, 64, 128)
+    k = C.KapParams(0.2, q_sub=32, k_sub=16)
+    need = (32 * 4096 * 128 * 4) + (8 * 8192 * 128 * 4) + 32 * 1024 * 2048 * 5
+    got = C.cosa_kap_workspace_size(s, k)
+    assert need <= got <= need + 4 * 256
+
+
+def _status(fn):
+    try:
+        fn()
+    except C.CosaError as e:
+        return e.status
+    return 0
+
+
+@pytest.mark.parametrize("bad,code", [
+    (dict(head_dim=96), 2), (dict(page_size=32), 2), (dict(q_block=256), 2),
+    (dict(seq_len=1000), 1), (dict(num_kv_heads=3), 1), (dict(batch=0), 1),
+    (dict(softmax_scale=-1.0), 1), (dict(pages_per_seq=3), 1)])
+def test_invalid_shapes_rejected_on_host(bad, code):
+    kw = dict(batch=1, num_q_heads=4, num_kv_heads=2, seq_len=1024, head_dim=128, page_size=64,
+              q_block=128)
+    kw.update(bad)
+    s = C.Shape(**kw)
+    if "softmax_scale" in bad:
+        s.softmax_scale = bad["softmax_scale"]
+    assert _status(lambda: C.cosa_kap_kcap(s, C.KapParams())) == code
+
+
+@pytest.mark.parametrize("bad,code", [
+    (dict(budget=1.5), 1), (dict(budget=-0.1), 1), (dict(budget=float("nan")), 1),
+    (dict(q_sub=48), 1), (dict(k_sub=5), 1), (dict(q_sub=8), 2), (dict(k_sub=4), 2),
+    (dict(sink_pages=-1), 1)])
+def test_invalid_kap_params_rejected_on_host(bad, code):
+    s = C.Shape(1, 4, 2, 1024, 128, 64, 128)
+    assert _status(lambda: C.cosa_kap_kcap(s, C.KapParams(**bad))) == code
+
+
+def test_null_pointers_and_bad_eps_rejected_before_launch():
+    lib = C.lib()
+    s = C.Shape(1, 4, 2, 1024, 128, 64, 128).c()
+    k = C.KapParams().c(C.Shape(1, 4, 2, 1024, 128, 64, 128))
+    o = C._Osk(1e-4)
+    # null q
+    assert lib.cosa_osk_attention(ctypes.byref(s), ctypes.byref(o), None, 16, 16, 16, 16, 16, 4,
+                                  16, None, None, None, None) == 1
+    # negative / NaN eps
+    for eps in (-1.0, float("nan")):
+        ob = C._Osk(eps)
+        assert lib.cosa_osk_attention(ctypes.byref(s), ctypes.byref(ob), 16, 16, 16, 16, 16, 16, 4,
+                                      16, None, None, None, None) == 1
+    # k_cap out of range
+    assert lib.cosa_osk_attention(ctypes.byref(s), ctypes.byref(o), 16, 16, 16, 16, 16, 16, 0,
+                                  16, None, None, None, None) == 1
+    # misaligned tensor pointer
+    assert lib.cosa_dense_attention(ctypes.byref(s), 18, 16, 16, 16, 16, None, None) == 1
+    # workspace missing / too small / misaligned
+    assert lib.cosa_kap_select(ctypes.byref(s), ctypes.byref(k), 16, 16, 16, 16, 16, None, None,
+                               None, 0, None) == 5
+    assert lib.cosa_kap_select(ctypes.byref(s), ctypes.byref(k), 16, 16, 16, 16, 16, None, None,
+                               256, 100, None) == 5
+    assert lib.cosa_kap_select(ctypes.byref(s), ctypes.byref(k), 16, 16, 16, 16, 16, None, None,
+                               16, 1 << 40, None) == 5
+    # null shape
+    assert lib.cosa_dense_attention(None, 16, 16, 16, 16, 16, None, None) == 1
