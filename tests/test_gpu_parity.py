@@ -239,35 +239,56 @@ def test_osk_full_budget_no_skip_equals_dense_and_is_order_invariant():
 
 
 def test_osk_never_reads_unlisted_pages():
-    """Pages no q-block lists, and physical pages no page-table entry names,
-    are filled with NaN: the output must not change by a single bit."""
+    """Lists are built host-side from a seeded generator: forced pages plus
+    random even pages.  Pages no list names, and physical pages no page-table
+    entry names, are filled with NaN: the output must not change by a bit."""
     wl = W.small_workload("gqa-32k", 4096, 4, 1, shuffle_pages=True)
     x = W.make_inputs(wl, seed=8)
     xd = to_dev(x)
-    B, nP = 1, wl.num_pages
+    B, nP, nQB, Hq = 1, wl.num_pages, wl.num_q_blocks, 4
     extra = 5
-    kp = torch.cat([xd["k_pool"], torch.full((extra,) + tuple(xd["k_pool"].shape[1:]), float("nan"),
-                                             dtype=torch.bfloat16, device="cuda")])
-    vp = torch.cat([xd["v_pool"], torch.full((extra,) + tuple(xd["v_pool"].shape[1:]), float("nan"),
-                                             dtype=torch.bfloat16, device="cuda")])
+    nanpad = lambda t: torch.cat([t, torch.full((extra,) + tuple(t.shape[1:]), float("nan"),
+                                                dtype=t.dtype, device=t.device)])
+    kp, vp = nanpad(xd["k_pool"]), nanpad(xd["v_pool"])
     pt = torch.full((B, nP + 3), -1, dtype=torch.int32, device="cuda")   # stride > nP
     pt[:, :nP] = xd["page_table"]
-    xd2 = dict(xd, k_pool=kp, v_pool=vp, page_table=pt)
-    shape = C.Shape(1, 4, 1, 4096, 128, 64, 128, pages_per_seq=nP + 3, num_phys_pages=B * nP + extra)
-    order, count, _, _ = gpu_kap(shape, C.KapParams(budget=0.1, q_sub=32), xd2, export=False)
-    out_a, lse_a, _, _ = gpu_osk(shape, 1e-4, xd2, order, count)
+    shape = C.Shape(1, 4, 1, 4096, 128, 64, 128, pages_per_seq=nP + 3,
+                    num_phys_pages=B * nP + extra)
+    g = np.random.default_rng(8)
+    kc = O.causal_pages(nQB - 1, 128, 64)
+    o = np.full((B, Hq, nQB, kc), -1, dtype=np.int32)
+    c = np.zeros((B, Hq, nQB), dtype=np.int32)
     listed = set()
-    o, c = order.cpu().numpy(), count.cpu().numpy()
-    for idx in np.ndindex(*c.shape):
-        listed.update(o[idx][:c[idx]].tolist())
+    for h in range(Hq):
+        for qb in range(nQB):
+            n_b = O.causal_pages(qb, 128, 64)
+            forced = O.forced_pages(qb, 128, 64, 1)
+            evens = [p for p in range(2, n_b, 2) if p not in forced]
+            pick = [int(p) for p in g.permutation(evens)[:max(0, len(evens) // 3)]]
+            lst = [int(p) for p in g.permutation(forced + pick)]
+            o[0, h, qb, :len(lst)] = lst
+            c[0, h, qb] = len(lst)
+            listed.update(lst)
+    order, count = torch.from_numpy(o).cuda(), torch.from_numpy(c).cuda()
+    xd2 = dict(xd, k_pool=kp, v_pool=vp, page_table=pt)
+    out_a, lse_a, _, _ = gpu_osk(shape, 1e-4, xd2, order, count)
     unlisted = [p for p in range(nP) if p not in listed]
-    assert unlisted, "budget too large for this check"
+    assert len(unlisted) > nP // 4
     phys = pt[0, torch.tensor(unlisted, device="cuda")].long()
     kp2, vp2 = kp.clone(), vp.clone()
     kp2[phys] = float("nan")
     vp2[phys] = float("nan")
     out_b, lse_b, _, _ = gpu_osk(shape, 1e-4, dict(xd2, k_pool=kp2, v_pool=vp2), order, count)
+    assert torch.isfinite(out_a.float()).all()
     assert torch.equal(out_a, out_b) and torch.equal(lse_a, lse_b)
+    # and the OSK result on these lists matches the oracle on them
+    oa = _oracle_args(wl, x)
+    ref = O.osk_attention(oa["q"], oa["k_pool"], oa["v_pool"], oa["page_table"], o, c,
+                          num_kv_heads=1, page_size=64, q_block=128, eps=1e-4,
+                          scale=1 / math.sqrt(128))
+    amb = np.abs(ref["margin"]) <= SKIP_MARGIN
+    if not amb.any():
+        assert_out_close(np64(out_a), ref["out"], "osk on host-built lists")
 
 
 def test_osk_infinite_eps_with_page0_first():
@@ -300,8 +321,8 @@ def test_osk_infinite_eps_with_page0_first():
 @pytest.mark.parametrize("case", ["tiny-2k", "gqa-4k", "wide-head-4k-p128", "gqa-2k-bq64",
                                   "single-qblock", "single-page"])
 def test_dense_parity(case):
-    extra = {"single-qblock": W.small_workload("gqa-32k", 128, 2, 1),
-             "single-page": W.small_workload("gqa-32k", 64, 2, 1, q_block=64)}
+    extra = {"single-qblock": W.small_workload("gqa-32k", 128, 2, 1, planted_frac=0.0),
+             "single-page": W.small_workload("gqa-32k", 64, 2, 1, q_block=64, planted_frac=0.0)}
     wl = extra[case] if case in extra else OSK_CASES[case][0]
     x = W.make_inputs(wl, seed=10)
     xd = to_dev(x)

@@ -171,10 +171,10 @@ def make_inputs(wl: Workload, seed: int = 0, device: str = "cpu",
         if wl.planted_queries == "last256":
             last_tok = N - 256
             hi = last_tok // P          # pages overlapping the last 256 tokens are excluded
-            cand = torch.arange(1, hi)
-            q_rows = slice(N - 256, N)
+            cand = torch.arange(1, max(1, hi))
+            q_rows = slice(max(0, N - 256), N)
         else:
-            cand = torch.arange(1, nP - 1)  # neither page 0 nor the last page
+            cand = torch.arange(1, max(1, nP - 1))  # neither page 0 nor the last page
             q_rows = slice(0, N)
         if cand.numel() < n_pl:
             raise ValueError("not enough candidate pages to plant")
