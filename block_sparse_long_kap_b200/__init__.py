@@ -17,8 +17,8 @@ from typing import Optional
 __all__ = [
     "CosaError", "Shape", "KapParams", "OskParams", "lib", "library_path",
     "cosa_status_string", "cosa_version", "cosa_kap_kcap", "cosa_kap_workspace_size",
-    "cosa_kap_select", "cosa_kap_order", "cosa_osk_attention", "cosa_dense_attention",
-    "cosa_get_status", "EXPORTED_SYMBOLS",
+    "cosa_kap_select", "cosa_kap_select_noalloc", "cosa_kap_order", "cosa_osk_attention",
+    "cosa_dense_attention", "cosa_get_status", "EXPORTED_SYMBOLS", "NOALLOC_SCRATCH_BYTES",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -26,9 +26,12 @@ library_path = os.path.join(_HERE, "libcosa.so")
 
 EXPORTED_SYMBOLS = (
     "cosa_status_string", "cosa_version", "cosa_kap_kcap", "cosa_kap_workspace_size",
-    "cosa_kap_select", "cosa_kap_order", "cosa_osk_attention", "cosa_dense_attention",
-    "cosa_get_status",
+    "cosa_kap_select", "cosa_kap_select_noalloc", "cosa_kap_order", "cosa_osk_attention",
+    "cosa_dense_attention", "cosa_get_status",
 )
+
+# Largest workspace the allocation-free Stage-1 entry point accepts (cosa.h).
+NOALLOC_SCRATCH_BYTES = 64 << 20
 
 STATUS_NAMES = {0: "COSA_OK", 1: "COSA_ERR_INVALID_ARG", 2: "COSA_ERR_UNSUPPORTED",
                 3: "COSA_ERR_CUDA", 4: "COSA_ERR_TIMEOUT", 5: "COSA_ERR_WORKSPACE"}
@@ -133,6 +136,7 @@ def lib():
     L.cosa_kap_kcap.argtypes = [P(_Shape), P(_Kap), P(i32)]
     L.cosa_kap_workspace_size.argtypes = [P(_Shape), P(_Kap), P(sz)]
     L.cosa_kap_select.argtypes = [P(_Shape), P(_Kap), vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+    L.cosa_kap_select_noalloc.argtypes = [P(_Shape), P(_Kap), vp, vp, vp, vp, vp, vp, vp, vp]
     L.cosa_kap_order.argtypes = [P(_Shape), P(_Kap), vp, vp, vp, vp, vp]
     L.cosa_osk_attention.argtypes = [P(_Shape), P(_Osk), vp, vp, vp, vp, vp, vp, i32, vp, vp, vp,
                                      vp, vp]
@@ -226,6 +230,30 @@ def cosa_kap_select(shape: Shape, kap: KapParams, q, k_pool, page_table, order, 
                                  _ptr(page_table), _ptr(order), _ptr(count), _ptr(scores),
                                  _ptr(hrm), _ptr(workspace), nbytes, _stream(stream)),
            "cosa_kap_select")
+
+
+def cosa_kap_select_noalloc(shape: Shape, kap: KapParams, q, k_pool, page_table, order, count,
+                            scores=None, hrm=None, stream=None) -> None:
+    """Stage 1 without a caller workspace: for callers that cannot allocate
+    device memory.  The library's fixed scratch array is used instead; shapes
+    whose workspace exceeds NOALLOC_SCRATCH_BYTES are rejected.  Calls that
+    overlap on the GPU share that array and race."""
+    import torch
+    s, k = shape.c(), kap.c(shape)
+    B, Hq, N, D = shape.batch, shape.num_q_heads, shape.seq_len, shape.head_dim
+    kc = cosa_kap_kcap(shape, kap)
+    _expect(q, "q", torch.bfloat16, (B, Hq, N, D))
+    _expect(k_pool, "k_pool", torch.bfloat16, _kv_shape(shape))
+    _expect(page_table, "page_table", torch.int32, (B, s.pages_per_seq))
+    _expect(order, "order", torch.int32, (B, Hq, shape.num_q_blocks, kc))
+    _expect(count, "count", torch.int32, (B, Hq, shape.num_q_blocks))
+    if scores is not None:
+        _expect(scores, "scores", torch.float32, (B, Hq, shape.num_q_blocks, shape.num_pages))
+    if hrm is not None:
+        _expect(hrm, "hrm", torch.uint8, (B, Hq, shape.num_q_blocks, shape.num_pages))
+    _check(lib().cosa_kap_select_noalloc(ctypes.byref(s), ctypes.byref(k), _ptr(q), _ptr(k_pool),
+                                         _ptr(page_table), _ptr(order), _ptr(count), _ptr(scores),
+                                         _ptr(hrm), _stream(stream)), "cosa_kap_select_noalloc")
 
 
 def cosa_kap_order(shape: Shape, kap: KapParams, scores, hrm, order, count, stream=None) -> None:

@@ -4,6 +4,7 @@
 #include <cmath>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 
 #include "common.cuh"
 #include "kap.cuh"
@@ -204,6 +205,38 @@ AttnParams make_params(const cosa_shape_t* s, const void* q, const void* k_pool,
   return p;
 }
 
+// ---------------------------------------------------------------------------
+// Scratch for cosa_kap_select_noalloc.  Some callers cannot allocate device
+// memory at call time (a runtime whose allocator is owned by someone else, a
+// pre-planned memory budget, code running where cudaMalloc is not allowed), so
+// this entry point uses a fixed array that lives in the library's module: it
+// is created on each device when the module loads there and stays until the
+// process exits.  Host code only sees a stand-in for it; its device address
+// is looked up once per device below.
+// ---------------------------------------------------------------------------
+static __device__ __align__(256) uint8_t g_kap_noalloc_scratch[COSA_KAP_NOALLOC_SCRATCH_BYTES];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mutex;
+void* g_noalloc_addr[kMaxDevices] = {};
+
+// Device address of the scratch array on the current device (looked up on the
+// first call for that device, with that device current).
+cosa_status_t noalloc_scratch_address(void** out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return COSA_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return COSA_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+  if (g_noalloc_addr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_kap_noalloc_scratch) != cudaSuccess || p == nullptr)
+      return COSA_ERR_CUDA;
+    g_noalloc_addr[dev] = p;
+  }
+  *out = g_noalloc_addr[dev];
+  return COSA_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -258,6 +291,30 @@ cosa_status_t cosa_kap_select(const cosa_shape_t* shape, const cosa_kap_params_t
   const int k_cap = kcap_of(shape, kap);
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   uint8_t* ws = reinterpret_cast<uint8_t*>(workspace);
+  if (shape->head_dim == 128)
+    return launch_kap<128>(shape, kap, q, k_pool, page_table, order, count, scores, hrm, L, ws,
+                           k_cap, st);
+  return launch_kap<64>(shape, kap, q, k_pool, page_table, order, count, scores, hrm, L, ws, k_cap,
+                        st);
+}
+
+cosa_status_t cosa_kap_select_noalloc(const cosa_shape_t* shape, const cosa_kap_params_t* kap,
+                                      const void* q, const void* k_pool,
+                                      const int32_t* page_table, int32_t* order, int32_t* count,
+                                      float* scores, uint8_t* hrm, cosa_stream_t stream) {
+  cosa_status_t e = check_shape(shape);
+  if (e != COSA_OK) return e;
+  if ((e = check_kap(shape, kap)) != COSA_OK) return e;
+  if (!q || !k_pool || !page_table || !order || !count) return COSA_ERR_INVALID_ARG;
+  KapLayout L = kap_layout(shape, kap);
+  if (L.total > (size_t)COSA_KAP_NOALLOC_SCRATCH_BYTES) return COSA_ERR_UNSUPPORTED;
+  if (reinterpret_cast<uintptr_t>(q) % 16 || reinterpret_cast<uintptr_t>(k_pool) % 16)
+    return COSA_ERR_INVALID_ARG;
+  void* scratch = nullptr;
+  if ((e = noalloc_scratch_address(&scratch)) != COSA_OK) return e;
+  const int k_cap = kcap_of(shape, kap);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* ws = reinterpret_cast<uint8_t*>(scratch);
   if (shape->head_dim == 128)
     return launch_kap<128>(shape, kap, q, k_pool, page_table, order, count, scores, hrm, L, ws,
                            k_cap, st);

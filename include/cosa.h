@@ -136,6 +136,33 @@ cosa_status_t cosa_kap_select(const cosa_shape_t* shape, const cosa_kap_params_t
                               int32_t* order, int32_t* count, float* scores, uint8_t* hrm,
                               void* workspace, size_t workspace_bytes, cosa_stream_t stream);
 
+/* Largest workspace (cosa_kap_workspace_size) that cosa_kap_select_noalloc
+ * accepts: 64 MiB, enough for a 32K-token layer with 32 query heads. */
+#define COSA_KAP_NOALLOC_SCRATCH_BYTES (64u << 20)
+
+/* cosa_kap_select for callers that cannot allocate device memory.  The paper
+ * has no counterpart: this is a packaging variant of the same Stage-1 kernels.
+ * Some callers cannot call cudaMalloc or hand out a workspace at call time (a
+ * runtime that owns the device allocator, a plan whose memory is fixed in
+ * advance), so the pooled vectors, scores and flags go to a fixed 64 MiB array
+ * inside the library instead.  Every GPU on which the library's kernels load
+ * holds that array until the process exits.  Arguments and results are those
+ * of cosa_kap_select without the workspace; the caller still allocates q,
+ * k_pool, page_table, order, count and the optional scores / hrm.
+ *   - Shapes whose cosa_kap_workspace_size exceeds COSA_KAP_NOALLOC_SCRATCH_BYTES
+ *     return COSA_ERR_UNSUPPORTED before anything is launched.
+ *   - The first call on a device looks up the array's device address (with that
+ *     device current); make that first call before any stream capture.
+ *   - Allocates nothing: no cudaMalloc, no cudaFree, no allocating library call.
+ *   - All calls on a device share the one array, and it keeps the last call's
+ *     contents (every kernel writes what it later reads, so nothing needs
+ *     clearing).  Calls whose execution overlaps on the GPU (different streams,
+ *     or different host threads on the same device) race on it: serialise them. */
+cosa_status_t cosa_kap_select_noalloc(const cosa_shape_t* shape, const cosa_kap_params_t* kap,
+                                      const void* q, const void* k_pool,
+                                      const int32_t* page_table, int32_t* order, int32_t* count,
+                                      float* scores, uint8_t* hrm, cosa_stream_t stream);
+
 /* Stage 1, selection and ordering only (gist.science/pt §2.2 "Ordenação por
  * Grupo de Flags"), from caller-given scores (fp32, >= 0) and HRM flags laid out
  * as above; entries past each q-block's causal pages are ignored.  Given the
