@@ -6,9 +6,11 @@
 #include <cstring>
 #include <mutex>
 
+#include <cudaTypedefs.h>
+
 #include "common.cuh"
 #include "kap.cuh"
-#include "attn_mma.cuh"
+#include "attn_tc.cuh"
 
 using namespace cosa;
 
@@ -47,6 +49,13 @@ cosa_status_t check_kap(const cosa_shape_t* s, const cosa_kap_params_t* k) {
   return COSA_OK;
 }
 
+// Row length of the transposed pooled-key array khatT[b][h_kv][d][.]: the
+// number of sub-keys nP * T rounded up to a multiple of 4 (16-byte rows).
+size_t khat_stride(const cosa_shape_t* s, const cosa_kap_params_t* k) {
+  size_t n = (size_t)(s->seq_len / s->page_size) * (s->page_size / k->k_sub);
+  return (n + 3) & ~size_t(3);
+}
+
 struct KapLayout {
   size_t qhat_off, khat_off, scores_off, hrm_off, total;
 };
@@ -62,7 +71,7 @@ KapLayout kap_layout(const cosa_shape_t* s, const cosa_kap_params_t* k) {
   L.qhat_off = off;
   off = align256(off + B * Hq * (N / k->q_sub) * D * sizeof(float));
   L.khat_off = off;
-  off = align256(off + B * Hk * (N / k->k_sub) * D * sizeof(float));
+  off = align256(off + B * Hk * D * khat_stride(s, k) * sizeof(float));
   L.scores_off = off;
   off = align256(off + B * Hq * nQB * nP * sizeof(float));
   L.hrm_off = off;
@@ -89,13 +98,27 @@ cosa_status_t last_launch() {
   return COSA_OK;
 }
 
-// Score kernel: heads per CTA = largest divisor of G whose representatives and
-// score rows fit the shared-memory budget.
+// Score kernel: heads per CTA = largest divisor of G whose representatives
+// (at most 32) and score rows fit the shared-memory budget.
 constexpr size_t kScoreSmemLimit = 200 * 1024;
 
 template <int D>
 size_t score_smem(int hpc, int R, int nP) {
-  return (size_t)SCORE_MAXNR * 4 * (D / 4 + 4) * sizeof(float) + (size_t)hpc * R * nP * sizeof(float);
+  const int nrmax = hpc * R <= 16 ? 16 : 32;
+  return (size_t)D * nrmax * sizeof(float) + (size_t)hpc * R * nP * sizeof(float);
+}
+
+template <int D, int NRMAX>
+cosa_status_t launch_score(dim3 grid, size_t smem, cudaStream_t st, const float* qhat,
+                           const float* khatT, float* sc, uint8_t* hr, int Hq, int Hk, int G,
+                           int hpc, int nQB, int nP, int kstride, int R, int T, int q_sub,
+                           int k_sub, int P, int Bq, float scale) {
+  if (cudaFuncSetAttribute(kap_score_kernel<D, NRMAX>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)smem) != cudaSuccess)
+    return COSA_ERR_CUDA;
+  kap_score_kernel<D, NRMAX><<<grid, SCORE_THREADS, smem, st>>>(
+      qhat, khatT, sc, hr, Hq, Hk, G, hpc, nQB, nP, kstride, R, T, q_sub, k_sub, P, Bq, scale);
+  return last_launch();
 }
 
 template <int D>
@@ -119,28 +142,30 @@ cosa_status_t launch_kap(const cosa_shape_t* s, const cosa_kap_params_t* k, cons
   if (blocks > 0x7fffffffll) return COSA_ERR_UNSUPPORTED;
   kap_pool_kernel<D><<<(unsigned)blocks, 256, 0, st>>>(
       reinterpret_cast<const __nv_bfloat16*>(q), reinterpret_cast<const __nv_bfloat16*>(k_pool),
-      page_table, qhat, khat, n_qvec, k->q_sub, n_kvec, k->k_sub, Hk, P, nP, s->pages_per_seq, T);
+      page_table, qhat, khat, n_qvec, k->q_sub, n_kvec, k->k_sub, Hk, P, nP, s->pages_per_seq, T,
+      (int)khat_stride(s, k));
   if (last_launch() != COSA_OK) return COSA_ERR_CUDA;
 
   // K2
   int hpc = 0;
   for (int d = G; d >= 1; --d) {
     if (G % d) continue;
-    if (d * R > SCORE_MAXNR) continue;
+    if (d * R > 32) continue;
     if (score_smem<D>(d, R, nP) > kScoreSmemLimit) continue;
     hpc = d;
     break;
   }
   if (hpc == 0) return COSA_ERR_UNSUPPORTED;
-  size_t smem2 = score_smem<D>(hpc, R, nP);
-  if (cudaFuncSetAttribute(kap_score_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)smem2) != cudaSuccess)
-    return COSA_ERR_CUDA;
-  dim3 g2(nQB, B * Hk * (G / hpc));
-  kap_score_kernel<D><<<g2, SCORE_THREADS, smem2, st>>>(qhat, khat, sc, hr, Hq, Hk, G, hpc, nQB,
-                                                       nP, R, T, k->q_sub, k->k_sub, P, Bq,
-                                                       s->softmax_scale);
-  if (last_launch() != COSA_OK) return COSA_ERR_CUDA;
+  const size_t smem2 = score_smem<D>(hpc, R, nP);
+  const dim3 g2(nQB, B * Hk * (G / hpc));
+  const int kstride = (int)khat_stride(s, k);
+  cosa_status_t e2 =
+      hpc * R <= 16
+          ? launch_score<D, 16>(g2, smem2, st, qhat, khat, sc, hr, Hq, Hk, G, hpc, nQB, nP, kstride,
+                                R, T, k->q_sub, k->k_sub, P, Bq, s->softmax_scale)
+          : launch_score<D, 32>(g2, smem2, st, qhat, khat, sc, hr, Hq, Hk, G, hpc, nQB, nP, kstride,
+                                R, T, k->q_sub, k->k_sub, P, Bq, s->softmax_scale);
+  if (e2 != COSA_OK) return e2;
 
   // K3
   int npow2 = 1;
@@ -156,41 +181,70 @@ cosa_status_t launch_kap(const cosa_shape_t* s, const cosa_kap_params_t* k, cons
   return last_launch();
 }
 
-template <int D, int P, int BQ, bool DENSE>
-cosa_status_t launch_attn_t(const AttnParams& prm, int grid, cudaStream_t st) {
-  const size_t smem = (size_t)(BQ * D + 4 * P * D) * sizeof(__nv_bfloat16);
-  auto kern = attn_mma_kernel<D, P, BQ, DENSE>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
-      cudaSuccess)
+// ---- tensor maps (TMA descriptors) ------------------------------------------------
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// bf16 [z][rows][D] viewed as a 3-D tensor; box = 64 columns x box_rows x 1,
+// 128-byte swizzle (the layout the UMMA descriptors expect).
+bool make_map(CUtensorMap* m, const void* base, int D, int rows, long long z, int box_rows) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)rows, (cuuint64_t)z};
+  cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)rows * D * 2};
+  cuuint32_t box[3] = {64u, (cuuint32_t)box_rows, 1u};
+  cuuint32_t estr[3] = {1u, 1u, 1u};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
+                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+constexpr unsigned long long kWaitTimeoutNs = 1000000000ull;  // 1 s without progress
+
+template <int D, int P, bool DENSE>
+cosa_status_t launch_tc_t(const cosa_shape_t* s, const TcParams& prm, const void* q,
+                          const void* k_pool, const void* v_pool, int grid, cudaStream_t st) {
+  using Cfg = TcCfg<D, P>;
+  CUtensorMap mq, mk, mv;
+  const long long BH = (long long)s->batch * s->num_q_heads;
+  const long long PZ = (long long)s->num_phys_pages * s->num_kv_heads;
+  if (!make_map(&mq, q, D, s->seq_len, BH, s->q_block) ||
+      !make_map(&mk, k_pool, D, P, PZ, P) || !make_map(&mv, v_pool, D, P, PZ, P))
     return COSA_ERR_CUDA;
-  kern<<<grid, BQ * 2, smem, st>>>(prm);
+  auto kern = attn_tc_kernel<D, P, DENSE>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)Cfg::SMEM_ALLOC) != cudaSuccess)
+    return COSA_ERR_CUDA;
+  kern<<<grid, 256, Cfg::SMEM_ALLOC, st>>>(mq, mk, mv, prm);
   return last_launch();
 }
 
 template <bool DENSE>
-cosa_status_t launch_attn(const cosa_shape_t* s, const AttnParams& prm, int grid, cudaStream_t st) {
-  const int D = s->head_dim, P = s->page_size, BQ = s->q_block;
-#define COSA_ATTN_CASE(d, p, bq) \
-  if (D == d && P == p && BQ == bq) return launch_attn_t<d, p, bq, DENSE>(prm, grid, st);
-  COSA_ATTN_CASE(128, 64, 128)
-  COSA_ATTN_CASE(128, 128, 128)
-  COSA_ATTN_CASE(128, 64, 64)
-  COSA_ATTN_CASE(128, 128, 64)
-  COSA_ATTN_CASE(64, 64, 128)
-  COSA_ATTN_CASE(64, 128, 128)
-  COSA_ATTN_CASE(64, 64, 64)
-  COSA_ATTN_CASE(64, 128, 64)
-#undef COSA_ATTN_CASE
+cosa_status_t launch_attn(const cosa_shape_t* s, const TcParams& prm, const void* q,
+                          const void* k_pool, const void* v_pool, int grid, cudaStream_t st) {
+  const int D = s->head_dim, P = s->page_size;
+  if (D == 128 && P == 64) return launch_tc_t<128, 64, DENSE>(s, prm, q, k_pool, v_pool, grid, st);
+  if (D == 128 && P == 128) return launch_tc_t<128, 128, DENSE>(s, prm, q, k_pool, v_pool, grid, st);
+  if (D == 64 && P == 64) return launch_tc_t<64, 64, DENSE>(s, prm, q, k_pool, v_pool, grid, st);
+  if (D == 64 && P == 128) return launch_tc_t<64, 128, DENSE>(s, prm, q, k_pool, v_pool, grid, st);
   return COSA_ERR_UNSUPPORTED;
 }
 
-AttnParams make_params(const cosa_shape_t* s, const void* q, const void* k_pool,
-                       const void* v_pool, const int32_t* page_table, void* out, float* lse) {
-  AttnParams p;
+TcParams make_params(const cosa_shape_t* s, void* out, float* lse, const int32_t* page_table) {
+  TcParams p;
   std::memset(&p, 0, sizeof(p));
-  p.q = reinterpret_cast<const __nv_bfloat16*>(q);
-  p.k_pool = reinterpret_cast<const __nv_bfloat16*>(k_pool);
-  p.v_pool = reinterpret_cast<const __nv_bfloat16*>(v_pool);
   p.page_table = page_table;
   p.out = reinterpret_cast<__nv_bfloat16*>(out);
   p.lse = lse;
@@ -200,8 +254,10 @@ AttnParams make_params(const cosa_shape_t* s, const void* q, const void* k_pool,
   p.seq_len = s->seq_len;
   p.num_q_blocks = s->seq_len / s->q_block;
   p.pages_per_seq = s->pages_per_seq;
+  p.q_block = s->q_block;
   p.scale_log2 = s->softmax_scale * 1.4426950408889634f;
   p.log2_eps = -INFINITY;
+  p.timeout_ns = kWaitTimeoutNs;
   return p;
 }
 
@@ -360,7 +416,7 @@ cosa_status_t cosa_osk_attention(const cosa_shape_t* shape, const cosa_osk_param
   if (reinterpret_cast<uintptr_t>(q) % 16 || reinterpret_cast<uintptr_t>(k_pool) % 16 ||
       reinterpret_cast<uintptr_t>(v_pool) % 16 || reinterpret_cast<uintptr_t>(out) % 16)
     return COSA_ERR_INVALID_ARG;
-  AttnParams p = make_params(shape, q, k_pool, v_pool, page_table, out, lse);
+  TcParams p = make_params(shape, out, lse, page_table);
   p.order = order;
   p.count = count;
   p.computed = computed;
@@ -369,7 +425,8 @@ cosa_status_t cosa_osk_attention(const cosa_shape_t* shape, const cosa_osk_param
   p.log2_eps = osk->eps > 0.f ? log2f(osk->eps) : -INFINITY;
   const long long grid = (long long)shape->batch * shape->num_q_heads * (shape->seq_len / shape->q_block);
   if (grid > 0x7fffffffll) return COSA_ERR_UNSUPPORTED;
-  return launch_attn<false>(shape, p, (int)grid, reinterpret_cast<cudaStream_t>(stream));
+  return launch_attn<false>(shape, p, q, k_pool, v_pool, (int)grid,
+                            reinterpret_cast<cudaStream_t>(stream));
 }
 
 cosa_status_t cosa_dense_attention(const cosa_shape_t* shape, const void* q, const void* k_pool,
@@ -381,10 +438,11 @@ cosa_status_t cosa_dense_attention(const cosa_shape_t* shape, const void* q, con
   if (reinterpret_cast<uintptr_t>(q) % 16 || reinterpret_cast<uintptr_t>(k_pool) % 16 ||
       reinterpret_cast<uintptr_t>(v_pool) % 16 || reinterpret_cast<uintptr_t>(out) % 16)
     return COSA_ERR_INVALID_ARG;
-  AttnParams p = make_params(shape, q, k_pool, v_pool, page_table, out, lse);
+  TcParams p = make_params(shape, out, lse, page_table);
   const long long grid = (long long)shape->batch * shape->num_q_heads * (shape->seq_len / shape->q_block);
   if (grid > 0x7fffffffll) return COSA_ERR_UNSUPPORTED;
-  return launch_attn<true>(shape, p, (int)grid, reinterpret_cast<cudaStream_t>(stream));
+  return launch_attn<true>(shape, p, q, k_pool, v_pool, (int)grid,
+                           reinterpret_cast<cudaStream_t>(stream));
 }
 
 cosa_status_t cosa_get_status(cosa_stream_t stream) {

@@ -27,19 +27,21 @@ namespace cosa {
 template <int D>
 __global__ void __launch_bounds__(256) kap_pool_kernel(
     const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k_pool,
-    const int32_t* __restrict__ page_table, float* __restrict__ qhat, float* __restrict__ khat,
+    const int32_t* __restrict__ page_table, float* __restrict__ qhat, float* __restrict__ khatT,
     long long n_qvec, int q_sub, long long n_kvec, int k_sub, int num_kv_heads, int page_size,
-    int num_pages, int pages_per_seq, int T) {
+    int num_pages, int pages_per_seq, int T, int khat_stride) {
   constexpr int LPR = D / 8;   // lanes per row: each lane loads 8 bf16 (16 B)
   constexpr int RPI = 32 / LPR;  // rows covered per warp-wide load
   const int lane = threadIdx.x & 31;
   const long long w = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const __nv_bfloat16* src;
   float* dst;
+  long long dst_stride;  // distance between consecutive d of the output vector
   int rows;
   if (w < n_qvec) {
     src = q + w * (long long)q_sub * D;
     dst = qhat + w * D;
+    dst_stride = 1;
     rows = q_sub;
   } else {
     long long kv = w - n_qvec;
@@ -52,7 +54,9 @@ __global__ void __launch_bounds__(256) kap_pool_kernel(
     int b = (int)(r / num_kv_heads);
     int phys = page_table[(long long)b * pages_per_seq + p];
     src = k_pool + (((long long)phys * num_kv_heads + hk) * page_size + (long long)t * k_sub) * D;
-    dst = khat + kv * D;
+    // transposed: khatT[b][hk][d][khat_stride], sub-key index p * T + t
+    dst = khatT + ((long long)(b * num_kv_heads + hk) * D) * khat_stride + (long long)p * T + t;
+    dst_stride = khat_stride;
     rows = k_sub;
   }
   const int c = lane % LPR;
@@ -77,37 +81,42 @@ __global__ void __launch_bounds__(256) kap_pool_kernel(
   }
   if (lane < LPR) {
     const float inv = 1.0f / (float)rows;  // rows is a power of two: exact
-    float4 o0 = make_float4(acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv);
-    float4 o1 = make_float4(acc[4] * inv, acc[5] * inv, acc[6] * inv, acc[7] * inv);
-    reinterpret_cast<float4*>(dst)[2 * c] = o0;
-    reinterpret_cast<float4*>(dst)[2 * c + 1] = o1;
+    if (dst_stride == 1) {
+      float4 o0 = make_float4(acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv);
+      float4 o1 = make_float4(acc[4] * inv, acc[5] * inv, acc[6] * inv, acc[7] * inv);
+      reinterpret_cast<float4*>(dst)[2 * c] = o0;
+      reinterpret_cast<float4*>(dst)[2 * c + 1] = o1;
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) dst[(long long)(c * 8 + i) * dst_stride] = acc[i] * inv;
+    }
   }
 }
 
 // ---------------------------------------------------------------------------
 // K2: scores, MaxPool, MaxNorm, HRM.
 // grid.x = nQB (heaviest q-block first), grid.y = B * H_kv * head_groups.
-// Threads are grouped in quads: one quad per sub-key, one lane per quarter of
-// the head dimension.  a[rep][page] lives in shared memory until the row
-// maxima are known.
+// The NR = hpc * R representatives of the CTA's heads sit in shared memory as
+// qT[d][rep]; each thread owns 4 consecutive sub-keys and computes their full
+// dot products with every representative (an NR x 4 register tile), reading
+// the pooled keys from the transposed layout khatT[d][sub-key] so that one
+// warp load is one contiguous 512-byte row.  a[rep][page] stays in shared
+// memory until the row maxima are known.
 // ---------------------------------------------------------------------------
-constexpr int SCORE_THREADS = 512;
-constexpr int SCORE_MAXNR = 32;
+constexpr int SCORE_THREADS = 256;
 
-template <int D>
+template <int D, int NRMAX>
 __global__ void __launch_bounds__(SCORE_THREADS) kap_score_kernel(
-    const float* __restrict__ qhat, const float* __restrict__ khat, float* __restrict__ scores,
+    const float* __restrict__ qhat, const float* __restrict__ khatT, float* __restrict__ scores,
     uint8_t* __restrict__ hrm_out, int num_q_heads, int num_kv_heads, int group, int hpc,
-    int num_q_blocks, int num_pages, int R, int T, int q_sub, int k_sub, int page_size,
-    int q_block, float scale) {
-  constexpr int DQ = D / 4;        // floats per quarter row
-  constexpr int QSTRIDE = DQ + 4;  // padded quarter (bank spread)
+    int num_q_blocks, int num_pages, int khat_stride, int R, int T, int q_sub, int k_sub,
+    int page_size, int q_block, float scale) {
   extern __shared__ float smem[];
   const int NR = hpc * R;
-  float* qs = smem;                                 // [NR][4][QSTRIDE]
-  float* a_s = qs + SCORE_MAXNR * 4 * QSTRIDE;      // [NR][num_pages]
-  __shared__ float m_s[SCORE_MAXNR];
-  __shared__ int arg_s[SCORE_MAXNR];
+  float* qT = smem;                   // [D][NRMAX]
+  float* a_s = qT + D * NRMAX;        // [NR][num_pages]
+  __shared__ float m_s[NRMAX];
+  __shared__ int arg_s[NRMAX];
 
   const int qb = num_q_blocks - 1 - blockIdx.x;
   const int head_groups = group / hpc;
@@ -118,56 +127,79 @@ __global__ void __launch_bounds__(SCORE_THREADS) kap_score_kernel(
   const int n_b = causal_pages(qb, q_block, page_size);
   const int tid = threadIdx.x;
 
-  // representatives of the group's heads for this q-block
-  for (int i = tid; i < NR * D; i += blockDim.x) {
-    int rep = i / D, d = i % D;
-    int hh = rep / R, r = rep % R;
-    long long src = (((long long)(b * num_q_heads + h0 + hh) * num_q_blocks + qb) * R + r) * D + d;
-    qs[(rep * 4 + d / DQ) * QSTRIDE + d % DQ] = qhat[src];
+  for (int i = tid; i < NRMAX * D; i += blockDim.x) {
+    const int rep = i % NRMAX, d = i / NRMAX;
+    float v = 0.f;
+    if (rep < NR) {
+      const int hh = rep / R, r = rep % R;
+      v = qhat[(((long long)(b * num_q_heads + h0 + hh) * num_q_blocks + qb) * R + r) * D + d];
+    }
+    qT[d * NRMAX + rep] = v;
   }
   __syncthreads();
 
-  const int quad = tid >> 2, dq = tid & 3;
-  const int quads = blockDim.x >> 2;
-  const int ns = n_b * T;
-  const float* kbase = khat + ((long long)(b * num_kv_heads + hk) * num_pages * T) * D + dq * DQ;
-  const int grp = 4 * T;  // lanes holding one page
-  for (int base = 0; base < ns; base += quads) {
-    const int s = base + quad;
-    const bool valid = s < ns;
-    float acc[SCORE_MAXNR];
+  const int ns = n_b * T;             // causal sub-keys
+  const int nq = (ns + 3) >> 2;       // quads of sub-keys
+  const float* kb = khatT + (long long)(b * num_kv_heads + hk) * D * khat_stride;
+  for (int base = 0; base < nq; base += blockDim.x) {
+    const int qd = base + tid;
+    const bool valid = qd < nq;
+    const int s0 = qd * 4;
+    float acc[NRMAX][4];
 #pragma unroll
-    for (int r = 0; r < SCORE_MAXNR; ++r) acc[r] = 0.f;
+    for (int r = 0; r < NRMAX; ++r) acc[r][0] = acc[r][1] = acc[r][2] = acc[r][3] = 0.f;
     if (valid) {
-      const float4* kp = reinterpret_cast<const float4*>(kbase + (long long)s * D);
+      const float* kp = kb + s0;
+#pragma unroll 8
+      for (int d = 0; d < D; ++d) {
+        const float4 kv = __ldg(reinterpret_cast<const float4*>(kp + (long long)d * khat_stride));
+        const float* qrow = qT + d * NRMAX;
 #pragma unroll
-      for (int i = 0; i < DQ / 4; ++i) {
-        float4 kv = __ldg(kp + i);
+        for (int r4 = 0; r4 < NRMAX / 4; ++r4) {
+          if (r4 * 4 < NR) {
+            const float4 qv = *reinterpret_cast<const float4*>(qrow + r4 * 4);
+            const float qq[4] = {qv.x, qv.y, qv.z, qv.w};
 #pragma unroll
-        for (int r = 0; r < SCORE_MAXNR; ++r) {
-          if (r < NR) {
-            float4 qv = *reinterpret_cast<const float4*>(qs + (r * 4 + dq) * QSTRIDE + 4 * i);
-            acc[r] = fmaf(qv.x, kv.x, acc[r]);
-            acc[r] = fmaf(qv.y, kv.y, acc[r]);
-            acc[r] = fmaf(qv.z, kv.z, acc[r]);
-            acc[r] = fmaf(qv.w, kv.w, acc[r]);
+            for (int e = 0; e < 4; ++e) {
+              acc[r4 * 4 + e][0] = fmaf(qq[e], kv.x, acc[r4 * 4 + e][0]);
+              acc[r4 * 4 + e][1] = fmaf(qq[e], kv.y, acc[r4 * 4 + e][1]);
+              acc[r4 * 4 + e][2] = fmaf(qq[e], kv.z, acc[r4 * 4 + e][2]);
+              acc[r4 * 4 + e][3] = fmaf(qq[e], kv.w, acc[r4 * 4 + e][3]);
+            }
           }
         }
       }
     }
-    const int p = s / T, t = s % T;
-    const int first_tok = p * page_size + t * k_sub;
-    const int gi = (tid & 31) % grp;
+    // causal visibility per (rep, sub-key), then MaxPool over each page's sub-keys
+    int first_tok[4], page_of[4];
+    bool in_range[4];
 #pragma unroll
-    for (int r = 0; r < SCORE_MAXNR; ++r) {
-      if (r < NR) {  // NR is uniform across the block
-        float v = acc[r];
-        v += __shfl_xor_sync(0xffffffffu, v, 1);
-        v += __shfl_xor_sync(0xffffffffu, v, 2);
+    for (int u = 0; u < 4; ++u) {
+      const int sidx = s0 + u;
+      page_of[u] = sidx / T;
+      first_tok[u] = page_of[u] * page_size + (sidx % T) * k_sub;
+      in_range[u] = valid && sidx < ns;
+    }
+#pragma unroll
+    for (int r = 0; r < NRMAX; ++r) {
+      if (r < NR) {
         const int rep_last = qb * q_block + ((r % R) + 1) * q_sub - 1;
-        v = (valid && first_tok <= rep_last) ? v * scale : -INFINITY;
-        for (int off = 4; off < grp; off <<= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, off));
-        if (valid && (r % grp) == gi) a_s[r * num_pages + p] = v;
+        float v[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+          v[u] = (in_range[u] && first_tok[u] <= rep_last) ? acc[r][u] * scale : -INFINITY;
+        if (T >= 4) {  // all four sub-keys belong to one page
+          float m = fmaxf(fmaxf(v[0], v[1]), fmaxf(v[2], v[3]));
+          if (T == 8) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
+          if (valid && (T == 4 || (qd & 1) == 0)) a_s[r * num_pages + page_of[0]] = m;
+        } else if (T == 2) {
+          if (in_range[0]) a_s[r * num_pages + page_of[0]] = fmaxf(v[0], v[1]);
+          if (in_range[2]) a_s[r * num_pages + page_of[2]] = fmaxf(v[2], v[3]);
+        } else {
+#pragma unroll
+          for (int u = 0; u < 4; ++u)
+            if (in_range[u]) a_s[r * num_pages + page_of[u]] = v[u];
+        }
       }
     }
   }

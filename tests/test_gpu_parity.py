@@ -239,9 +239,11 @@ def test_osk_full_budget_no_skip_equals_dense_and_is_order_invariant():
 
 
 def test_osk_never_reads_unlisted_pages():
-    """Lists are built host-side from a seeded generator: forced pages plus
-    random even pages.  Pages no list names, and physical pages no page-table
-    entry names, are filled with NaN: the output must not change by a bit."""
+    """Lists are built host-side from a seeded generator: the forced pages plus
+    random odd pages.  The even pages 2..18 are then filled with NaN, as are
+    physical pages no page-table entry names.  A q-block from 10 on lists none
+    of them (its own pages are 2qb, 2qb+1 >= 20), so its output must not change
+    by a single bit; earlier q-blocks own a poisoned page and are not checked."""
     wl = W.small_workload("gqa-32k", 4096, 4, 1, shuffle_pages=True)
     x = W.make_inputs(wl, seed=8)
     xd = to_dev(x)
@@ -258,35 +260,35 @@ def test_osk_never_reads_unlisted_pages():
     kc = O.causal_pages(nQB - 1, 128, 64)
     o = np.full((B, Hq, nQB, kc), -1, dtype=np.int32)
     c = np.zeros((B, Hq, nQB), dtype=np.int32)
-    listed = set()
     for h in range(Hq):
         for qb in range(nQB):
             n_b = O.causal_pages(qb, 128, 64)
             forced = O.forced_pages(qb, 128, 64, 1)
-            evens = [p for p in range(2, n_b, 2) if p not in forced]
-            pick = [int(p) for p in g.permutation(evens)[:max(0, len(evens) // 3)]]
+            odds = [p for p in range(1, n_b, 2) if p not in forced]
+            pick = [int(p) for p in g.permutation(odds)[:len(odds) // 2]]
             lst = [int(p) for p in g.permutation(forced + pick)]
             o[0, h, qb, :len(lst)] = lst
             c[0, h, qb] = len(lst)
-            listed.update(lst)
     order, count = torch.from_numpy(o).cuda(), torch.from_numpy(c).cuda()
     xd2 = dict(xd, k_pool=kp, v_pool=vp, page_table=pt)
     out_a, lse_a, _, _ = gpu_osk(shape, 1e-4, xd2, order, count)
-    unlisted = [p for p in range(nP) if p not in listed]
-    assert len(unlisted) > nP // 4
-    phys = pt[0, torch.tensor(unlisted, device="cuda")].long()
+    poisoned = list(range(2, 20, 2))
+    phys = pt[0, torch.tensor(poisoned, device="cuda")].long()
     kp2, vp2 = kp.clone(), vp.clone()
     kp2[phys] = float("nan")
     vp2[phys] = float("nan")
     out_b, lse_b, _, _ = gpu_osk(shape, 1e-4, dict(xd2, k_pool=kp2, v_pool=vp2), order, count)
+    r0 = 10 * 128
     assert torch.isfinite(out_a.float()).all()
-    assert torch.equal(out_a, out_b) and torch.equal(lse_a, lse_b)
+    assert torch.equal(out_a[:, :, r0:], out_b[:, :, r0:])
+    assert torch.equal(lse_a[:, :, r0:], lse_b[:, :, r0:])
+    assert not torch.isfinite(out_b[:, :, :r0].float()).all()   # the poison is really read there
     # and the OSK result on these lists matches the oracle on them
     oa = _oracle_args(wl, x)
     ref = O.osk_attention(oa["q"], oa["k_pool"], oa["v_pool"], oa["page_table"], o, c,
                           num_kv_heads=1, page_size=64, q_block=128, eps=1e-4,
                           scale=1 / math.sqrt(128))
-    amb = np.abs(ref["margin"]) <= SKIP_MARGIN
+    amb = np.abs(np.nan_to_num(ref["margin"], nan=1.0)) <= SKIP_MARGIN
     if not amb.any():
         assert_out_close(np64(out_a), ref["out"], "osk on host-built lists")
 
