@@ -1,30 +1,41 @@
 // Ordered-Skipping Kernel (and dense causal attention) on the sm_100a tensor
 // cores: TMA page loads through the page table, tcgen05.mma into TMEM, one
-// softmax thread per query row.  (gist.science/pt "CoSA" technical summary,
+// query row per TMEM lane.  (gist.science/pt "CoSA" technical summary,
 // §2.3 "Estágio 2: OSK": mask-skipped pages are never loaded, "KV page
 // remapping"; in-kernel skip from the page's local max vs the running max;
 // computed pages get the full softmax + PV.)
 //
-// One CTA (256 threads) per (b, h_q, q-block) tile of up to 128 query rows:
-//   warp 0     TMA producer: the Q tile once, then K of every listed page, in
-//              list order, into a KS-stage ring (page table gives the
-//              physical page; no multicast).
-//   warp 1     MMA issuer (one thread): S_j = Q K_j^T into one of SB TMEM
-//              buffers; once page j is decided "computed" and its P and V
-//              tiles are ready, O += P_j V_j into the TMEM accumulator.  It
-//              polls both streams so that a late V never stalls QK^T.
-//   warp 2     TMA producer for V: loads V_j only for pages the vote keeps,
-//              so a skipped page costs its K tile and one QK^T, nothing more.
-//   warps 4-7  softmax, thread i <-> query row i <-> TMEM lane i: reads S_j,
-//              masks the causal diagonal, takes the row max, votes on the
-//              skip rule (any row with (page max - running max) >= log2 eps
-//              keeps the page; the first listed page is always kept), and for
-//              kept pages writes P = exp2(s - m_ref) as bf16 into a swizzled
-//              shared-memory tile.  m_ref, the exponent base, moves only when
-//              the running max passes it by more than 2^8 (then O and l are
-//              rescaled in TMEM), which keeps the result exact.
+// One CTA (384 threads) per (b, h_q, q-block) tile of up to 128 query rows:
+//   warp 0      TMA producer: the Q tile once, then K of every listed page, in
+//               list order, into a KS-stage ring (page table gives the
+//               physical page; no multicast).
+//   warp 1      QK^T issuer (one thread): S_j = Q K_j^T into one of SB TMEM
+//               buffers, in list order.
+//   warp 2      TMA producer for V: loads V_j only for pages the vote keeps,
+//               so a skipped page costs its K tile and one QK^T, nothing more.
+//   warp 3      PV issuer (one thread): for each kept page, once its P and V
+//               tiles are ready, O += P_j V_j into the TMEM accumulator.  With
+//               two issuing threads a late V never stalls QK^T.
+//   warps 4-11  softmax, two warpgroups: warpgroup h (0/1) owns columns
+//               [h P/2, (h+1) P/2) of every S tile and [h D/2, (h+1) D/2) of O;
+//               thread (warp % 4, lane) owns query row 32 (warp % 4) + lane,
+//               which is its TMEM lane.  Per page: read the half row of S,
+//               mask the causal diagonal, take the half-row max, then one
+//               barrier round among the 256 softmax threads exchanges the
+//               half maxima and the votes.  The skip rule "some row has
+//               (page max - running max) >= log2 eps" is decided exactly on
+//               half rows, because max(a, b) - m >= t  <=>  a - m >= t or
+//               b - m >= t.  The first listed page is always kept.  For kept
+//               pages each thread writes P = exp2(s - m_ref) (bf16) for its
+//               half row into a swizzled shared-memory tile; m_ref, the
+//               exponent base, moves only when the running max passes it by
+//               more than 2^8 (O and l are then rescaled in TMEM), which keeps
+//               the result exact.
+// Decisions reach the V producer and the PV issuer as sequence-tagged words in
+// a shared-memory ring; their progress counters give the ring back-pressure.
 // Every wait is bounded: on timeout the CTA records COSA_ERR_TIMEOUT in the
-// status word, drains what it issued, frees TMEM and exits.
+// status word, drains what it issued, frees TMEM and exits; a timed-out CTA
+// makes every later CTA of the launch exit at once.
 #pragma once
 
 #include "common.cuh"
@@ -48,11 +59,14 @@ struct TcParams {
 template <int D, int P>
 struct TcCfg {
   static constexpr int QB = 128;                  // MMA M (rows per tile, padded)
-  static constexpr int KS = (P == 64) ? 4 : 2;    // K ring stages
-  static constexpr int VS = (P == 64) ? 3 : 2;    // V ring stages
-  static constexpr int PS = (P == 64) ? 3 : 2;    // P tile ring stages
+  static constexpr int NT = 384;                  // 4 role warps + 2 softmax warpgroups
+  static constexpr int HP = P / 2;                // S columns per softmax thread
+  static constexpr int HD = D / 2;                // O columns per softmax thread
+  static constexpr int KS = (P == 64) ? 6 : 2;    // K ring stages
+  static constexpr int VS = 2;                    // V ring stages
+  static constexpr int PS = (P == 64) ? 2 : 1;    // P tile ring stages
   static constexpr int SB = (P == 64) ? 4 : 3;    // S buffers in TMEM
-  static constexpr int DS = 16;                   // decision ring
+  static constexpr int DS = 64;                   // decision ring (words)
   static constexpr uint32_t Q_BYTES = QB * D * 2;
   static constexpr uint32_t KV_BYTES = P * D * 2;
   static constexpr uint32_t P_BYTES = QB * P * 2;
@@ -61,25 +75,31 @@ struct TcCfg {
   static constexpr uint32_t OFF_V = OFF_K + KS * KV_BYTES;
   static constexpr uint32_t OFF_P = OFF_V + VS * KV_BYTES;
   static constexpr uint32_t OFF_BAR = OFF_P + PS * P_BYTES;
-  // q, k_full/empty, v_full/empty, s_full/free, p_full/empty, dec, vote[2], mma_done
-  static constexpr int NBAR = 1 + 2 * KS + 2 * VS + 2 * SB + 2 * PS + DS + 2 + 1;
+  // q, k_full/empty, v_full/empty, s_full/free, p_full/empty, done (QK), done (PV)
+  static constexpr int NBAR = 1 + 2 * KS + 2 * VS + 2 * SB + 2 * PS + 2;
   static constexpr uint32_t OFF_MISC = OFF_BAR + NBAR * 8;
-  static constexpr uint32_t SMEM = OFF_MISC + 128;
+  // misc: +0 TMEM address, +4 abort flag, +8 PV progress, +12 V progress,
+  //       +16 votes [2][8], +80 decision words [DS], +512 half-row maxima
+  //       [2 parities][2 halves][128], +2560 half-row sums [2][128]
+  static constexpr uint32_t MISC_BYTES = 3584;
+  static constexpr uint32_t SMEM = OFF_MISC + MISC_BYTES;
   static constexpr uint32_t SMEM_ALLOC = SMEM + 1024;  // 1024-byte alignment slack
   static constexpr int COL_O = SB * P;
   static constexpr int TMEM_COLS = (SB * P + D <= 256) ? 256 : 512;
   static_assert(SB * P + D <= 512, "TMEM budget");
   static_assert(SMEM_ALLOC <= 227 * 1024, "shared memory budget");
+  static_assert(80 + 4 * DS <= 512, "decision ring fits its slot");
 };
 
 constexpr float kRescaleLog2 = 8.0f;  // m_ref trails the running max by < 2^8
 
 template <int D, int P, bool DENSE>
-__global__ void __launch_bounds__(256, 1)
+__global__ void __launch_bounds__(384, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const TcParams prm) {
   using C = TcCfg<D, P>;
   using namespace tc;
+  constexpr int HP = C::HP, HD = C::HD;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t sraw = static_cast<uint32_t>(__cvta_generic_to_shared(smem_raw));
   const uint32_t sb0 = (sraw + 1023u) & ~1023u;
@@ -98,15 +118,17 @@ __global__ void __launch_bounds__(256, 1)
   auto b_pempty = [&](int s) {
     return bar + 8u * (1 + 2 * C::KS + 2 * C::VS + 2 * C::SB + C::PS + s);
   };
-  auto b_dec = [&](int s) {
-    return bar + 8u * (1 + 2 * C::KS + 2 * C::VS + 2 * C::SB + 2 * C::PS + s);
-  };
-  auto b_vote = [&](int s) { return bar + 8u * (C::NBAR - 3 + s); };
-  const uint32_t b_done = bar + 8u * (C::NBAR - 1);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sg + C::OFF_MISC);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(sg + C::OFF_MISC + 4);
-  volatile int* votes = reinterpret_cast<volatile int*>(sg + C::OFF_MISC + 16);     // [2][4]
-  volatile int* dec_flag = reinterpret_cast<volatile int*>(sg + C::OFF_MISC + 48);  // [DS]
+  const uint32_t b_done_s = bar + 8u * (C::NBAR - 2);
+  const uint32_t b_done_pv = bar + 8u * (C::NBAR - 1);
+  uint8_t* misc = sg + C::OFF_MISC;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(misc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 4);
+  volatile int* pv_pos = reinterpret_cast<volatile int*>(misc + 8);
+  volatile int* v_pos = reinterpret_cast<volatile int*>(misc + 12);
+  volatile int* votes = reinterpret_cast<volatile int*>(misc + 16);               // [2][8]
+  volatile uint32_t* dec_word = reinterpret_cast<volatile uint32_t*>(misc + 80);  // [DS]
+  volatile float* hmax = reinterpret_cast<volatile float*>(misc + 512);     // [2][2][128]
+  volatile float* hsum = reinterpret_cast<volatile float*>(misc + 2560);    // [2][128]
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   // a CTA that ran out of time anywhere in this launch stops the others early
@@ -144,13 +166,14 @@ __global__ void __launch_bounds__(256, 1)
     mbar_init(b_q, 1);
     for (int s = 0; s < C::KS; ++s) { mbar_init(b_kfull(s), 1); mbar_init(b_kempty(s), 1); }
     for (int s = 0; s < C::VS; ++s) { mbar_init(b_vfull(s), 1); mbar_init(b_vempty(s), 1); }
-    for (int s = 0; s < C::SB; ++s) { mbar_init(b_sfull(s), 1); mbar_init(b_sfree(s), 128); }
-    for (int s = 0; s < C::PS; ++s) { mbar_init(b_pfull(s), 128); mbar_init(b_pempty(s), 1); }
-    for (int s = 0; s < C::DS; ++s) mbar_init(b_dec(s), 1);
-    mbar_init(b_vote(0), 4);
-    mbar_init(b_vote(1), 4);
-    mbar_init(b_done, 1);
+    for (int s = 0; s < C::SB; ++s) { mbar_init(b_sfull(s), 1); mbar_init(b_sfree(s), 8); }
+    for (int s = 0; s < C::PS; ++s) { mbar_init(b_pfull(s), 8); mbar_init(b_pempty(s), 1); }
+    mbar_init(b_done_s, 1);
+    mbar_init(b_done_pv, 1);
     *abort_flag = 0;
+    *pv_pos = 0;
+    *v_pos = 0;
+    for (int s = 0; s < C::DS; ++s) dec_word[s] = 0xFFFFFFFFu;
     fence_barrier_init();
   }
   if (warp == 1) {
@@ -159,9 +182,9 @@ __global__ void __launch_bounds__(256, 1)
   }
   if (prm.q_block < C::QB && warp >= 4) {
     // rows past the q-block are padding: zero them once (the TMA box fills the rest)
-    for (int i = tid - 128; i < (C::QB - prm.q_block) * (D / 64) * 8; i += 128) {
-      const int chunk = i & 7, r = prm.q_block + (i >> 3) % (C::QB - prm.q_block);
-      const int kb = (i >> 3) / (C::QB - prm.q_block);
+    const int pad = C::QB - prm.q_block;
+    for (int i = tid - 128; i < pad * (D / 64) * 8; i += 256) {
+      const int chunk = i & 7, r = prm.q_block + (i >> 3) % pad, kb = (i >> 3) / pad;
       st_shared_v4(sQ + kb * (C::QB * 128) + r * 128 + chunk * 16, 0u, 0u, 0u, 0u);
     }
     fence_proxy_async_smem();
@@ -171,22 +194,41 @@ __global__ void __launch_bounds__(256, 1)
   const uint32_t tmem = *tmem_slot;
 
   const unsigned long long tmo = prm.timeout_ns;
-  // bounded blocking wait; false on timeout or abort
+  auto give_up = [&]() {
+    *abort_flag = 1;
+    set_status(COSA_ERR_TIMEOUT);
+  };
+  // bounded blocking wait on an mbarrier phase; false on timeout or abort
   auto wait = [&](uint32_t bar_addr, uint32_t parity) -> bool {
     if (mbar_try_wait(bar_addr, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
     uint32_t spins = 0;
     while (!mbar_try_wait(bar_addr, parity)) {
       if (*abort_flag) return false;
-      if ((++spins & 63u) == 0) {
-        if (*(volatile int*)&g_status == COSA_ERR_TIMEOUT || globaltimer_ns() - t0 > tmo) {
-          *abort_flag = 1;
-          set_status(COSA_ERR_TIMEOUT);
-          return false;
-        }
+      if ((++spins & 63u) == 0 &&
+          (*(volatile int*)&g_status == COSA_ERR_TIMEOUT || globaltimer_ns() - t0 > tmo)) {
+        give_up();
+        return false;
       }
     }
     return true;
+  };
+  // bounded wait for the decision on page i; returns -1 on timeout, else 0/1
+  auto decision = [&](int i) -> int {
+    const uint32_t want = (uint32_t)i << 1;
+    uint32_t w = dec_word[i % C::DS];
+    if ((w & ~1u) == want) return (int)(w & 1u);
+    const uint64_t t0 = globaltimer_ns();
+    uint32_t spins = 0;
+    while (((w = dec_word[i % C::DS]) & ~1u) != want) {
+      if (*abort_flag) return -1;
+      if ((++spins & 63u) == 0 &&
+          (*(volatile int*)&g_status == COSA_ERR_TIMEOUT || globaltimer_ns() - t0 > tmo)) {
+        give_up();
+        return -1;
+      }
+    }
+    return (int)(w & 1u);
   };
 
   if (warp == 0) {
@@ -242,10 +284,12 @@ __global__ void __launch_bounds__(256, 1)
       for (int ii = 0; ii < nb; ++ii) {
         const int i = base + ii;
         const int cz = __shfl_sync(0xffffffffu, cz_l, ii);
-        if (!DENSE && i > 0) {
-          ok = __all_sync(0xffffffffu, wait(b_dec(i % C::DS), (i / C::DS) & 1));
+        if (!DENSE && i > 0) {  // page 0 is always kept: its V goes out before the vote
+          const int d = decision(i);
+          ok = __all_sync(0xffffffffu, d >= 0);
           if (!ok) break;
-          if (dec_flag[i % C::DS] == 0) continue;
+          if (lane == 0) *v_pos = i + 1;
+          if (d == 0) continue;
         }
         const int s = vc % C::VS;
         if (vc >= C::VS) {
@@ -260,6 +304,11 @@ __global__ void __launch_bounds__(256, 1)
         }
         ++vc;
         __syncwarp();
+        if (!DENSE && i == 0) {
+          ok = __all_sync(0xffffffffu, decision(0) >= 0);
+          if (!ok) break;
+          if (lane == 0) *v_pos = 1;
+        }
       }
     }
     if (lane == 0 && *abort_flag) {
@@ -270,208 +319,221 @@ __global__ void __launch_bounds__(256, 1)
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      // ================= MMA issuer =================
+      // ================= QK^T issuer, list order =================
       constexpr uint32_t ID_QK = idesc_bf16_f32(128, P, 0);
-      constexpr uint32_t ID_PV = idesc_bf16_f32(128, D, 1);
       bool ok = wait(b_q, 0);
-      tc_fence_after();
-      int js = 0, ipv = 0, cpv = 0;
-      uint64_t last = globaltimer_ns();
-      while (ok && ipv < n_list) {
-        bool prog = false;
-        // ---- PV for page ipv once it is decided (and, if kept, P and V are ready)
-        bool known = true, keep = true;
-        if (!DENSE) {
-          known = mbar_test_wait(b_dec(ipv % C::DS), (ipv / C::DS) & 1);
-          keep = known && dec_flag[ipv % C::DS] != 0;
-        }
-        if (known) {
-          if (!keep) {
-            ++ipv;
-            prog = true;
-          } else {
-            const int vs = cpv % C::VS, ps = cpv % C::PS;
-            if (mbar_test_wait(b_vfull(vs), (cpv / C::VS) & 1) &&
-                mbar_test_wait(b_pfull(ps), (cpv / C::PS) & 1)) {
-              tc_fence_after();
+      for (int j = 0; ok && j < n_list; ++j) {
+        const int ks = j % C::KS, sbuf = j % C::SB;
+        if (!wait(b_kfull(ks), (j / C::KS) & 1)) break;
+        if (j >= C::SB && !wait(b_sfree(sbuf), ((j / C::SB) - 1) & 1)) break;
+        tc_fence_after();
 #pragma unroll
-              for (int k = 0; k < P / 16; ++k) {
-                const uint64_t a = smem_desc_sw128(
-                    sP + ps * C::P_BYTES + (k >> 2) * (C::QB * 128) + (k & 3) * 32, 16, 1024);
-                const uint64_t bd =
-                    smem_desc_sw128(sV + vs * C::KV_BYTES + k * 16 * 128, P * 128, 1024);
-                mma_bf16_ss(tmem + C::COL_O, a, bd, ID_PV, (cpv > 0 || k > 0) ? 1u : 0u);
-              }
-              mma_commit(b_vempty(vs));
-              mma_commit(b_pempty(ps));
-              ++cpv;
-              ++ipv;
-              prog = true;
-            }
-          }
+        for (int k = 0; k < D / 16; ++k) {
+          const uint64_t a = smem_desc_sw128(sQ + (k >> 2) * (C::QB * 128) + (k & 3) * 32, 16, 1024);
+          const uint64_t bd =
+              smem_desc_sw128(sK + ks * C::KV_BYTES + (k >> 2) * (P * 128) + (k & 3) * 32, 16, 1024);
+          mma_bf16_ss(tmem + sbuf * P, a, bd, ID_QK, k > 0 ? 1u : 0u);
         }
-        // ---- S for page js (bounded lead over the PV pointer: decision ring)
-        if (js < n_list && js < ipv + C::DS - 2) {
-          const int ks = js % C::KS, sbuf = js % C::SB;
-          if (mbar_test_wait(b_kfull(ks), (js / C::KS) & 1) &&
-              (js < C::SB || mbar_test_wait(b_sfree(sbuf), ((js / C::SB) - 1) & 1))) {
-            tc_fence_after();
-#pragma unroll
-            for (int k = 0; k < D / 16; ++k) {
-              const uint64_t a =
-                  smem_desc_sw128(sQ + (k >> 2) * (C::QB * 128) + (k & 3) * 32, 16, 1024);
-              const uint64_t bd = smem_desc_sw128(
-                  sK + ks * C::KV_BYTES + (k >> 2) * (P * 128) + (k & 3) * 32, 16, 1024);
-              mma_bf16_ss(tmem + sbuf * P, a, bd, ID_QK, k > 0 ? 1u : 0u);
-            }
-            mma_commit(b_kempty(ks));
-            mma_commit(b_sfull(sbuf));
-            ++js;
-            prog = true;
-          }
-        }
-        const uint64_t now = globaltimer_ns();
-        if (prog) {
-          last = now;
-        } else {
-          if (*abort_flag) break;
-          if (now - last > tmo || *(volatile int*)&g_status == COSA_ERR_TIMEOUT) {
-            *abort_flag = 1;
-            set_status(COSA_ERR_TIMEOUT);
-            break;
-          }
-          __nanosleep(20);
-        }
+        mma_commit(b_kempty(ks));
+        mma_commit(b_sfull(sbuf));
       }
-      // all issued MMAs complete before teardown frees TMEM
-      mma_commit(b_done);
+      // every issued MMA completes before teardown frees TMEM
+      mma_commit(b_done_s);
       const uint64_t t0 = globaltimer_ns();
-      while (!mbar_try_wait(b_done, 0) && globaltimer_ns() - t0 < tmo) {}
+      while (!mbar_try_wait(b_done_s, 0) && globaltimer_ns() - t0 < tmo) {}
     }
-  } else if (warp >= 4) {
-    // ================= softmax: thread <-> row <-> TMEM lane =================
-    const int q4 = warp & 3;
+  } else if (warp == 3) {
+    if (lane == 0) {
+      // ================= PV issuer, kept pages in list order =================
+      constexpr uint32_t ID_PV = idesc_bf16_f32(128, D, 1);
+      uint8_t* slog = prm.skip_log ? prm.skip_log + (bh * prm.num_q_blocks + qb) * prm.k_cap : nullptr;
+      int cpv = 0;
+      for (int i = 0; i < n_list; ++i) {
+        if (!DENSE) {
+          const int d = decision(i);
+          if (d < 0) break;
+          *pv_pos = i + 1;
+          if (slog) slog[i] = d ? 0 : 1;
+          if (d == 0) continue;
+        }
+        const int vs = cpv % C::VS, ps = cpv % C::PS;
+        if (!wait(b_vfull(vs), (cpv / C::VS) & 1)) break;
+        if (!wait(b_pfull(ps), (cpv / C::PS) & 1)) break;
+        tc_fence_after();
+#pragma unroll
+        for (int k = 0; k < P / 16; ++k) {
+          const uint64_t a = smem_desc_sw128(
+              sP + ps * C::P_BYTES + (k >> 2) * (C::QB * 128) + (k & 3) * 32, 16, 1024);
+          const uint64_t bd = smem_desc_sw128(sV + vs * C::KV_BYTES + k * 16 * 128, P * 128, 1024);
+          mma_bf16_ss(tmem + C::COL_O, a, bd, ID_PV, (cpv > 0 || k > 0) ? 1u : 0u);
+        }
+        mma_commit(b_vempty(vs));
+        mma_commit(b_pempty(ps));
+        ++cpv;
+      }
+      mma_commit(b_done_pv);
+      const uint64_t t0 = globaltimer_ns();
+      while (!mbar_try_wait(b_done_pv, 0) && globaltimer_ns() - t0 < tmo) {}
+    }
+  } else {
+    // ================= softmax: two warpgroups, half a row each =================
+    const int hw = (warp - 4) >> 2;      // which half of the columns
+    const int q4 = warp & 3;             // TMEM lane quarter
     const int row = q4 * 32 + lane;
     const bool row_valid = row < prm.q_block;
     const int grow = row0 + row;
+    const int c0 = hw * HP;              // first S column of this thread
     const uint32_t t_row = tmem + ((uint32_t)(q4 * 32) << 16);
     const bool leader = (tid == 128);
+    const float sl2 = prm.scale_log2, le = prm.log2_eps;
     float m_run = -INFINITY, m_ref = -INFINITY, l = 0.f;
     int ci = 0;
-    bool ok = true;
+    bool ok = true;     // collective: every softmax warp leaves the loop at the same page
+    bool fail = false;  // this warp missed a wait after the vote; reported at the next vote
     int pid_l = 0;
+    auto load_half = [&](int sbuf, uint32_t* raw) {
+      if constexpr (HP == 64) {
+        tmem_ld64(t_row + sbuf * P + c0, raw);
+      } else {
+        tmem_ld32(t_row + sbuf * P + c0, raw);
+      }
+    };
     for (int j = 0; j < n_list; ++j) {
       if ((j & 31) == 0) pid_l = (j + lane < n_list) ? page_at(j + lane) : 0;
-      const int page = __shfl_sync(0xffffffffu, pid_l, j & 31);
-      const int sbuf = j % C::SB;
-      ok = __all_sync(0xffffffffu, wait(b_sfull(sbuf), (j / C::SB) & 1));
-      if (!ok) break;
-      tc_fence_after();
-      float s[P];
-#pragma unroll
-      for (int c = 0; c < P / 32; ++c) {
-        uint32_t raw[32];
-        tmem_ld32(t_row + sbuf * P + c * 32, raw);
-#pragma unroll
-        for (int e = 0; e < 32; ++e) s[c * 32 + e] = __uint_as_float(raw[e]);
-      }
-      tc_fence_before();
-      mbar_arrive(b_sfree(sbuf));
-      const int key0 = page * P;
+      const int key0 = __shfl_sync(0xffffffffu, pid_l, j & 31) * P;
       const bool diag = key0 + P - 1 > row0;
-      float mloc = -INFINITY;
+      const int sbuf = j % C::SB;
+      const bool okw = !fail && __all_sync(0xffffffffu, wait(b_sfull(sbuf), (j / C::SB) & 1));
+      // ---- half-row max of S_j (raw logits, causal mask on the diagonal)
+      float mh = -INFINITY;
+      if (okw) {
+        tc_fence_after();
+        uint32_t raw[HP];
+        load_half(sbuf, raw);
+        float v[HP];
 #pragma unroll
-      for (int c = 0; c < P; ++c) {
-        float v = s[c] * prm.scale_log2;
-        if (!row_valid || (diag && key0 + c > grow)) v = -INFINITY;
-        s[c] = v;
-        mloc = fmaxf(mloc, v);
+        for (int e = 0; e < HP; ++e) {
+          v[e] = __uint_as_float(raw[e]);
+          if (diag && key0 + c0 + e > grow) v[e] = -INFINITY;
+        }
+#pragma unroll
+        for (int w = HP / 2; w > 0; w >>= 1)
+#pragma unroll
+          for (int e = 0; e < w; ++e) v[e] = fmaxf(v[e], v[e + w]);
+        mh = v[0];
       }
-      bool skip = false;
-      if (!DENSE) {
-        if (j > 0) {
-          const bool need =
-              mloc != -INFINITY && (m_run == -INFINITY || mloc - m_run >= prm.log2_eps);
-          const int any = __any_sync(0xffffffffu, need) ? 1 : 0;
-          if (lane == 0) {
-            votes[(j & 1) * 4 + q4] = any;
-            mbar_arrive(b_vote(j & 1));
+      const bool lv = row_valid && mh != -INFINITY;
+      const float mlh = lv ? mh * sl2 : -INFINITY;
+      // ---- one barrier round: half maxima + votes (+ failure bits)
+      const bool need = lv && (m_run == -INFINITY || mlh - m_run >= le);
+      const uint32_t bits = (okw ? 0u : 1u) | (__any_sync(0xffffffffu, need) ? 2u : 0u);
+      hmax[((j & 1) * 2 + hw) * 128 + row] = mlh;
+      if (lane == 0) votes[(j & 1) * 8 + (warp - 4)] = (int)bits;
+      named_bar_sync(1, 256);
+      uint32_t all = 0;
+#pragma unroll
+      for (int w = 0; w < 8; ++w) all |= (uint32_t)votes[(j & 1) * 8 + w];
+      if (all & 1u) { ok = false; break; }
+      const float mloc = fmaxf(mlh, hmax[((j & 1) * 2 + (hw ^ 1)) * 128 + row]);
+      const bool keep = DENSE || j == 0 || (all & 2u);
+      if (!DENSE && leader) {
+        // publish the decision once both consumers are past page j - DS
+        if (j >= C::DS) {
+          const uint64_t t0 = globaltimer_ns();
+          while (min(*pv_pos, *v_pos) <= j - C::DS) {
+            if (*abort_flag || globaltimer_ns() - t0 > tmo) { give_up(); break; }
           }
-          ok = __all_sync(0xffffffffu, wait(b_vote(j & 1), ((j - 1) >> 1) & 1));
-          if (!ok) break;
-          skip = (votes[(j & 1) * 4 + 0] | votes[(j & 1) * 4 + 1] | votes[(j & 1) * 4 + 2] |
-                  votes[(j & 1) * 4 + 3]) == 0;
         }
-        if (leader) {
-          dec_flag[j % C::DS] = skip ? 0 : 1;
-          mbar_arrive(b_dec(j % C::DS));
-          if (prm.skip_log)
-            prm.skip_log[(bh * prm.num_q_blocks + qb) * prm.k_cap + j] = skip ? 1 : 0;
-        }
+        dec_word[j % C::DS] = ((uint32_t)j << 1) | (keep ? 1u : 0u);
       }
-      if (skip) continue;
+      if (!keep) {
+        tc_fence_before();
+        if (lane == 0) mbar_arrive(b_sfree(sbuf));
+        continue;
+      }
       // ---- kept page: online softmax with a lazily moved exponent base
       const float m_new = fmaxf(m_run, mloc);
       m_run = m_new;
       const bool resc = (m_ref != -INFINITY) && (m_new > m_ref + kRescaleLog2);
       if (__any_sync(0xffffffffu, resc)) {
-        // O holds earlier pages: wait for the last issued PV, rescale rows in TMEM
-        ok = __all_sync(0xffffffffu, wait(b_pempty((ci - 1) % C::PS), ((ci - 1) / C::PS) & 1));
-        if (!ok) break;
-        tc_fence_after();
-        const float alpha = resc ? exp2f(m_ref - m_new) : 1.f;
+        // O holds earlier pages: wait for the last issued PV, rescale this half of the rows
+        fail = !__all_sync(0xffffffffu, wait(b_pempty((ci - 1) % C::PS), ((ci - 1) / C::PS) & 1));
+        if (!fail) {
+          tc_fence_after();
+          const float alpha = resc ? ex2_approx(m_ref - m_new) : 1.f;
+#pragma unroll 1
+          for (int c = 0; c < HD / 16; ++c) {
+            uint32_t r[16];
+            tmem_ld16(t_row + C::COL_O + hw * HD + c * 16, r);
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t r[32];
-          tmem_ld32(t_row + C::COL_O + c * 32, r);
-#pragma unroll
-          for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
-          tmem_st32(t_row + C::COL_O + c * 32, r);
+            for (int e = 0; e < 16; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
+            tmem_st16(t_row + C::COL_O + hw * HD + c * 16, r);
+          }
+          tmem_st_wait();
+          l *= alpha;
         }
-        tmem_st_wait();
-        l *= alpha;
       }
       if (m_new != -INFINITY && (m_ref == -INFINITY || resc)) m_ref = m_new;
-      // P row (bf16) into the swizzled K-major tile of ring slot ci % PS
+      // P half row (bf16) into the swizzled K-major tile of ring slot ci % PS
       const int ps = ci % C::PS;
-      if (ci >= C::PS) {
-        ok = __all_sync(0xffffffffu, wait(b_pempty(ps), ((ci / C::PS) - 1) & 1));
-        if (!ok) break;
-      }
-      const bool live = m_ref != -INFINITY;
-      float rs = 0.f;
+      if (!fail && ci >= C::PS)
+        fail = !__all_sync(0xffffffffu, wait(b_pempty(ps), ((ci / C::PS) - 1) & 1));
+      if (fail) continue;  // reported at the next vote
+      const bool rlive = row_valid && m_ref != -INFINITY;
+      const float nb2 = rlive ? -m_ref : 0.f;
+      float rs[4] = {0.f, 0.f, 0.f, 0.f};
       const uint32_t prow = sP + ps * C::P_BYTES + row * 128;
+      tc_fence_after();
+      {
+        uint32_t raw[HP];
+        load_half(sbuf, raw);
 #pragma unroll
-      for (int c8 = 0; c8 < P / 8; ++c8) {
-        uint32_t w[4];
+        for (int c8 = 0; c8 < HP / 8; ++c8) {
+          uint32_t w4[4];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float p0 = live ? exp2f(s[c8 * 8 + 2 * e] - m_ref) : 0.f;
-          const float p1 = live ? exp2f(s[c8 * 8 + 2 * e + 1] - m_ref) : 0.f;
-          rs += p0 + p1;
-          __nv_bfloat162 v2 = __floats2bfloat162_rn(p0, p1);
-          w[e] = *reinterpret_cast<uint32_t*>(&v2);
+          for (int e = 0; e < 4; ++e) {
+            const int i0 = c8 * 8 + 2 * e;
+            float x0 = fmaf(__uint_as_float(raw[i0]), sl2, nb2);
+            float x1 = fmaf(__uint_as_float(raw[i0 + 1]), sl2, nb2);
+            if (!rlive || (diag && key0 + c0 + i0 > grow)) x0 = -INFINITY;
+            if (!rlive || (diag && key0 + c0 + i0 + 1 > grow)) x1 = -INFINITY;
+            const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+            rs[e] += p0 + p1;
+            __nv_bfloat162 v2 = __floats2bfloat162_rn(p0, p1);
+            w4[e] = *reinterpret_cast<uint32_t*>(&v2);
+          }
+          const int cg = (c0 >> 3) + c8;  // 16-byte chunk index within the row
+          const int blk = cg >> 3, cc = cg & 7;
+          st_shared_v4(prow + blk * (C::QB * 128) + ((cc ^ (row & 7)) << 4), w4[0], w4[1], w4[2],
+                       w4[3]);
         }
-        const int blk = c8 >> 3, cc = c8 & 7;
-        st_shared_v4(prow + blk * (C::QB * 128) + ((cc ^ (row & 7)) << 4), w[0], w[1], w[2], w[3]);
       }
-      l += rs;
+      l += (rs[0] + rs[1]) + (rs[2] + rs[3]);
       fence_proxy_async_smem();
       tc_fence_before();
-      mbar_arrive(b_pfull(ps));
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(b_sfree(sbuf));
+        mbar_arrive(b_pfull(ps));
+      }
       ++ci;
     }
-    // ---- epilogue: O / l -> bf16, LSE (natural log), computed count
-    if (ok && ci > 0)
-      ok = __all_sync(0xffffffffu, wait(b_pempty((ci - 1) % C::PS), ((ci - 1) / C::PS) & 1));
+    // ---- epilogue: O / l -> bf16 (each warpgroup its half of the columns), LSE
+    if (ok && !fail && ci > 0)
+      fail = !__all_sync(0xffffffffu, wait(b_pempty((ci - 1) % C::PS), ((ci - 1) / C::PS) & 1));
+    if (ok) {  // all softmax warps are here together: exchange the half-row sums
+      hsum[hw * 128 + row] = l;
+      named_bar_sync(1, 256);
+      l += hsum[(hw ^ 1) * 128 + row];
+    }
     tc_fence_after();
     const float inv = l > 0.f ? 1.f / l : 0.f;
-    __nv_bfloat16* orow = prm.out + (bh * prm.seq_len + grow) * D;
+    __nv_bfloat16* orow = prm.out + (bh * prm.seq_len + grow) * D + hw * HD;
 #pragma unroll
-    for (int c = 0; c < D / 32; ++c) {
+    for (int c = 0; c < HD / 32; ++c) {
       uint32_t r[32];
-      if (ok && ci > 0) {
-        tmem_ld32(t_row + C::COL_O + c * 32, r);
+      if (ok && !fail && ci > 0) {
+        tmem_ld32(t_row + C::COL_O + hw * HD + c * 32, r);
       } else {
 #pragma unroll
         for (int e = 0; e < 32; ++e) r[e] = 0u;
@@ -491,7 +553,7 @@ __global__ void __launch_bounds__(256, 1)
         dst[3] = make_uint4(w[12], w[13], w[14], w[15]);
       }
     }
-    if (row_valid && prm.lse)
+    if (hw == 0 && row_valid && prm.lse)
       prm.lse[bh * prm.seq_len + grow] =
           l > 0.f ? (m_ref + log2f(l)) * 0.69314718055994531f : -INFINITY;
     if (!DENSE && leader && prm.computed) prm.computed[bh * prm.num_q_blocks + qb] = ci;

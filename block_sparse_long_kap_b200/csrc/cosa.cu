@@ -227,7 +227,7 @@ cosa_status_t launch_tc_t(const cosa_shape_t* s, const TcParams& prm, const void
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)Cfg::SMEM_ALLOC) != cudaSuccess)
     return COSA_ERR_CUDA;
-  kern<<<grid, 256, Cfg::SMEM_ALLOC, st>>>(mq, mk, mv, prm);
+  kern<<<grid, Cfg::NT, Cfg::SMEM_ALLOC, st>>>(mq, mk, mv, prm);
   return last_launch();
 }
 
