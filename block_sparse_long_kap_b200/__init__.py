@@ -31,7 +31,7 @@ EXPORTED_SYMBOLS = (
 )
 
 # Largest workspace the allocation-free Stage-1 entry point accepts (cosa.h).
-NOALLOC_SCRATCH_BYTES = 64 << 20
+NOALLOC_SCRATCH_BYTES = 128 << 20
 
 STATUS_NAMES = {0: "COSA_OK", 1: "COSA_ERR_INVALID_ARG", 2: "COSA_ERR_UNSUPPORTED",
                 3: "COSA_ERR_CUDA", 4: "COSA_ERR_TIMEOUT", 5: "COSA_ERR_WORKSPACE"}

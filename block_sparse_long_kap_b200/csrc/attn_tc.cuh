@@ -77,18 +77,20 @@ struct TcCfg {
   static constexpr uint32_t OFF_BAR = OFF_P + PS * P_BYTES;
   // q, k_full/empty, v_full/empty, s_full/free, p_full/empty, done (QK), done (PV)
   static constexpr int NBAR = 1 + 2 * KS + 2 * VS + 2 * SB + 2 * PS + 2;
-  static constexpr uint32_t OFF_MISC = OFF_BAR + NBAR * 8;
+  static constexpr uint32_t OFF_MISC = (OFF_BAR + NBAR * 8 + 127) & ~127u;  // vector-aligned
   // misc: +0 TMEM address, +4 abort flag, +8 PV progress, +12 V progress,
-  //       +16 votes [2][8], +80 decision words [DS], +512 half-row maxima
-  //       [2 parities][2 halves][128], +2560 half-row sums [2][128]
-  static constexpr uint32_t MISC_BYTES = 3584;
+  //       +16 votes [2 rounds][2 parities][8], +256 decision words [DS],
+  //       +512 half-row maxima [2 parities][2 pages][2 halves][128],
+  //       +4608 half-row sums [2][128]
+  static constexpr uint32_t MISC_BYTES = 5632;
   static constexpr uint32_t SMEM = OFF_MISC + MISC_BYTES;
   static constexpr uint32_t SMEM_ALLOC = SMEM + 1024;  // 1024-byte alignment slack
   static constexpr int COL_O = SB * P;
   static constexpr int TMEM_COLS = (SB * P + D <= 256) ? 256 : 512;
   static_assert(SB * P + D <= 512, "TMEM budget");
   static_assert(SMEM_ALLOC <= 227 * 1024, "shared memory budget");
-  static_assert(80 + 4 * DS <= 512, "decision ring fits its slot");
+  static_assert(256 + 4 * DS <= 512, "decision ring fits its slot");
+  static_assert(OFF_MISC % 128 == 0, "16-byte vector access to the vote words");
 };
 
 constexpr float kRescaleLog2 = 8.0f;  // m_ref trails the running max by < 2^8
@@ -125,10 +127,10 @@ __global__ void __launch_bounds__(384, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 4);
   volatile int* pv_pos = reinterpret_cast<volatile int*>(misc + 8);
   volatile int* v_pos = reinterpret_cast<volatile int*>(misc + 12);
-  volatile int* votes = reinterpret_cast<volatile int*>(misc + 16);               // [2][8]
-  volatile uint32_t* dec_word = reinterpret_cast<volatile uint32_t*>(misc + 80);  // [DS]
-  volatile float* hmax = reinterpret_cast<volatile float*>(misc + 512);     // [2][2][128]
-  volatile float* hsum = reinterpret_cast<volatile float*>(misc + 2560);    // [2][128]
+  volatile int* votes = reinterpret_cast<volatile int*>(misc + 16);               // [2][2][8]
+  volatile uint32_t* dec_word = reinterpret_cast<volatile uint32_t*>(misc + 256);  // [DS]
+  volatile float* hmax = reinterpret_cast<volatile float*>(misc + 512);     // [2][2][2][128]
+  volatile float* hsum = reinterpret_cast<volatile float*>(misc + 4608);    // [2][128]
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   // a CTA that ran out of time anywhere in this launch stops the others early
@@ -203,9 +205,9 @@ __global__ void __launch_bounds__(384, 1)
     if (mbar_try_wait(bar_addr, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
     uint32_t spins = 0;
-    while (!mbar_try_wait(bar_addr, parity)) {
+    while (!mbar_try_wait_sleep(bar_addr, parity, 20000u)) {
       if (*abort_flag) return false;
-      if ((++spins & 63u) == 0 &&
+      if ((++spins & 3u) == 0 &&
           (*(volatile int*)&g_status == COSA_ERR_TIMEOUT || globaltimer_ns() - t0 > tmo)) {
         give_up();
         return false;
@@ -227,6 +229,7 @@ __global__ void __launch_bounds__(384, 1)
         give_up();
         return -1;
       }
+      __nanosleep(64);  // leave the issue slots to the softmax warps sharing this scheduler
     }
     return (int)(w & 1u);
   };
@@ -391,132 +394,192 @@ __global__ void __launch_bounds__(384, 1)
     bool ok = true;     // collective: every softmax warp leaves the loop at the same page
     bool fail = false;  // this warp missed a wait after the vote; reported at the next vote
     int pid_l = 0;
-    auto load_half = [&](int sbuf, uint32_t* raw) {
-      if constexpr (HP == 64) {
-        tmem_ld64(t_row + sbuf * P + c0, raw);
-      } else {
-        tmem_ld32(t_row + sbuf * P + c0, raw);
-      }
-    };
-    for (int j = 0; j < n_list; ++j) {
+    // page id of list entry j (warp-uniform); call once per j, in order
+    auto page_of = [&](int j) -> int {
       if ((j & 31) == 0) pid_l = (j + lane < n_list) ? page_at(j + lane) : 0;
-      const int key0 = __shfl_sync(0xffffffffu, pid_l, j & 31) * P;
-      const bool diag = key0 + P - 1 > row0;
-      const int sbuf = j % C::SB;
-      const bool okw = !fail && __all_sync(0xffffffffu, wait(b_sfull(sbuf), (j / C::SB) & 1));
-      // ---- half-row max of S_j (raw logits, causal mask on the diagonal)
-      float mh = -INFINITY;
-      if (okw) {
-        tc_fence_after();
-        uint32_t raw[HP];
-        load_half(sbuf, raw);
-        float v[HP];
+      return __shfl_sync(0xffffffffu, pid_l, j & 31);
+    };
+    // half-row max of raw logits, causal mask on the diagonal page
+    auto half_max = [&](const uint32_t* src, int key0) -> float {
+      float v[HP];
+      if (key0 + P - 1 > row0) {  // diagonal page (warp-uniform): causal mask
 #pragma unroll
-        for (int e = 0; e < HP; ++e) {
-          v[e] = __uint_as_float(raw[e]);
-          if (diag && key0 + c0 + e > grow) v[e] = -INFINITY;
+        for (int e = 0; e < HP; ++e)
+          v[e] = key0 + c0 + e > grow ? -INFINITY : __uint_as_float(src[e]);
+      } else {
+#pragma unroll
+        for (int e = 0; e < HP; ++e) v[e] = __uint_as_float(src[e]);
+      }
+#pragma unroll
+      for (int w = HP / 2; w > 0; w >>= 1)
+#pragma unroll
+        for (int e = 0; e < w; ++e) v[e] = fmaxf(v[e], v[e + w]);
+      return v[0];
+    };
+    // publish the decision on page j for the V producer and the PV issuer, once
+    // both are past page j - DS
+    auto publish = [&](int j, bool keep) {
+      if (j >= C::DS) {
+        const uint64_t t0 = globaltimer_ns();
+        while (min(*pv_pos, *v_pos) <= j - C::DS) {
+          if (*abort_flag || globaltimer_ns() - t0 > tmo) { give_up(); break; }
+          __nanosleep(32);
         }
-#pragma unroll
-        for (int w = HP / 2; w > 0; w >>= 1)
-#pragma unroll
-          for (int e = 0; e < w; ++e) v[e] = fmaxf(v[e], v[e + w]);
-        mh = v[0];
       }
-      const bool lv = row_valid && mh != -INFINITY;
-      const float mlh = lv ? mh * sl2 : -INFINITY;
-      // ---- one barrier round: half maxima + votes (+ failure bits)
-      const bool need = lv && (m_run == -INFINITY || mlh - m_run >= le);
-      const uint32_t bits = (okw ? 0u : 1u) | (__any_sync(0xffffffffu, need) ? 2u : 0u);
-      hmax[((j & 1) * 2 + hw) * 128 + row] = mlh;
-      if (lane == 0) votes[(j & 1) * 8 + (warp - 4)] = (int)bits;
-      named_bar_sync(1, 256);
-      uint32_t all = 0;
-#pragma unroll
-      for (int w = 0; w < 8; ++w) all |= (uint32_t)votes[(j & 1) * 8 + w];
-      if (all & 1u) { ok = false; break; }
-      const float mloc = fmaxf(mlh, hmax[((j & 1) * 2 + (hw ^ 1)) * 128 + row]);
-      const bool keep = DENSE || j == 0 || (all & 2u);
-      if (!DENSE && leader) {
-        // publish the decision once both consumers are past page j - DS
-        if (j >= C::DS) {
-          const uint64_t t0 = globaltimer_ns();
-          while (min(*pv_pos, *v_pos) <= j - C::DS) {
-            if (*abort_flag || globaltimer_ns() - t0 > tmo) { give_up(); break; }
-          }
-        }
-        dec_word[j % C::DS] = ((uint32_t)j << 1) | (keep ? 1u : 0u);
-      }
-      if (!keep) {
-        tc_fence_before();
-        if (lane == 0) mbar_arrive(b_sfree(sbuf));
-        continue;
-      }
-      // ---- kept page: online softmax with a lazily moved exponent base
+      dec_word[j % C::DS] = ((uint32_t)j << 1) | (keep ? 1u : 0u);
+    };
+    // kept page: online softmax with a lazily moved exponent base, then the P half
+    // row (bf16) into the swizzled K-major tile of ring slot ci % PS
+    auto kept_page = [&](const uint32_t* cur, float mloc, int key0) {
       const float m_new = fmaxf(m_run, mloc);
       m_run = m_new;
       const bool resc = (m_ref != -INFINITY) && (m_new > m_ref + kRescaleLog2);
       if (__any_sync(0xffffffffu, resc)) {
         // O holds earlier pages: wait for the last issued PV, rescale this half of the rows
-        fail = !__all_sync(0xffffffffu, wait(b_pempty((ci - 1) % C::PS), ((ci - 1) / C::PS) & 1));
-        if (!fail) {
-          tc_fence_after();
-          const float alpha = resc ? ex2_approx(m_ref - m_new) : 1.f;
+        fail = !__all_sync(0xffffffffu,
+                           wait(b_pempty((ci - 1) % C::PS), ((ci - 1) / C::PS) & 1));
+        if (fail) return;
+        tc_fence_after();
+        const float alpha = resc ? ex2_approx(m_ref - m_new) : 1.f;
 #pragma unroll 1
-          for (int c = 0; c < HD / 16; ++c) {
-            uint32_t r[16];
-            tmem_ld16(t_row + C::COL_O + hw * HD + c * 16, r);
+        for (int c = 0; c < HD / 16; ++c) {
+          uint32_t r[16];
+          tmem_ld16(t_row + C::COL_O + hw * HD + c * 16, r);
 #pragma unroll
-            for (int e = 0; e < 16; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
-            tmem_st16(t_row + C::COL_O + hw * HD + c * 16, r);
-          }
-          tmem_st_wait();
-          l *= alpha;
+          for (int e = 0; e < 16; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
+          tmem_st16(t_row + C::COL_O + hw * HD + c * 16, r);
         }
+        tmem_st_wait();
+        l *= alpha;
       }
       if (m_new != -INFINITY && (m_ref == -INFINITY || resc)) m_ref = m_new;
-      // P half row (bf16) into the swizzled K-major tile of ring slot ci % PS
       const int ps = ci % C::PS;
-      if (!fail && ci >= C::PS)
+      if (ci >= C::PS) {
         fail = !__all_sync(0xffffffffu, wait(b_pempty(ps), ((ci / C::PS) - 1) & 1));
-      if (fail) continue;  // reported at the next vote
+        if (fail) return;
+      }
+      const bool diag = key0 + P - 1 > row0;
       const bool rlive = row_valid && m_ref != -INFINITY;
       const float nb2 = rlive ? -m_ref : 0.f;
       float rs[4] = {0.f, 0.f, 0.f, 0.f};
       const uint32_t prow = sP + ps * C::P_BYTES + row * 128;
-      tc_fence_after();
-      {
-        uint32_t raw[HP];
-        load_half(sbuf, raw);
 #pragma unroll
-        for (int c8 = 0; c8 < HP / 8; ++c8) {
-          uint32_t w4[4];
+      for (int c8 = 0; c8 < HP / 8; ++c8) {
+        uint32_t w4[4];
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int i0 = c8 * 8 + 2 * e;
-            float x0 = fmaf(__uint_as_float(raw[i0]), sl2, nb2);
-            float x1 = fmaf(__uint_as_float(raw[i0 + 1]), sl2, nb2);
-            if (!rlive || (diag && key0 + c0 + i0 > grow)) x0 = -INFINITY;
-            if (!rlive || (diag && key0 + c0 + i0 + 1 > grow)) x1 = -INFINITY;
-            const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
-            rs[e] += p0 + p1;
-            __nv_bfloat162 v2 = __floats2bfloat162_rn(p0, p1);
-            w4[e] = *reinterpret_cast<uint32_t*>(&v2);
-          }
-          const int cg = (c0 >> 3) + c8;  // 16-byte chunk index within the row
-          const int blk = cg >> 3, cc = cg & 7;
-          st_shared_v4(prow + blk * (C::QB * 128) + ((cc ^ (row & 7)) << 4), w4[0], w4[1], w4[2],
-                       w4[3]);
+        for (int e = 0; e < 4; ++e) {
+          const int i0 = c8 * 8 + 2 * e;
+          float x0 = fmaf(__uint_as_float(cur[i0]), sl2, nb2);
+          float x1 = fmaf(__uint_as_float(cur[i0 + 1]), sl2, nb2);
+          if (!rlive || (diag && key0 + c0 + i0 > grow)) x0 = -INFINITY;
+          if (!rlive || (diag && key0 + c0 + i0 + 1 > grow)) x1 = -INFINITY;
+          const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+          rs[e] += p0 + p1;
+          __nv_bfloat162 v2 = __floats2bfloat162_rn(p0, p1);
+          w4[e] = *reinterpret_cast<uint32_t*>(&v2);
         }
+        const int cg = (c0 >> 3) + c8;  // 16-byte chunk index within the row
+        const int blk = cg >> 3, cc = cg & 7;
+        st_shared_v4(prow + blk * (C::QB * 128) + ((cc ^ (row & 7)) << 4), w4[0], w4[1], w4[2],
+                     w4[3]);
       }
       l += (rs[0] + rs[1]) + (rs[2] + rs[3]);
       fence_proxy_async_smem();
-      tc_fence_before();
       __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(b_sfree(sbuf));
-        mbar_arrive(b_pfull(ps));
-      }
+      if (lane == 0) mbar_arrive(b_pfull(ps));
       ++ci;
+    };
+    // votes of all eight softmax warps for round r of iteration it
+    auto vote_round = [&](int r, int it, uint32_t bits) -> uint32_t {
+      int* vt = const_cast<int*>(votes) + (r * 2 + (it & 1)) * 8;
+      if (lane == 0) vt[warp - 4] = (int)bits;
+      named_bar_sync(1, 256);  // orders the shared-memory exchange around it
+      const int4 v0 = *reinterpret_cast<const int4*>(vt);
+      const int4 v1 = *reinterpret_cast<const int4*>(vt + 4);
+      return (uint32_t)(v0.x | v0.y | v0.z | v0.w | v1.x | v1.y | v1.z | v1.w);
+    };
+    // pages per iteration: two when a half row is 32 columns (the registers allow it)
+    constexpr int BATCH = (HP == 32) ? 2 : 1;
+    for (int j = 0, it = 0; j < n_list; j += BATCH, ++it) {
+      const int nb = min(BATCH, n_list - j);
+      int key0[BATCH];
+      uint32_t sv[BATCH][HP];
+      float mlh[BATCH];
+      bool lv[BATCH];
+#pragma unroll
+      for (int t = 0; t < BATCH; ++t) key0[t] = t < nb ? page_of(j + t) * P : 0;
+      // ---- S half rows of the batch: TMEM -> registers (one round trip), buffers back
+      bool okw = !fail;
+#pragma unroll
+      for (int t = 0; t < BATCH; ++t)
+        if (t < nb) okw = okw && wait(b_sfull((j + t) % C::SB), ((j + t) / C::SB) & 1);
+      okw = __all_sync(0xffffffffu, okw);
+      if (okw) {
+        tc_fence_after();
+#pragma unroll
+        for (int t = 0; t < BATCH; ++t)
+          if (t < nb)
+#pragma unroll
+            for (int c = 0; c < HP / 32; ++c)
+              tmem_ld32_async(t_row + ((j + t) % C::SB) * P + c0 + c * 32, sv[t] + c * 32);
+#pragma unroll
+        for (int t = 0; t < BATCH; ++t)
+#pragma unroll
+          for (int c = 0; c < HP / 32; ++c) {
+            if (t == 0 && c == 0) tmem_ld_wait32(sv[0]);
+            else reg_tie32(sv[t] + c * 32);
+          }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0)
+#pragma unroll
+          for (int t = 0; t < BATCH; ++t)
+            if (t < nb) mbar_arrive(b_sfree((j + t) % C::SB));
+      }
+      // ---- half-row maxima -> round 1 exchange
+      float* hm = const_cast<float*>(hmax) + (it & 1) * 512;
+#pragma unroll
+      for (int t = 0; t < BATCH; ++t) {
+        const float mh = (okw && t < nb) ? half_max(sv[t], key0[t]) : -INFINITY;
+        lv[t] = row_valid && mh != -INFINITY;
+        mlh[t] = lv[t] ? mh * sl2 : -INFINITY;
+        hm[(t * 2 + hw) * 128 + row] = mlh[t];
+      }
+      const uint32_t all1 = vote_round(0, it, okw ? 0u : 1u);
+      if (all1 & 1u) { ok = false; break; }
+      float mloc[BATCH];
+#pragma unroll
+      for (int t = 0; t < BATCH; ++t) {
+        mloc[t] = fmaxf(mlh[t], hm[(t * 2 + (hw ^ 1)) * 128 + row]);
+        lv[t] = mloc[t] != -INFINITY;
+      }
+      // ---- round 2: votes on full row maxima.  Page j + 1 is voted for both
+      // outcomes of page j, so the decisions stay exactly sequential.
+      bool keep[BATCH];
+      if (DENSE) {
+#pragma unroll
+        for (int t = 0; t < BATCH; ++t) keep[t] = true;
+      } else {
+        const bool n0 = lv[0] && (m_run == -INFINITY || mloc[0] - m_run >= le);
+        uint32_t bits = __any_sync(0xffffffffu, n0) ? 2u : 0u;
+        if (BATCH == 2 && nb == 2) {
+          const float mk = fmaxf(m_run, mloc[0]);
+          const bool nk = lv[BATCH - 1] && (mk == -INFINITY || mloc[BATCH - 1] - mk >= le);
+          const bool ns = lv[BATCH - 1] && (m_run == -INFINITY || mloc[BATCH - 1] - m_run >= le);
+          bits |= __any_sync(0xffffffffu, nk) ? 4u : 0u;
+          bits |= __any_sync(0xffffffffu, ns) ? 8u : 0u;
+        }
+        const uint32_t all2 = vote_round(1, it, bits);
+        keep[0] = (j == 0) || (all2 & 2u);
+        if (BATCH == 2) keep[BATCH - 1] = keep[0] ? (all2 & 4u) != 0 : (all2 & 8u) != 0;
+        if (leader)
+#pragma unroll
+          for (int t = 0; t < BATCH; ++t)
+            if (t < nb) publish(j + t, keep[t]);
+      }
+#pragma unroll
+      for (int t = 0; t < BATCH; ++t)
+        if (t < nb && keep[t] && !fail) kept_page(sv[t], mloc[t], key0[t]);
     }
     // ---- epilogue: O / l -> bf16 (each warpgroup its half of the columns), LSE
     if (ok && !fail && ci > 0)

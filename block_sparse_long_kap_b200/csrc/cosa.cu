@@ -10,6 +10,7 @@
 
 #include "common.cuh"
 #include "kap.cuh"
+#include "kap_tc.cuh"
 #include "attn_tc.cuh"
 
 using namespace cosa;
@@ -49,33 +50,38 @@ cosa_status_t check_kap(const cosa_shape_t* s, const cosa_kap_params_t* k) {
   return COSA_OK;
 }
 
-// Row length of the transposed pooled-key array khatT[b][h_kv][d][.]: the
-// number of sub-keys nP * T rounded up to a multiple of 4 (16-byte rows).
-size_t khat_stride(const cosa_shape_t* s, const cosa_kap_params_t* k) {
-  size_t n = (size_t)(s->seq_len / s->page_size) * (s->page_size / k->k_sub);
-  return (n + 3) & ~size_t(3);
-}
-
 struct KapLayout {
-  size_t qhat_off, khat_off, scores_off, hrm_off, total;
+  size_t q_hi, q_lo, k_hi, k_lo, a, row_max, row_arg, total;
 };
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
+// Workspace of cosa_kap_select: pooled queries and keys (TF32 hi and lo
+// terms), the triangular page-max array, and per representative row its max
+// and the first page attaining it.
 KapLayout kap_layout(const cosa_shape_t* s, const cosa_kap_params_t* k) {
   KapLayout L;
   const size_t B = s->batch, Hq = s->num_q_heads, Hk = s->num_kv_heads, N = s->seq_len,
                D = s->head_dim;
-  const size_t nP = N / s->page_size, nQB = N / s->q_block;
+  const size_t R = s->q_block / k->q_sub, nQB = N / s->q_block, nP = N / s->page_size;
+  const size_t T = s->page_size / k->k_sub, GR = (Hq / Hk) * R;
+  const size_t qrows = B * Hq * nQB * R, krows = B * Hk * nP * T;
+  const size_t tri = (size_t)cum_pages((int)nQB, s->q_block, s->page_size);
   size_t off = 0;
-  L.qhat_off = off;
-  off = align256(off + B * Hq * (N / k->q_sub) * D * sizeof(float));
-  L.khat_off = off;
-  off = align256(off + B * Hk * D * khat_stride(s, k) * sizeof(float));
-  L.scores_off = off;
-  off = align256(off + B * Hq * nQB * nP * sizeof(float));
-  L.hrm_off = off;
-  off = align256(off + B * Hq * nQB * nP);
+  L.q_hi = off;
+  off = align256(off + qrows * D * sizeof(float));
+  L.q_lo = off;
+  off = align256(off + qrows * D * sizeof(float));
+  L.k_hi = off;
+  off = align256(off + krows * D * sizeof(float));
+  L.k_lo = off;
+  off = align256(off + krows * D * sizeof(float));
+  L.a = off;
+  off = align256(off + B * Hk * GR * tri * sizeof(float));
+  L.row_max = off;
+  off = align256(off + qrows * sizeof(float));
+  L.row_arg = off;
+  off = align256(off + qrows * sizeof(int));
   L.total = off;
   return L;
 }
@@ -96,89 +102,6 @@ cosa_status_t last_launch() {
     return COSA_ERR_CUDA;
   }
   return COSA_OK;
-}
-
-// Score kernel: heads per CTA = largest divisor of G whose representatives
-// (at most 32) and score rows fit the shared-memory budget.
-constexpr size_t kScoreSmemLimit = 200 * 1024;
-
-template <int D>
-size_t score_smem(int hpc, int R, int nP) {
-  const int nrmax = hpc * R <= 16 ? 16 : 32;
-  return (size_t)D * nrmax * sizeof(float) + (size_t)hpc * R * nP * sizeof(float);
-}
-
-template <int D, int NRMAX>
-cosa_status_t launch_score(dim3 grid, size_t smem, cudaStream_t st, const float* qhat,
-                           const float* khatT, float* sc, uint8_t* hr, int Hq, int Hk, int G,
-                           int hpc, int nQB, int nP, int kstride, int R, int T, int q_sub,
-                           int k_sub, int P, int Bq, float scale) {
-  if (cudaFuncSetAttribute(kap_score_kernel<D, NRMAX>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)smem) != cudaSuccess)
-    return COSA_ERR_CUDA;
-  kap_score_kernel<D, NRMAX><<<grid, SCORE_THREADS, smem, st>>>(
-      qhat, khatT, sc, hr, Hq, Hk, G, hpc, nQB, nP, kstride, R, T, q_sub, k_sub, P, Bq, scale);
-  return last_launch();
-}
-
-template <int D>
-cosa_status_t launch_kap(const cosa_shape_t* s, const cosa_kap_params_t* k, const void* q,
-                         const void* k_pool, const int32_t* page_table, int32_t* order,
-                         int32_t* count, float* scores, uint8_t* hrm, const KapLayout& L,
-                         uint8_t* ws, int k_cap, cudaStream_t st) {
-  const int B = s->batch, Hq = s->num_q_heads, Hk = s->num_kv_heads, N = s->seq_len;
-  const int P = s->page_size, Bq = s->q_block, nP = N / P, nQB = N / Bq;
-  const int R = Bq / k->q_sub, T = P / k->k_sub, G = Hq / Hk;
-  float* qhat = reinterpret_cast<float*>(ws + L.qhat_off);
-  float* khat = reinterpret_cast<float*>(ws + L.khat_off);
-  float* sc = scores ? scores : reinterpret_cast<float*>(ws + L.scores_off);
-  uint8_t* hr = hrm ? hrm : ws + L.hrm_off;
-
-  // K1
-  const long long n_qvec = (long long)B * Hq * (N / k->q_sub);
-  const long long n_kvec = (long long)B * Hk * nP * T;
-  const long long warps = n_qvec + n_kvec;
-  const long long blocks = (warps + 7) / 8;
-  if (blocks > 0x7fffffffll) return COSA_ERR_UNSUPPORTED;
-  kap_pool_kernel<D><<<(unsigned)blocks, 256, 0, st>>>(
-      reinterpret_cast<const __nv_bfloat16*>(q), reinterpret_cast<const __nv_bfloat16*>(k_pool),
-      page_table, qhat, khat, n_qvec, k->q_sub, n_kvec, k->k_sub, Hk, P, nP, s->pages_per_seq, T,
-      (int)khat_stride(s, k));
-  if (last_launch() != COSA_OK) return COSA_ERR_CUDA;
-
-  // K2
-  int hpc = 0;
-  for (int d = G; d >= 1; --d) {
-    if (G % d) continue;
-    if (d * R > 32) continue;
-    if (score_smem<D>(d, R, nP) > kScoreSmemLimit) continue;
-    hpc = d;
-    break;
-  }
-  if (hpc == 0) return COSA_ERR_UNSUPPORTED;
-  const size_t smem2 = score_smem<D>(hpc, R, nP);
-  const dim3 g2(nQB, B * Hk * (G / hpc));
-  const int kstride = (int)khat_stride(s, k);
-  cosa_status_t e2 =
-      hpc * R <= 16
-          ? launch_score<D, 16>(g2, smem2, st, qhat, khat, sc, hr, Hq, Hk, G, hpc, nQB, nP, kstride,
-                                R, T, k->q_sub, k->k_sub, P, Bq, s->softmax_scale)
-          : launch_score<D, 32>(g2, smem2, st, qhat, khat, sc, hr, Hq, Hk, G, hpc, nQB, nP, kstride,
-                                R, T, k->q_sub, k->k_sub, P, Bq, s->softmax_scale);
-  if (e2 != COSA_OK) return e2;
-
-  // K3
-  int npow2 = 1;
-  while (npow2 < nP) npow2 <<= 1;
-  size_t smem3 = (size_t)npow2 * 8 + (size_t)nP * 4;
-  if (smem3 > 200 * 1024) return COSA_ERR_UNSUPPORTED;
-  if (cudaFuncSetAttribute(kap_order_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)smem3) != cudaSuccess)
-    return COSA_ERR_CUDA;
-  dim3 g3(nQB, B * Hq);
-  kap_order_kernel<<<g3, ORDER_THREADS, smem3, st>>>(sc, hr, order, count, nQB, nP, Bq, P,
-                                                     k->budget, k->sink_pages, k->ascending, k_cap);
-  return last_launch();
 }
 
 // ---- tensor maps (TMA descriptors) ------------------------------------------------
@@ -211,7 +134,122 @@ bool make_map(CUtensorMap* m, const void* base, int D, int rows, long long z, in
   return r == CUDA_SUCCESS;
 }
 
+// fp32 [rows][D] as a 2-D tensor; box = 32 columns (128 bytes) x 128 rows, 128-byte swizzle.
+bool make_map_f32(CUtensorMap* m, const void* base, int D, long long rows) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)D * 4};
+  cuuint32_t box[2] = {32u, 128u};
+  cuuint32_t estr[2] = {1u, 1u};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(base), dims, strides,
+                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 constexpr unsigned long long kWaitTimeoutNs = 1000000000ull;  // 1 s without progress
+
+template <int D, int T>
+cosa_status_t launch_score_tc(const ScoreParams& prm, const CUtensorMap* maps, int grid,
+                              cudaStream_t st) {
+  using Cfg = ScoreCfg<D>;
+  auto kern = kap_score_tc<D, T>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)Cfg::SMEM_ALLOC) != cudaSuccess)
+    return COSA_ERR_CUDA;
+  kern<<<grid, 192, Cfg::SMEM_ALLOC, st>>>(maps[0], maps[1], maps[2], maps[3], prm);
+  return last_launch();
+}
+
+cosa_status_t launch_order(const cosa_shape_t* s, const cosa_kap_params_t* k, bool from_a,
+                           const float* scores, const uint8_t* hrm, const KapPageMax& pm,
+                           float* scores_out, uint8_t* hrm_out, int32_t* order, int32_t* count,
+                           int k_cap, cudaStream_t st) {
+  const int N = s->seq_len, P = s->page_size, Bq = s->q_block, nP = N / P, nQB = N / Bq;
+  int npow2 = 1;
+  while (npow2 < nP) npow2 <<= 1;
+  const size_t smem = (size_t)npow2 * 8 + (size_t)nP * 4;
+  if (smem > 200 * 1024) return COSA_ERR_UNSUPPORTED;
+  auto kern = from_a ? kap_order_kernel<true> : kap_order_kernel<false>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+      cudaSuccess)
+    return COSA_ERR_CUDA;
+  dim3 grid(nQB, s->batch * s->num_q_heads);
+  kern<<<grid, ORDER_THREADS, smem, st>>>(scores, hrm, pm, scores_out, hrm_out, order, count,
+                                          s->num_q_heads, nQB, nP, Bq, P, k->budget,
+                                          k->sink_pages, k->ascending, k_cap);
+  return last_launch();
+}
+
+template <int D>
+cosa_status_t launch_kap(const cosa_shape_t* s, const cosa_kap_params_t* k, const void* q,
+                         const void* k_pool, const int32_t* page_table, int32_t* order,
+                         int32_t* count, float* scores, uint8_t* hrm, const KapLayout& L,
+                         uint8_t* ws, int k_cap, cudaStream_t st) {
+  const int B = s->batch, Hq = s->num_q_heads, Hk = s->num_kv_heads, N = s->seq_len;
+  const int P = s->page_size, Bq = s->q_block, nP = N / P, nQB = N / Bq;
+  const int R = Bq / k->q_sub, T = P / k->k_sub, G = Hq / Hk;
+  float* q_hi = reinterpret_cast<float*>(ws + L.q_hi);
+  float* q_lo = reinterpret_cast<float*>(ws + L.q_lo);
+  float* k_hi = reinterpret_cast<float*>(ws + L.k_hi);
+  float* k_lo = reinterpret_cast<float*>(ws + L.k_lo);
+
+  // K1: pooling
+  const long long n_qvec = (long long)B * Hq * nQB * R;
+  const long long n_kvec = (long long)B * Hk * nP * T;
+  const long long blocks = (n_qvec + n_kvec + 7) / 8;
+  if (blocks > 0x7fffffffll) return COSA_ERR_UNSUPPORTED;
+  kap_pool_kernel<D><<<(unsigned)blocks, 256, 0, st>>>(
+      reinterpret_cast<const __nv_bfloat16*>(q), reinterpret_cast<const __nv_bfloat16*>(k_pool),
+      page_table, q_hi, q_lo, k_hi, k_lo, n_qvec, k->q_sub, n_kvec, k->k_sub, Hq, Hk, G, R, nQB,
+      P, nP, s->pages_per_seq, T);
+  if (last_launch() != COSA_OK) return COSA_ERR_CUDA;
+
+  // K2: scores + MaxPool on the tensor cores
+  ScoreParams sp;
+  std::memset(&sp, 0, sizeof(sp));
+  sp.a = reinterpret_cast<float*>(ws + L.a);
+  sp.row_max = reinterpret_cast<float*>(ws + L.row_max);
+  sp.row_arg = reinterpret_cast<int*>(ws + L.row_arg);
+  sp.group = G;
+  sp.R = R;
+  sp.T = T;
+  sp.num_q_blocks = nQB;
+  sp.q_block = Bq;
+  sp.page_size = P;
+  sp.q_sub = k->q_sub;
+  sp.k_sub = k->k_sub;
+  sp.rows_per_slab = nQB * G * R;
+  sp.keys_per_slab = nP * T;
+  sp.tiles_per_slab = (sp.rows_per_slab + 127) / 128;
+  sp.scale = s->softmax_scale;
+  sp.timeout_ns = kWaitTimeoutNs;
+  CUtensorMap maps[4];
+  if (!make_map_f32(&maps[0], q_hi, D, n_qvec) || !make_map_f32(&maps[1], q_lo, D, n_qvec) ||
+      !make_map_f32(&maps[2], k_hi, D, n_kvec) || !make_map_f32(&maps[3], k_lo, D, n_kvec))
+    return COSA_ERR_CUDA;
+  const long long grid2 = (long long)B * Hk * sp.tiles_per_slab;
+  if (grid2 > 0x7fffffffll) return COSA_ERR_UNSUPPORTED;
+  cosa_status_t e = COSA_ERR_UNSUPPORTED;
+  switch (T) {
+    case 1: e = launch_score_tc<D, 1>(sp, maps, (int)grid2, st); break;
+    case 2: e = launch_score_tc<D, 2>(sp, maps, (int)grid2, st); break;
+    case 4: e = launch_score_tc<D, 4>(sp, maps, (int)grid2, st); break;
+    case 8: e = launch_score_tc<D, 8>(sp, maps, (int)grid2, st); break;
+  }
+  if (e != COSA_OK) return e;
+
+  // K3: MaxNorm + HRM, budgeted selection, ordering
+  KapPageMax pm;
+  pm.a = sp.a;
+  pm.row_max = sp.row_max;
+  pm.row_arg = sp.row_arg;
+  pm.num_kv_heads = Hk;
+  pm.group = G;
+  pm.R = R;
+  return launch_order(s, k, true, nullptr, nullptr, pm, scores, hrm, order, count, k_cap, st);
+}
 
 template <int D, int P, bool DENSE>
 cosa_status_t launch_tc_t(const cosa_shape_t* s, const TcParams& prm, const void* q,
@@ -385,21 +423,10 @@ cosa_status_t cosa_kap_order(const cosa_shape_t* shape, const cosa_kap_params_t*
   if (e != COSA_OK) return e;
   if ((e = check_kap(shape, kap)) != COSA_OK) return e;
   if (!scores || !hrm || !order || !count) return COSA_ERR_INVALID_ARG;
-  const int N = shape->seq_len, P = shape->page_size, Bq = shape->q_block;
-  const int nP = N / P, nQB = N / Bq;
-  int npow2 = 1;
-  while (npow2 < nP) npow2 <<= 1;
-  size_t smem3 = (size_t)npow2 * 8 + (size_t)nP * 4;
-  if (smem3 > 200 * 1024) return COSA_ERR_UNSUPPORTED;
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  if (cudaFuncSetAttribute(kap_order_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)smem3) != cudaSuccess)
-    return COSA_ERR_CUDA;
-  dim3 g3(nQB, shape->batch * shape->num_q_heads);
-  kap_order_kernel<<<g3, ORDER_THREADS, smem3, st>>>(scores, hrm, order, count, nQB, nP, Bq, P,
-                                                     kap->budget, kap->sink_pages, kap->ascending,
-                                                     kcap_of(shape, kap));
-  return last_launch();
+  KapPageMax pm;
+  std::memset(&pm, 0, sizeof(pm));
+  return launch_order(shape, kap, false, scores, hrm, pm, nullptr, nullptr, order, count,
+                      kcap_of(shape, kap), reinterpret_cast<cudaStream_t>(stream));
 }
 
 cosa_status_t cosa_osk_attention(const cosa_shape_t* shape, const cosa_osk_params_t* osk,

@@ -113,8 +113,9 @@ int32_t cosa_version(void);
 cosa_status_t cosa_kap_kcap(const cosa_shape_t* shape, const cosa_kap_params_t* kap,
                             int32_t* k_cap);
 
-/* Bytes of device workspace cosa_kap_select needs (pooled queries and keys,
- * scores and HRM flags).  Host-only; no CUDA call. */
+/* Bytes of device workspace cosa_kap_select needs (pooled queries and keys as
+ * two TF32 terms each, the per-page maxima of every representative row, and
+ * each row's maximum and first page attaining it).  Host-only; no CUDA call. */
 cosa_status_t cosa_kap_workspace_size(const cosa_shape_t* shape, const cosa_kap_params_t* kap,
                                       size_t* bytes);
 
@@ -137,14 +138,14 @@ cosa_status_t cosa_kap_select(const cosa_shape_t* shape, const cosa_kap_params_t
                               void* workspace, size_t workspace_bytes, cosa_stream_t stream);
 
 /* Largest workspace (cosa_kap_workspace_size) that cosa_kap_select_noalloc
- * accepts: 64 MiB, enough for a 32K-token layer with 32 query heads. */
-#define COSA_KAP_NOALLOC_SCRATCH_BYTES (64u << 20)
+ * accepts: 128 MiB, enough for a 32K-token layer with 32 query heads. */
+#define COSA_KAP_NOALLOC_SCRATCH_BYTES (128u << 20)
 
 /* cosa_kap_select for callers that cannot allocate device memory.  The paper
  * has no counterpart: this is a packaging variant of the same Stage-1 kernels.
  * Some callers cannot call cudaMalloc or hand out a workspace at call time (a
  * runtime that owns the device allocator, a plan whose memory is fixed in
- * advance), so the pooled vectors, scores and flags go to a fixed 64 MiB array
+ * advance), so the pooled vectors and page maxima go to a fixed 128 MiB array
  * inside the library instead.  Every GPU on which the library's kernels load
  * holds that array until the process exits.  Arguments and results are those
  * of cosa_kap_select without the workspace; the caller still allocates q,

@@ -46,12 +46,15 @@ def test_kcap_matches_oracle(N, P, Bq, budget, sink):
     assert C.cosa_kap_kcap(s, k) == O.k_cap(N, Bq, P, sink, budget)
 
 
-def test_workspace_size_covers_pooled_vectors_and_scores():
+def test_workspace_size_covers_pooled_vectors_and_page_maxima():
     s = C.Shape(1, 32, 8, 131072, 128, 64, 128)
     k = C.KapParams(0.2, q_sub=32, k_sub=16)
-    need = (32 * 4096 * 128 * 4) + (8 * 8192 * 128 * 4) + 32 * 1024 * 2048 * 5
+    rows = 32 * 1024 * 4                       # representatives
+    keys = 8 * 2048 * 4                        # sub-keys
+    tri = sum(O.causal_pages(qb, 128, 64) for qb in range(1024))
+    need = 2 * rows * 128 * 4 + 2 * keys * 128 * 4 + 8 * 16 * tri * 4 + rows * 8
     got = C.cosa_kap_workspace_size(s, k)
-    assert need <= got <= need + 4 * 256
+    assert need <= got <= need + 8 * 256
 
 
 def _status(fn):
