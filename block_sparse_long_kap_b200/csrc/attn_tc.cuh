@@ -5,37 +5,46 @@
 // remapping"; in-kernel skip from the page's local max vs the running max;
 // computed pages get the full softmax + PV.)
 //
-// One CTA (384 threads) per (b, h_q, q-block) tile of up to 128 query rows:
-//   warp 0      TMA producer: the Q tile once, then K of every listed page, in
-//               list order, into a KS-stage ring (page table gives the
-//               physical page; no multicast).
-//   warp 1      QK^T issuer (one thread): S_j = Q K_j^T into one of SB TMEM
-//               buffers, in list order.
-//   warp 2      TMA producer for V: loads V_j only for pages the vote keeps,
-//               so a skipped page costs its K tile and one QK^T, nothing more.
-//   warp 3      PV issuer (one thread): for each kept page, once its P and V
-//               tiles are ready, O += P_j V_j into the TMEM accumulator.  With
-//               two issuing threads a late V never stalls QK^T.
-//   warps 4-11  softmax, two warpgroups: warpgroup h (0/1) owns columns
-//               [h P/2, (h+1) P/2) of every S tile and [h D/2, (h+1) D/2) of O;
-//               thread (warp % 4, lane) owns query row 32 (warp % 4) + lane,
-//               which is its TMEM lane.  Per page: read the half row of S,
-//               mask the causal diagonal, take the half-row max, then one
-//               barrier round among the 256 softmax threads exchanges the
-//               half maxima and the votes.  The skip rule "some row has
-//               (page max - running max) >= log2 eps" is decided exactly on
-//               half rows, because max(a, b) - m >= t  <=>  a - m >= t or
-//               b - m >= t.  The first listed page is always kept.  For kept
-//               pages each thread writes P = exp2(s - m_ref) (bf16) for its
-//               half row into a swizzled shared-memory tile; m_ref, the
-//               exponent base, moves only when the running max passes it by
-//               more than 2^8 (O and l are then rescaled in TMEM), which keeps
-//               the result exact.
-// Decisions reach the V producer and the PV issuer as sequence-tagged words in
-// a shared-memory ring; their progress counters give the ring back-pressure.
-// Every wait is bounded: on timeout the CTA records COSA_ERR_TIMEOUT in the
-// status word, drains what it issued, frees TMEM and exits; a timed-out CTA
-// makes every later CTA of the launch exit at once.
+// One CTA (384 threads) per (b, h_q, q-block) tile of up to 128 query rows.
+// Listed pages are taken in list order in groups of 128 keys (two pages of 64
+// keys, or one of 128): one QK^T of N = 128 per group, into one of three S
+// buffers in TMEM.
+//   warps 0, 1  K producers: group g is loaded by warp g % 2 into ring slot
+//               g % KG, so two TMA streams run side by side (warp 0 also loads
+//               Q).  The physical page comes from the page table; no multicast.
+//   warp 2      V producer: loads V of the kept pages only, once the vote has
+//               kept them, so a skipped page costs its K tile and its share of
+//               one QK^T, nothing more.
+//   warp 3      MMA issuer (one thread, polling): QK^T of the next group when
+//               its K tile and an S buffer are ready, PV of the next kept page
+//               when its P and V are ready.
+//   warps 4-7,  softmax, two warpgroups taking the groups in turn (even groups
+//   8-11        warpgroup 0, odd groups warpgroup 1).  Thread (warp % 4, lane)
+//               owns query row 32 (warp % 4) + lane, which is its TMEM lane,
+//               and reads the whole row of S.  The skip rule "page j is skipped
+//               when no row has (page max - running max) >= log2 eps" is first
+//               voted against the running max this warpgroup last saw: the
+//               running max only grows, so a page skipped against an older
+//               value is skipped against the current one, and an all-skip group
+//               is settled without waiting for the other warpgroup.  A group
+//               with a page that may be kept (and the first group, and every
+//               group of dense attention) waits until the groups before it are
+//               settled, reads the exact running max and exponent base of every
+//               row from shared memory and votes again; its pages are then
+//               published in list order.  One barrier round among the 128
+//               threads of a warpgroup carries each vote, for the group's second
+//               page under both outcomes of the first.  The first listed page is
+//               always kept.  For kept pages each thread writes
+//               P = exp2(s - m_ref) (bf16) for its row over the page's S
+//               columns; m_ref, the exponent base, moves only when the running
+//               max passes it by more than 2^8 (O and l are then rescaled),
+//               which keeps the result exact.
+// Kept pages reach the V producer and the MMA issuer through a shared-memory
+// queue that carries each page's TMA coordinate and P location; the
+// consumers' progress counters give it back-pressure.  Every wait is bounded: on
+// timeout the CTA records COSA_ERR_TIMEOUT in the status word, drains what it
+// issued, frees TMEM and exits; a timed-out CTA makes every later CTA of the
+// launch exit at once.
 #pragma once
 
 #include "common.cuh"
@@ -59,38 +68,45 @@ struct TcParams {
 template <int D, int P>
 struct TcCfg {
   static constexpr int QB = 128;                  // MMA M (rows per tile, padded)
-  static constexpr int NT = 384;                  // 4 role warps + 2 softmax warpgroups
-  static constexpr int HP = P / 2;                // S columns per softmax thread
-  static constexpr int HD = D / 2;                // O columns per softmax thread
-  static constexpr int KS = (P == 64) ? 6 : 2;    // K ring stages
-  static constexpr int VS = 2;                    // V ring stages
-  static constexpr int PS = (P == 64) ? 2 : 1;    // P tile ring stages
-  static constexpr int SB = (P == 64) ? 4 : 3;    // S buffers in TMEM
-  static constexpr int DS = 64;                   // decision ring (words)
+  static constexpr int NT = 384;                  // 12 warps
+  static constexpr int GP = 128 / P;              // pages per QK group (128 keys)
   static constexpr uint32_t Q_BYTES = QB * D * 2;
-  static constexpr uint32_t KV_BYTES = P * D * 2;
-  static constexpr uint32_t P_BYTES = QB * P * 2;
+  static constexpr uint32_t KV_BYTES = P * D * 2; // one page of K or of V
+  static constexpr uint32_t KG_BYTES = GP * KV_BYTES;
+  static constexpr int KG = (D == 128) ? 3 : 4;   // K ring slots (groups)
+  static constexpr int VS0 = (int)(65536u / KV_BYTES);
+  static constexpr int VS = VS0 > 6 ? 6 : VS0;    // V ring slots (pages)
+  static constexpr int SBG = 3;                   // S group buffers in TMEM, 128 columns each
+  static constexpr int COL_O = SBG * 128;         // O accumulator (D columns)
+  static constexpr int PF = 8;                    // P-ready barrier ring (kept pages)
+  static constexpr int PD = 8;                    // PV-done barrier ring (kept pages)
+  static constexpr int KQ = 64;                   // kept-page queue entries
+  static constexpr int TMEM_COLS = 512;
   static constexpr uint32_t OFF_Q = 0;
   static constexpr uint32_t OFF_K = OFF_Q + Q_BYTES;
-  static constexpr uint32_t OFF_V = OFF_K + KS * KV_BYTES;
-  static constexpr uint32_t OFF_P = OFF_V + VS * KV_BYTES;
-  static constexpr uint32_t OFF_BAR = OFF_P + PS * P_BYTES;
-  // q, k_full/empty, v_full/empty, s_full/free, p_full/empty, done (QK), done (PV)
-  static constexpr int NBAR = 1 + 2 * KS + 2 * VS + 2 * SB + 2 * PS + 2;
+  static constexpr uint32_t OFF_V = OFF_K + KG * KG_BYTES;
+  static constexpr uint32_t OFF_BAR = OFF_V + VS * KV_BYTES;
+  // q, k_full/empty, v_full/empty, s_full/free, p_full, pv_done, done
+  static constexpr int NBAR = 1 + 2 * KG + 2 * VS + 2 * SBG + PF + PD + 1;
   static constexpr uint32_t OFF_MISC = (OFF_BAR + NBAR * 8 + 127) & ~127u;  // vector-aligned
-  // misc: +0 TMEM address, +4 abort flag, +8 PV progress, +12 V progress,
-  //       +16 votes [2 rounds][2 parities][8], +256 decision words [DS],
-  //       +512 half-row maxima [2 parities][2 pages][2 halves][128],
-  //       +4608 half-row sums [2][128]
-  static constexpr uint32_t MISC_BYTES = 5632;
+  // misc: +0 TMEM address, +4 abort flag, +8 kept count (P location published),
+  //       +12 final kept count (-1 while the votes run), +16 V progress,
+  //       +20 warpgroups finished, +36 PV progress, +40 kept count (TMA coordinate
+  //       published), +48 votes [2 wg][2][4], +128 kept queue [KQ] {TMA coordinate,
+  //       P column | last << 15}, +640 settled state rows [128] {m_run, m_ref},
+  //       +1664 last settled group per softmax warp [8], +2688 final rows [2][128] {l, m_ref}
+  static constexpr uint32_t M_STATE = 640, M_SETTLED = 1664, M_FIN = 2688;
+  static constexpr uint32_t MISC_BYTES = M_FIN + 2 * 128 * 8;
   static constexpr uint32_t SMEM = OFF_MISC + MISC_BYTES;
   static constexpr uint32_t SMEM_ALLOC = SMEM + 1024;  // 1024-byte alignment slack
-  static constexpr int COL_O = SB * P;
-  static constexpr int TMEM_COLS = (SB * P + D <= 256) ? 256 : 512;
-  static_assert(SB * P + D <= 512, "TMEM budget");
+  static_assert(COL_O + D <= TMEM_COLS, "TMEM budget");
+  static_assert(VS >= 2 && KG >= 2, "ring depths");
+  static_assert(PF >= 2 * SBG + 1 && PD >= 2 * SBG + 1, "barrier rings cover the kept pages in flight");
   static_assert(SMEM_ALLOC <= 227 * 1024, "shared memory budget");
-  static_assert(256 + 4 * DS <= 512, "decision ring fits its slot");
   static_assert(OFF_MISC % 128 == 0, "16-byte vector access to the vote words");
+  static_assert(KV_BYTES % 1024 == 0, "tiles stay 1024-byte aligned for the 128-byte swizzle");
+  static_assert(48 + 64 <= 128 && 128 + 8 * KQ <= M_STATE, "vote words and kept queue fit");
+  static_assert(M_STATE + 128 * 8 <= M_SETTLED && M_SETTLED + 8 * 4 <= M_FIN, "state rows and flags fit");
 };
 
 constexpr float kRescaleLog2 = 8.0f;  // m_ref trails the running max by < 2^8
@@ -101,36 +117,39 @@ __global__ void __launch_bounds__(384, 1)
                    const __grid_constant__ CUtensorMap tm_v, const TcParams prm) {
   using C = TcCfg<D, P>;
   using namespace tc;
-  constexpr int HP = C::HP, HD = C::HD;
+  constexpr int GP = C::GP;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t sraw = static_cast<uint32_t>(__cvta_generic_to_shared(smem_raw));
   const uint32_t sb0 = (sraw + 1023u) & ~1023u;
   uint8_t* sg = smem_raw + (sb0 - sraw);
-  const uint32_t sQ = sb0 + C::OFF_Q, sK = sb0 + C::OFF_K, sV = sb0 + C::OFF_V,
-                 sP = sb0 + C::OFF_P;
+  const uint32_t sQ = sb0 + C::OFF_Q, sK = sb0 + C::OFF_K, sV = sb0 + C::OFF_V;
   const uint32_t bar = sb0 + C::OFF_BAR;
   const uint32_t b_q = bar;
   auto b_kfull = [&](int s) { return bar + 8u * (1 + s); };
-  auto b_kempty = [&](int s) { return bar + 8u * (1 + C::KS + s); };
-  auto b_vfull = [&](int s) { return bar + 8u * (1 + 2 * C::KS + s); };
-  auto b_vempty = [&](int s) { return bar + 8u * (1 + 2 * C::KS + C::VS + s); };
-  auto b_sfull = [&](int s) { return bar + 8u * (1 + 2 * C::KS + 2 * C::VS + s); };
-  auto b_sfree = [&](int s) { return bar + 8u * (1 + 2 * C::KS + 2 * C::VS + C::SB + s); };
-  auto b_pfull = [&](int s) { return bar + 8u * (1 + 2 * C::KS + 2 * C::VS + 2 * C::SB + s); };
-  auto b_pempty = [&](int s) {
-    return bar + 8u * (1 + 2 * C::KS + 2 * C::VS + 2 * C::SB + C::PS + s);
+  auto b_kempty = [&](int s) { return bar + 8u * (1 + C::KG + s); };
+  auto b_vfull = [&](int s) { return bar + 8u * (1 + 2 * C::KG + s); };
+  auto b_vempty = [&](int s) { return bar + 8u * (1 + 2 * C::KG + C::VS + s); };
+  auto b_sfull = [&](int s) { return bar + 8u * (1 + 2 * C::KG + 2 * C::VS + s); };
+  auto b_sfree = [&](int s) { return bar + 8u * (1 + 2 * C::KG + 2 * C::VS + C::SBG + s); };
+  auto b_pfull = [&](int s) { return bar + 8u * (1 + 2 * C::KG + 2 * C::VS + 2 * C::SBG + s); };
+  auto b_pvdone = [&](int s) {
+    return bar + 8u * (1 + 2 * C::KG + 2 * C::VS + 2 * C::SBG + C::PF + s);
   };
-  const uint32_t b_done_s = bar + 8u * (C::NBAR - 2);
-  const uint32_t b_done_pv = bar + 8u * (C::NBAR - 1);
+  const uint32_t b_done = bar + 8u * (C::NBAR - 1);
   uint8_t* misc = sg + C::OFF_MISC;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(misc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 4);
-  volatile int* pv_pos = reinterpret_cast<volatile int*>(misc + 8);
-  volatile int* v_pos = reinterpret_cast<volatile int*>(misc + 12);
-  volatile int* votes = reinterpret_cast<volatile int*>(misc + 16);               // [2][2][8]
-  volatile uint32_t* dec_word = reinterpret_cast<volatile uint32_t*>(misc + 256);  // [DS]
-  volatile float* hmax = reinterpret_cast<volatile float*>(misc + 512);     // [2][2][2][128]
-  volatile float* hsum = reinterpret_cast<volatile float*>(misc + 4608);    // [2][128]
+  volatile int* kq_count = reinterpret_cast<volatile int*>(misc + 8);
+  volatile int* kq_final = reinterpret_cast<volatile int*>(misc + 12);
+  volatile int* v_pos = reinterpret_cast<volatile int*>(misc + 16);
+  int* wg_done = reinterpret_cast<int*>(misc + 20);
+  volatile int* pv_pos = reinterpret_cast<volatile int*>(misc + 36);
+  volatile int* vq_count = reinterpret_cast<volatile int*>(misc + 40);
+  volatile int* votes = reinterpret_cast<volatile int*>(misc + 48);     // [2][2][4]
+  volatile int* settled = reinterpret_cast<volatile int*>(misc + C::M_SETTLED);  // [8]
+  volatile int2* kq = reinterpret_cast<volatile int2*>(misc + 128);     // [KQ]
+  volatile float2* st_rows = reinterpret_cast<volatile float2*>(misc + C::M_STATE);  // [128]
+  volatile float2* fin_rows = reinterpret_cast<volatile float2*>(misc + C::M_FIN);    // [2][128]
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   // a CTA that ran out of time anywhere in this launch stops the others early
@@ -160,32 +179,43 @@ __global__ void __launch_bounds__(384, 1)
       n_list = 0;
     }
   }
+  const int n_groups = (n_list + GP - 1) / GP;
   const int32_t* ptab = prm.page_table + (long long)b * prm.pages_per_seq;
   auto page_at = [&](int j) { return DENSE ? j : __ldg(olist + j); };
+  // TMA z coordinate of a logical page in the [phys page][kv head] pools
+  auto coord_of = [&](int page) { return __ldg(ptab + page) * prm.num_kv_heads + hk; };
 
   // ---- setup
   if (tid == 0) {
     mbar_init(b_q, 1);
-    for (int s = 0; s < C::KS; ++s) { mbar_init(b_kfull(s), 1); mbar_init(b_kempty(s), 1); }
+    for (int s = 0; s < C::KG; ++s) { mbar_init(b_kfull(s), 1); mbar_init(b_kempty(s), 1); }
     for (int s = 0; s < C::VS; ++s) { mbar_init(b_vfull(s), 1); mbar_init(b_vempty(s), 1); }
-    for (int s = 0; s < C::SB; ++s) { mbar_init(b_sfull(s), 1); mbar_init(b_sfree(s), 8); }
-    for (int s = 0; s < C::PS; ++s) { mbar_init(b_pfull(s), 8); mbar_init(b_pempty(s), 1); }
-    mbar_init(b_done_s, 1);
-    mbar_init(b_done_pv, 1);
+    for (int s = 0; s < C::SBG; ++s) { mbar_init(b_sfull(s), 1); mbar_init(b_sfree(s), 1); }
+    for (int s = 0; s < C::PF; ++s) mbar_init(b_pfull(s), 4);
+    for (int s = 0; s < C::PD; ++s) mbar_init(b_pvdone(s), 1);
+    mbar_init(b_done, 1);
     *abort_flag = 0;
-    *pv_pos = 0;
+    *kq_count = 0;
+    *kq_final = -1;
     *v_pos = 0;
-    for (int s = 0; s < C::DS; ++s) dec_word[s] = 0xFFFFFFFFu;
+    *pv_pos = 0;
+    *vq_count = 0;
+    *wg_done = 0;
+    for (int w = 0; w < 8; ++w) settled[w] = -1;
+    for (int r = 0; r < 128; ++r) {
+      st_rows[r].x = -INFINITY;
+      st_rows[r].y = -INFINITY;
+    }
     fence_barrier_init();
   }
-  if (warp == 1) {
+  if (warp == 3) {
     tmem_alloc(sb0 + C::OFF_MISC, C::TMEM_COLS);
     tmem_relinquish();
   }
-  if (prm.q_block < C::QB && warp >= 4) {
+  if (prm.q_block < C::QB && warp >= 4 && warp < 8) {
     // rows past the q-block are padding: zero them once (the TMA box fills the rest)
     const int pad = C::QB - prm.q_block;
-    for (int i = tid - 128; i < pad * (D / 64) * 8; i += 256) {
+    for (int i = tid - 128; i < pad * (D / 64) * 8; i += 128) {
       const int chunk = i & 7, r = prm.q_block + (i >> 3) % pad, kb = (i >> 3) / pad;
       st_shared_v4(sQ + kb * (C::QB * 128) + r * 128 + chunk * 16, 0u, 0u, 0u, 0u);
     }
@@ -200,43 +230,54 @@ __global__ void __launch_bounds__(384, 1)
     *abort_flag = 1;
     set_status(COSA_ERR_TIMEOUT);
   };
-  // bounded blocking wait on an mbarrier phase; false on timeout or abort
+  auto timed_out = [&](uint64_t t0) {
+    return *(volatile int*)&g_status == COSA_ERR_TIMEOUT || globaltimer_ns() - t0 > tmo;
+  };
+  // bounded blocking wait on an mbarrier phase; false on timeout or abort.  The
+  // suspend hint lets a waiting warp sleep instead of taking issue slots.
   auto wait = [&](uint32_t bar_addr, uint32_t parity) -> bool {
     if (mbar_try_wait(bar_addr, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
-    uint32_t spins = 0;
     while (!mbar_try_wait_sleep(bar_addr, parity, 20000u)) {
       if (*abort_flag) return false;
-      if ((++spins & 3u) == 0 &&
-          (*(volatile int*)&g_status == COSA_ERR_TIMEOUT || globaltimer_ns() - t0 > tmo)) {
+      if (timed_out(t0)) {
         give_up();
         return false;
       }
     }
     return true;
   };
-  // bounded wait for the decision on page i; returns -1 on timeout, else 0/1
-  auto decision = [&](int i) -> int {
-    const uint32_t want = (uint32_t)i << 1;
-    uint32_t w = dec_word[i % C::DS];
-    if ((w & ~1u) == want) return (int)(w & 1u);
+  // the same, waited on by lane 0 for the whole warp
+  auto wait_warp = [&](uint32_t bar_addr, uint32_t parity) -> bool {
+    int okl = 1;
+    if (lane == 0) okl = wait(bar_addr, parity) ? 1 : 0;
+    return __shfl_sync(0xffffffffu, okl, 0) != 0;
+  };
+
+  // bounded wait (one thread) until counter cnt passes kept page c: 1 = it exists,
+  // 0 = the list ended before it, -1 = abort
+  auto kept_ready = [&](volatile int* cnt, int c) -> int {
+    if (*cnt > c) return 1;
     const uint64_t t0 = globaltimer_ns();
-    uint32_t spins = 0;
-    while (((w = dec_word[i % C::DS]) & ~1u) != want) {
+    uint32_t spins = 0, nap = 64;
+    while (true) {
+      const int f = *kq_final;
+      if (*cnt > c) return 1;
+      if (f >= 0) return 0;
       if (*abort_flag) return -1;
-      if ((++spins & 63u) == 0 &&
-          (*(volatile int*)&g_status == COSA_ERR_TIMEOUT || globaltimer_ns() - t0 > tmo)) {
+      if ((++spins & 15u) == 0 && timed_out(t0)) {
         give_up();
         return -1;
       }
-      __nanosleep(64);  // leave the issue slots to the softmax warps sharing this scheduler
+      __nanosleep(nap);
+      nap = min(nap * 2, 512u);
     }
-    return (int)(w & 1u);
   };
 
-  if (warp == 0) {
-    // ================= Q / K producer (lane 0 issues; the warp prefetches page ids)
-    if (lane == 0) {
+  if (warp < 2) {
+    // ================= K producers: groups g = warp, warp + 2, ... ==============
+    const int kp = warp;
+    if (kp == 0 && lane == 0) {
       prefetch_tmap(&tm_q);
       prefetch_tmap(&tm_k);
       mbar_arrive_expect_tx(b_q, (uint32_t)((D / 64) * prm.q_block * 128));
@@ -244,359 +285,534 @@ __global__ void __launch_bounds__(384, 1)
       for (int kb = 0; kb < D / 64; ++kb)
         tma_load_3d(sQ + kb * (C::QB * 128), &tm_q, b_q, kb * 64, row0, (int)bh);
     }
-    int issued = 0;
+    int last = -1;  // last group this warp issued
     bool ok = true;
-    for (int base = 0; ok && base < n_list; base += 32) {
-      const int jl = base + lane;
-      const int cz_l = jl < n_list ? ptab[page_at(jl)] * prm.num_kv_heads + hk : 0;
-      const int nb = min(32, n_list - base);
-      for (int jj = 0; jj < nb; ++jj) {
-        const int j = base + jj;
-        const int cz = __shfl_sync(0xffffffffu, cz_l, jj);
-        const int s = j % C::KS;
-        if (j >= C::KS) {
-          ok = __all_sync(0xffffffffu, wait(b_kempty(s), ((j / C::KS) - 1) & 1));
+    // lane l holds the coordinate of page l % GP of this warp's group m0 + l / GP
+    for (int m0 = 0; ok && kp + 2 * m0 < n_groups; m0 += 32 / GP) {
+      int cz_l = 0;
+      {
+        const int gl = kp + 2 * (m0 + lane / GP);
+        const int jl = gl * GP + lane % GP;
+        if (gl < n_groups && jl < n_list) cz_l = coord_of(page_at(jl));
+      }
+      for (int mm = 0; mm < 32 / GP; ++mm) {
+        const int g = kp + 2 * (m0 + mm);
+        if (g >= n_groups) break;
+        const int s = g % C::KG;
+        if (g >= C::KG) {
+          ok = wait_warp(b_kempty(s), ((g / C::KG) - 1) & 1);
           if (!ok) break;
         }
-        if (lane == 0) {
-          mbar_arrive_expect_tx(b_kfull(s), C::KV_BYTES);
+        const int nb = min(GP, n_list - g * GP);
+        int cz[GP];
 #pragma unroll
-          for (int kb = 0; kb < D / 64; ++kb)
-            tma_load_3d(sK + s * C::KV_BYTES + kb * (P * 128), &tm_k, b_kfull(s), kb * 64, 0, cz);
+        for (int t = 0; t < GP; ++t) cz[t] = __shfl_sync(0xffffffffu, cz_l, mm * GP + t);
+        if (lane == 0) {
+          mbar_arrive_expect_tx(b_kfull(s), (uint32_t)nb * C::KV_BYTES);
+#pragma unroll
+          for (int t = 0; t < GP; ++t)
+            if (t < nb)
+#pragma unroll
+              for (int kb = 0; kb < D / 64; ++kb)
+                tma_load_3d(sK + s * C::KG_BYTES + kb * (GP * P * 128) + t * (P * 128), &tm_k,
+                            b_kfull(s), kb * 64, 0, cz[t]);
         }
-        ++issued;
+        last = g;
         __syncwarp();
       }
     }
     if (lane == 0 && *abort_flag) {  // drain what was issued and never consumed
       const uint64_t t0 = globaltimer_ns();
-      while (!mbar_try_wait(b_q, 0) && globaltimer_ns() - t0 < tmo) {}
-      for (int j = max(0, issued - C::KS); j < issued; ++j)
-        while (!mbar_try_wait(b_kfull(j % C::KS), (j / C::KS) & 1) &&
+      if (kp == 0)
+        while (!mbar_try_wait(b_q, 0) && globaltimer_ns() - t0 < tmo) {}
+      for (int g = last; g >= 0 && g > last - 2 * C::KG; g -= 2)
+        while (!mbar_try_wait(b_kfull(g % C::KG), (g / C::KG) & 1) &&
                globaltimer_ns() - t0 < tmo) {}
     }
   } else if (warp == 2) {
-    // ================= V producer: only pages the vote keeps =================
+    // ================= V producer: kept pages in list order ======================
     if (lane == 0) prefetch_tmap(&tm_v);
-    int vc = 0;
+    int last = -1;
     bool ok = true;
-    for (int base = 0; ok && base < n_list; base += 32) {
-      const int il = base + lane;
-      const int cz_l = il < n_list ? ptab[page_at(il)] * prm.num_kv_heads + hk : 0;
-      const int nb = min(32, n_list - base);
-      for (int ii = 0; ii < nb; ++ii) {
-        const int i = base + ii;
-        const int cz = __shfl_sync(0xffffffffu, cz_l, ii);
-        if (!DENSE && i > 0) {  // page 0 is always kept: its V goes out before the vote
-          const int d = decision(i);
-          ok = __all_sync(0xffffffffu, d >= 0);
-          if (!ok) break;
-          if (lane == 0) *v_pos = i + 1;
-          if (d == 0) continue;
-        }
-        const int s = vc % C::VS;
-        if (vc >= C::VS) {
-          ok = __all_sync(0xffffffffu, wait(b_vempty(s), ((vc / C::VS) - 1) & 1));
-          if (!ok) break;
-        }
+    int cz_l = 0;
+    for (int c = 0; ok; ++c) {
+      int cz;
+      if (DENSE) {
+        if (c >= n_list) break;
+        if ((c & 31) == 0) cz_l = c + lane < n_list ? coord_of(c + lane) : 0;
+        cz = __shfl_sync(0xffffffffu, cz_l, c & 31);
+      } else {
+        int r = 0, e = 0;
         if (lane == 0) {
-          mbar_arrive_expect_tx(b_vfull(s), C::KV_BYTES);
-#pragma unroll
-          for (int kb = 0; kb < D / 64; ++kb)
-            tma_load_3d(sV + s * C::KV_BYTES + kb * (P * 128), &tm_v, b_vfull(s), kb * 64, 0, cz);
+          r = kept_ready(vq_count, c);
+          if (r > 0) {
+            __threadfence_block();
+            e = kq[c % C::KQ].x;
+            *v_pos = c + 1;  // queue entry c has been read
+          }
         }
-        ++vc;
-        __syncwarp();
-        if (!DENSE && i == 0) {
-          ok = __all_sync(0xffffffffu, decision(0) >= 0);
-          if (!ok) break;
-          if (lane == 0) *v_pos = 1;
-        }
+        r = __shfl_sync(0xffffffffu, r, 0);
+        if (r < 0) ok = false;
+        if (r <= 0) break;
+        cz = __shfl_sync(0xffffffffu, e, 0);
       }
+      const int s = c % C::VS;
+      if (c >= C::VS) {
+        ok = wait_warp(b_vempty(s), ((c / C::VS) - 1) & 1);
+        if (!ok) break;
+      }
+      if (lane == 0) {
+        mbar_arrive_expect_tx(b_vfull(s), C::KV_BYTES);
+#pragma unroll
+        for (int kb = 0; kb < D / 64; ++kb)
+          tma_load_3d(sV + s * C::KV_BYTES + kb * (P * 128), &tm_v, b_vfull(s), kb * 64, 0, cz);
+      }
+      last = c;
+      __syncwarp();
     }
     if (lane == 0 && *abort_flag) {
       const uint64_t t0 = globaltimer_ns();
-      for (int c = max(0, vc - C::VS); c < vc; ++c)
+      for (int c = last; c >= 0 && c > last - C::VS; --c)
         while (!mbar_try_wait(b_vfull(c % C::VS), (c / C::VS) & 1) &&
                globaltimer_ns() - t0 < tmo) {}
     }
-  } else if (warp == 1) {
-    if (lane == 0) {
-      // ================= QK^T issuer, list order =================
-      constexpr uint32_t ID_QK = idesc_bf16_f32(128, P, 0);
-      bool ok = wait(b_q, 0);
-      for (int j = 0; ok && j < n_list; ++j) {
-        const int ks = j % C::KS, sbuf = j % C::SB;
-        if (!wait(b_kfull(ks), (j / C::KS) & 1)) break;
-        if (j >= C::SB && !wait(b_sfree(sbuf), ((j / C::SB) - 1) & 1)) break;
-        tc_fence_after();
-#pragma unroll
-        for (int k = 0; k < D / 16; ++k) {
-          const uint64_t a = smem_desc_sw128(sQ + (k >> 2) * (C::QB * 128) + (k & 3) * 32, 16, 1024);
-          const uint64_t bd =
-              smem_desc_sw128(sK + ks * C::KV_BYTES + (k >> 2) * (P * 128) + (k & 3) * 32, 16, 1024);
-          mma_bf16_ss(tmem + sbuf * P, a, bd, ID_QK, k > 0 ? 1u : 0u);
-        }
-        mma_commit(b_kempty(ks));
-        mma_commit(b_sfull(sbuf));
-      }
-      // every issued MMA completes before teardown frees TMEM
-      mma_commit(b_done_s);
-      const uint64_t t0 = globaltimer_ns();
-      while (!mbar_try_wait(b_done_s, 0) && globaltimer_ns() - t0 < tmo) {}
-    }
   } else if (warp == 3) {
     if (lane == 0) {
-      // ================= PV issuer, kept pages in list order =================
+      // ================= MMA issuer: QK^T per group, PV per kept page =============
+      constexpr uint32_t ID_FULL = idesc_bf16_f32(128, 128, 0);
+      constexpr uint32_t ID_PAGE = idesc_bf16_f32(128, P, 0);  // a lone last page
       constexpr uint32_t ID_PV = idesc_bf16_f32(128, D, 1);
-      uint8_t* slog = prm.skip_log ? prm.skip_log + (bh * prm.num_q_blocks + qb) * prm.k_cap : nullptr;
-      int cpv = 0;
-      for (int i = 0; i < n_list; ++i) {
-        if (!DENSE) {
-          const int d = decision(i);
-          if (d < 0) break;
-          *pv_pos = i + 1;
-          if (slog) slog[i] = d ? 0 : 1;
-          if (d == 0) continue;
-        }
-        const int vs = cpv % C::VS, ps = cpv % C::PS;
-        if (!wait(b_vfull(vs), (cpv / C::VS) & 1)) break;
-        if (!wait(b_pfull(ps), (cpv / C::PS) & 1)) break;
-        tc_fence_after();
+      bool ok = wait(b_q, 0);
+      int g = 0, c = 0, pv_end = DENSE ? n_list : -1;
+      uint64_t t_idle = globaltimer_ns();
+      uint32_t spins = 0, nap = 32;
+      while (ok) {
+        bool did = false;
+        if (g < n_groups) {
+          const int ks = g % C::KG, sbuf = g % C::SBG;
+          if (mbar_test_wait(b_kfull(ks), (g / C::KG) & 1) &&
+              (g < C::SBG || mbar_test_wait(b_sfree(sbuf), ((g / C::SBG) - 1) & 1))) {
+            tc_fence_after();
+            const uint32_t id = (g * GP + GP <= n_list) ? ID_FULL : ID_PAGE;
 #pragma unroll
-        for (int k = 0; k < P / 16; ++k) {
-          const uint64_t a = smem_desc_sw128(
-              sP + ps * C::P_BYTES + (k >> 2) * (C::QB * 128) + (k & 3) * 32, 16, 1024);
-          const uint64_t bd = smem_desc_sw128(sV + vs * C::KV_BYTES + k * 16 * 128, P * 128, 1024);
-          mma_bf16_ss(tmem + C::COL_O, a, bd, ID_PV, (cpv > 0 || k > 0) ? 1u : 0u);
+            for (int k = 0; k < D / 16; ++k) {
+              const uint64_t a =
+                  smem_desc_sw128(sQ + (k >> 2) * (C::QB * 128) + (k & 3) * 32, 16, 1024);
+              const uint64_t bd = smem_desc_sw128(
+                  sK + ks * C::KG_BYTES + (k >> 2) * (GP * P * 128) + (k & 3) * 32, 16, 1024);
+              mma_bf16_ss(tmem + sbuf * 128, a, bd, id, k > 0 ? 1u : 0u);
+            }
+            mma_commit(b_kempty(ks));
+            mma_commit(b_sfull(sbuf));
+            ++g;
+            did = true;
+          }
         }
-        mma_commit(b_vempty(vs));
-        mma_commit(b_pempty(ps));
-        ++cpv;
+        if (!DENSE && pv_end < 0) {
+          const int f = *kq_final;  // read before the count: the count is final once f >= 0
+          if (f >= 0) pv_end = f;
+        }
+        if (pv_end < 0 || c < pv_end) {
+          bool avail = true;
+          int col, lastg;
+          if (DENSE) {
+            const int t = c % GP;
+            col = ((c / GP) % C::SBG) * 128 + t * P;
+            lastg = (t == GP - 1 || c == n_list - 1) ? 1 : 0;
+          } else {
+            avail = *kq_count > c;
+            int info = 0;
+            if (avail) {
+              __threadfence_block();
+              info = kq[c % C::KQ].y;
+            }
+            col = info & 0x7fff;
+            lastg = info >> 15;
+          }
+          const int vs = c % C::VS, pf = c % C::PF;
+          if (avail && mbar_test_wait(b_vfull(vs), (c / C::VS) & 1) &&
+              mbar_test_wait(b_pfull(pf), (c / C::PF) & 1)) {
+            tc_fence_after();
+#pragma unroll
+            for (int k = 0; k < P / 16; ++k) {
+              const uint64_t bd =
+                  smem_desc_sw128(sV + vs * C::KV_BYTES + k * 16 * 128, P * 128, 1024);
+              mma_bf16_ts(tmem + C::COL_O, tmem + col + k * 8, bd, ID_PV,
+                          (c > 0 || k > 0) ? 1u : 0u);
+            }
+            mma_commit(b_vempty(vs));
+            mma_commit(b_pvdone(c % C::PD));
+            if (lastg) mma_commit(b_sfree(col >> 7));  // the group's S buffer goes back
+            ++c;
+            *pv_pos = c;  // queue entry c - 1 has been read
+            did = true;
+          }
+        }
+        if (g >= n_groups && pv_end >= 0 && c >= pv_end) break;
+        if (did) {
+          t_idle = globaltimer_ns();
+          spins = 0;
+          nap = 32;
+        } else {
+          if (*abort_flag) break;
+          if ((++spins & 15u) == 0 && timed_out(t_idle)) {
+            give_up();
+            break;
+          }
+          __nanosleep(nap);  // back off while idle: polling takes issue slots
+          nap = min(nap * 2, 256u);
+        }
       }
-      mma_commit(b_done_pv);
+      // every issued MMA completes before teardown frees TMEM
+      mma_commit(b_done);
       const uint64_t t0 = globaltimer_ns();
-      while (!mbar_try_wait(b_done_pv, 0) && globaltimer_ns() - t0 < tmo) {}
+      while (!mbar_try_wait(b_done, 0) && globaltimer_ns() - t0 < tmo) {}
     }
   } else {
-    // ================= softmax: two warpgroups, half a row each =================
-    const int hw = (warp - 4) >> 2;      // which half of the columns
+    // ================= softmax: two warpgroups taking the groups in turn ========
+    const int wg = (warp - 4) >> 2;      // groups g with g % 2 == wg
     const int q4 = warp & 3;             // TMEM lane quarter
     const int row = q4 * 32 + lane;
     const bool row_valid = row < prm.q_block;
     const int grow = row0 + row;
-    const int c0 = hw * HP;              // first S column of this thread
     const uint32_t t_row = tmem + ((uint32_t)(q4 * 32) << 16);
-    const bool leader = (tid == 128);
+    const bool lead_warp = (q4 == 0);
+    const bool leader = lead_warp && lane == 0;
     const float sl2 = prm.scale_log2, le = prm.log2_eps;
-    float m_run = -INFINITY, m_ref = -INFINITY, l = 0.f;
-    int ci = 0;
-    bool ok = true;     // collective: every softmax warp leaves the loop at the same page
+    float m_run = -INFINITY, m_ref = -INFINITY, l = 0.f;  // l: this warpgroup's share, base m_ref
+    bool ok = true;     // OSK: collective within the warpgroup
     bool fail = false;  // this warp missed a wait after the vote; reported at the next vote
-    int pid_l = 0;
-    // page id of list entry j (warp-uniform); call once per j, in order
-    auto page_of = [&](int j) -> int {
-      if ((j & 31) == 0) pid_l = (j + lane < n_list) ? page_at(j + lane) : 0;
+    int fb = -1, pid_l = 0, cz_l = 0;
+    // page id (and, in the leading warp, TMA coordinate) of list entry j; j only grows
+    auto fetch = [&](int j, int& cz) -> int {
+      const int base = j & ~31;
+      if (base != fb) {
+        fb = base;
+        const int jl = base + lane;
+        pid_l = jl < n_list ? page_at(jl) : 0;
+        if (!DENSE && lead_warp) cz_l = jl < n_list ? coord_of(pid_l) : 0;
+      }
+      cz = __shfl_sync(0xffffffffu, cz_l, j & 31);
       return __shfl_sync(0xffffffffu, pid_l, j & 31);
     };
-    // half-row max of raw logits, causal mask on the diagonal page
-    auto half_max = [&](const uint32_t* src, int key0) -> float {
-      float v[HP];
-      if (key0 + P - 1 > row0) {  // diagonal page (warp-uniform): causal mask
-#pragma unroll
-        for (int e = 0; e < HP; ++e)
-          v[e] = key0 + c0 + e > grow ? -INFINITY : __uint_as_float(src[e]);
-      } else {
-#pragma unroll
-        for (int e = 0; e < HP; ++e) v[e] = __uint_as_float(src[e]);
-      }
-#pragma unroll
-      for (int w = HP / 2; w > 0; w >>= 1)
-#pragma unroll
-        for (int e = 0; e < w; ++e) v[e] = fmaxf(v[e], v[e + w]);
-      return v[0];
-    };
-    // publish the decision on page j for the V producer and the PV issuer, once
-    // both are past page j - DS
-    auto publish = [&](int j, bool keep) {
-      if (j >= C::DS) {
-        const uint64_t t0 = globaltimer_ns();
-        while (min(*pv_pos, *v_pos) <= j - C::DS) {
-          if (*abort_flag || globaltimer_ns() - t0 > tmo) { give_up(); break; }
-          __nanosleep(32);
-        }
-      }
-      dec_word[j % C::DS] = ((uint32_t)j << 1) | (keep ? 1u : 0u);
-    };
-    // kept page: online softmax with a lazily moved exponent base, then the P half
-    // row (bf16) into the swizzled K-major tile of ring slot ci % PS
-    auto kept_page = [&](const uint32_t* cur, float mloc, int key0) {
-      const float m_new = fmaxf(m_run, mloc);
-      m_run = m_new;
-      const bool resc = (m_ref != -INFINITY) && (m_new > m_ref + kRescaleLog2);
-      if (__any_sync(0xffffffffu, resc)) {
-        // O holds earlier pages: wait for the last issued PV, rescale this half of the rows
-        fail = !__all_sync(0xffffffffu,
-                           wait(b_pempty((ci - 1) % C::PS), ((ci - 1) / C::PS) & 1));
-        if (fail) return;
-        tc_fence_after();
-        const float alpha = resc ? ex2_approx(m_ref - m_new) : 1.f;
+    // row max of raw logits over the page at TMEM column col (key key0), 64 columns
+    // at a time, causal mask on the diagonal page
+    auto row_max = [&](uint32_t col, int key0) -> float {
+      float mx = -INFINITY;
 #pragma unroll 1
-        for (int c = 0; c < HD / 16; ++c) {
+      for (int c = 0; c < P / 64; ++c) {
+        uint32_t v[64];
+        tmem_ld64(t_row + col + c * 64, v);
+        const int k0 = key0 + c * 64;
+        if (k0 + 63 > row0) {  // diagonal page (warp-uniform): causal mask
+#pragma unroll
+          for (int e = 0; e < 64; ++e)
+            if (k0 + e > grow) v[e] = __float_as_uint(-INFINITY);
+        }
+        float a[8];
+#pragma unroll
+        for (int e = 0; e < 64; ++e)
+          a[e & 7] = e < 8 ? __uint_as_float(v[e]) : fmaxf(a[e & 7], __uint_as_float(v[e]));
+#pragma unroll
+        for (int w = 4; w > 0; w >>= 1)
+#pragma unroll
+          for (int e = 0; e < w; ++e) a[e] = fmaxf(a[e], a[e + w]);
+        mx = fmaxf(mx, a[0]);
+      }
+      return mx;
+    };
+    // leader: publish kept page c to the queue: its TMA coordinate (for the V
+    // producer), then its P column and last-of-group flag (for the MMA issuer)
+    auto bounded_until = [&](volatile int* pos, int c) {
+      if (c < C::KQ) return;
+      const uint64_t t0 = globaltimer_ns();
+      while (*pos <= c - C::KQ) {  // the entry's previous use has been read
+        if (*abort_flag || timed_out(t0)) { give_up(); break; }
+        __nanosleep(32);
+      }
+    };
+    auto publish_v = [&](int c, int cz) {
+      bounded_until(v_pos, c);
+      kq[c % C::KQ].x = cz;
+      __threadfence_block();
+      *vq_count = c + 1;
+    };
+    auto publish_info = [&](int c, int info) {
+      bounded_until(pv_pos, c);
+      kq[c % C::KQ].y = info;
+      __threadfence_block();
+      *kq_count = c + 1;
+    };
+    uint8_t* slog = (!DENSE && prm.skip_log) ? prm.skip_log + (bh * prm.num_q_blocks + qb) * prm.k_cap
+                                             : nullptr;
+    // kept page c: P = exp2(s * scale - mb) (bf16 pairs) written over the page's first
+    // P / 2 S columns, after the O rescale by alpha when this page moved the base
+    auto kept_page = [&](uint32_t col, int key0, float mb, bool resc_any, float alpha,
+                         int c) -> bool {
+      if (resc_any) {
+        // O holds the pages before c: wait for their last PV, rescale this warp's rows
+        if (c > 0 && !wait_warp(b_pvdone((c - 1) % C::PD), ((c - 1) / C::PD) & 1)) return false;
+        tc_fence_after();
+#pragma unroll 1
+        for (int k = 0; k < D / 16; ++k) {
           uint32_t r[16];
-          tmem_ld16(t_row + C::COL_O + hw * HD + c * 16, r);
+          tmem_ld16(t_row + C::COL_O + k * 16, r);
 #pragma unroll
           for (int e = 0; e < 16; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
-          tmem_st16(t_row + C::COL_O + hw * HD + c * 16, r);
+          tmem_st16(t_row + C::COL_O + k * 16, r);
         }
         tmem_st_wait();
         l *= alpha;
       }
-      if (m_new != -INFINITY && (m_ref == -INFINITY || resc)) m_ref = m_new;
-      const int ps = ci % C::PS;
-      if (ci >= C::PS) {
-        fail = !__all_sync(0xffffffffu, wait(b_pempty(ps), ((ci / C::PS) - 1) & 1));
-        if (fail) return;
-      }
       const bool diag = key0 + P - 1 > row0;
-      const bool rlive = row_valid && m_ref != -INFINITY;
-      const float nb2 = rlive ? -m_ref : 0.f;
+      const bool rlive = row_valid && mb != -INFINITY;
+      const float nb2 = rlive ? -mb : 0.f;
       float rs[4] = {0.f, 0.f, 0.f, 0.f};
-      const uint32_t prow = sP + ps * C::P_BYTES + row * 128;
+#pragma unroll 1
+      for (int k = 0; k < P / 64; ++k) {
+        uint32_t cur[64];
+        tmem_ld64(t_row + col + k * 64, cur);
 #pragma unroll
-      for (int c8 = 0; c8 < HP / 8; ++c8) {
-        uint32_t w4[4];
+        for (int h2 = 0; h2 < 2; ++h2) {
+          uint32_t w[16];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int i0 = c8 * 8 + 2 * e;
-          float x0 = fmaf(__uint_as_float(cur[i0]), sl2, nb2);
-          float x1 = fmaf(__uint_as_float(cur[i0 + 1]), sl2, nb2);
-          if (!rlive || (diag && key0 + c0 + i0 > grow)) x0 = -INFINITY;
-          if (!rlive || (diag && key0 + c0 + i0 + 1 > grow)) x1 = -INFINITY;
-          const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
-          rs[e] += p0 + p1;
-          __nv_bfloat162 v2 = __floats2bfloat162_rn(p0, p1);
-          w4[e] = *reinterpret_cast<uint32_t*>(&v2);
+          for (int e = 0; e < 16; ++e) {
+            const int i0 = h2 * 32 + 2 * e, key = key0 + k * 64 + i0;
+            float x0 = fmaf(__uint_as_float(cur[i0]), sl2, nb2);
+            float x1 = fmaf(__uint_as_float(cur[i0 + 1]), sl2, nb2);
+            if (!rlive || (diag && key > grow)) x0 = -INFINITY;
+            if (!rlive || (diag && key + 1 > grow)) x1 = -INFINITY;
+            const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+            rs[e & 3] += p0 + p1;
+            __nv_bfloat162 v2 = __floats2bfloat162_rn(p0, p1);
+            w[e] = *reinterpret_cast<uint32_t*>(&v2);
+          }
+          // S columns [k * 64, k * 64 + 64) are read: P pairs go to [k * 32, k * 32 + 32)
+          tmem_st16(t_row + col + k * 32 + h2 * 16, w);
         }
-        const int cg = (c0 >> 3) + c8;  // 16-byte chunk index within the row
-        const int blk = cg >> 3, cc = cg & 7;
-        st_shared_v4(prow + blk * (C::QB * 128) + ((cc ^ (row & 7)) << 4), w4[0], w4[1], w4[2],
-                     w4[3]);
       }
       l += (rs[0] + rs[1]) + (rs[2] + rs[3]);
-      fence_proxy_async_smem();
+      tmem_st_wait();
+      tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(b_pfull(ps));
-      ++ci;
+      if (lane == 0) mbar_arrive(b_pfull(c % C::PF));
+      return true;
     };
-    // votes of all eight softmax warps for round r of iteration it
-    auto vote_round = [&](int r, int it, uint32_t bits) -> uint32_t {
-      int* vt = const_cast<int*>(votes) + (r * 2 + (it & 1)) * 8;
-      if (lane == 0) vt[warp - 4] = (int)bits;
-      named_bar_sync(1, 256);  // orders the shared-memory exchange around it
-      const int4 v0 = *reinterpret_cast<const int4*>(vt);
-      const int4 v1 = *reinterpret_cast<const int4*>(vt + 4);
-      return (uint32_t)(v0.x | v0.y | v0.z | v0.w | v1.x | v1.y | v1.z | v1.w);
+    // votes of this warpgroup's four warps for its iteration it
+    auto vote_round = [&](int it, uint32_t bits) -> uint32_t {
+      int* vt = const_cast<int*>(votes) + (wg * 2 + (it & 1)) * 4;
+      if (lane == 0) vt[q4] = (int)bits;
+      named_bar_sync(1 + wg, 128);  // orders the shared-memory exchange around it
+      const int4 v = *reinterpret_cast<const int4*>(vt);
+      return (uint32_t)(v.x | v.y | v.z | v.w);
     };
-    // pages per iteration: two when a half row is 32 columns (the registers allow it)
-    constexpr int BATCH = (HP == 32) ? 2 : 1;
-    for (int j = 0, it = 0; j < n_list; j += BATCH, ++it) {
-      const int nb = min(BATCH, n_list - j);
-      int key0[BATCH];
-      uint32_t sv[BATCH][HP];
-      float mlh[BATCH];
-      bool lv[BATCH];
-#pragma unroll
-      for (int t = 0; t < BATCH; ++t) key0[t] = t < nb ? page_of(j + t) * P : 0;
-      // ---- S half rows of the batch: TMEM -> registers (one round trip), buffers back
-      bool okw = !fail;
-#pragma unroll
-      for (int t = 0; t < BATCH; ++t)
-        if (t < nb) okw = okw && wait(b_sfull((j + t) % C::SB), ((j + t) / C::SB) & 1);
-      okw = __all_sync(0xffffffffu, okw);
-      if (okw) {
-        tc_fence_after();
-#pragma unroll
-        for (int t = 0; t < BATCH; ++t)
-          if (t < nb)
-#pragma unroll
-            for (int c = 0; c < HP / 32; ++c)
-              tmem_ld32_async(t_row + ((j + t) % C::SB) * P + c0 + c * 32, sv[t] + c * 32);
-#pragma unroll
-        for (int t = 0; t < BATCH; ++t)
-#pragma unroll
-          for (int c = 0; c < HP / 32; ++c) {
-            if (t == 0 && c == 0) tmem_ld_wait32(sv[0]);
-            else reg_tie32(sv[t] + c * 32);
+    // wait (lane 0 of each warp) until every warp of the other warpgroup has settled
+    // group g (all groups before the next one of this warpgroup are then settled)
+    auto wait_settled = [&](int g) -> bool {
+      int okl = 1;
+      if (lane == 0) {
+        volatile int* o = settled + (wg ^ 1) * 4;
+        auto done = [&]() { return min(min(o[0], o[1]), min(o[2], o[3])) >= g; };
+        if (!done()) {
+          const uint64_t t0 = globaltimer_ns();
+          uint32_t spins = 0, nap = 32;
+          while (!done()) {
+            if (*abort_flag) { okl = 0; break; }
+            if ((++spins & 15u) == 0 && timed_out(t0)) { give_up(); okl = 0; break; }
+            __nanosleep(nap);
+            nap = min(nap * 2, 256u);
           }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0)
-#pragma unroll
-          for (int t = 0; t < BATCH; ++t)
-            if (t < nb) mbar_arrive(b_sfree((j + t) % C::SB));
+        }
       }
-      // ---- half-row maxima -> round 1 exchange
-      float* hm = const_cast<float*>(hmax) + (it & 1) * 512;
+      return __shfl_sync(0xffffffffu, okl, 0) != 0;
+    };
+    // this warp has settled group g (its state rows and queue entries are written)
+    auto mark_settled = [&](int g) {
+      __threadfence_block();
+      __syncwarp();
+      if (lane == 0) settled[wg * 4 + q4] = g;
+    };
+    // the first listed page is always kept: its V can go out before any vote
+    if (!DENSE && wg == 0 && n_list > 0) {
+      int cz0;
+      fetch(0, cz0);
+      if (leader) publish_v(0, cz0);
+    }
+    int rnd = 0;  // vote rounds of this warpgroup
+    for (int g = wg; g < n_groups; g += 2) {
+      const int j = g * GP;
+      const int nb = min(GP, n_list - j);
+      const int sb = g % C::SBG;
+      int key0[GP], czp[GP];
 #pragma unroll
-      for (int t = 0; t < BATCH; ++t) {
-        const float mh = (okw && t < nb) ? half_max(sv[t], key0[t]) : -INFINITY;
-        lv[t] = row_valid && mh != -INFINITY;
-        mlh[t] = lv[t] ? mh * sl2 : -INFINITY;
-        hm[(t * 2 + hw) * 128 + row] = mlh[t];
+      for (int t = 0; t < GP; ++t) {
+        czp[t] = 0;
+        key0[t] = t < nb ? fetch(j + t, czp[t]) * P : 0;
       }
-      const uint32_t all1 = vote_round(0, it, okw ? 0u : 1u);
-      if (all1 & 1u) { ok = false; break; }
-      float mloc[BATCH];
-#pragma unroll
-      for (int t = 0; t < BATCH; ++t) {
-        mloc[t] = fmaxf(mlh[t], hm[(t * 2 + (hw ^ 1)) * 128 + row]);
-        lv[t] = mloc[t] != -INFINITY;
+      // ---- row maxima of the group's pages, read from TMEM
+      const bool okw = !fail && wait_warp(b_sfull(sb), (g / C::SBG) & 1);
+      if (okw) tc_fence_after();
+      // (one copy of the per-page code: the loop is not unrolled)
+      float ml0 = -INFINITY, ml1 = -INFINITY;
+#pragma unroll 1
+      for (int t = 0; t < (okw ? nb : 0); ++t) {
+        const float mr = row_max(sb * 128 + t * P, t == 0 ? key0[0] : key0[GP - 1]);
+        if (t == 0) ml0 = mr;
+        else ml1 = mr;
       }
-      // ---- round 2: votes on full row maxima.  Page j + 1 is voted for both
-      // outcomes of page j, so the decisions stay exactly sequential.
-      bool keep[BATCH];
-      if (DENSE) {
+      float mloc[GP];
+      bool lv[GP];
 #pragma unroll
-        for (int t = 0; t < BATCH; ++t) keep[t] = true;
-      } else {
-        const bool n0 = lv[0] && (m_run == -INFINITY || mloc[0] - m_run >= le);
+      for (int t = 0; t < GP; ++t) {
+        const float mr = row_valid ? (t == 0 ? ml0 : ml1) : -INFINITY;
+        lv[t] = mr != -INFINITY;
+        mloc[t] = lv[t] ? mr * sl2 : -INFINITY;
+      }
+      tc_fence_before();
+      // votes of this group's pages against running max m: page 1 (2), page 2 after
+      // page 1 kept (4), page 2 after page 1 skipped (8)
+      auto vote_bits = [&](float m) -> uint32_t {
+        const bool n0 = lv[0] && (m == -INFINITY || mloc[0] - m >= le);
         uint32_t bits = __any_sync(0xffffffffu, n0) ? 2u : 0u;
-        if (BATCH == 2 && nb == 2) {
-          const float mk = fmaxf(m_run, mloc[0]);
-          const bool nk = lv[BATCH - 1] && (mk == -INFINITY || mloc[BATCH - 1] - mk >= le);
-          const bool ns = lv[BATCH - 1] && (m_run == -INFINITY || mloc[BATCH - 1] - m_run >= le);
+        if (GP == 2 && nb == 2) {
+          const float mk = fmaxf(m, mloc[0]);
+          const bool nk = lv[GP - 1] && (mk == -INFINITY || mloc[GP - 1] - mk >= le);
+          const bool ns = lv[GP - 1] && (m == -INFINITY || mloc[GP - 1] - m >= le);
           bits |= __any_sync(0xffffffffu, nk) ? 4u : 0u;
           bits |= __any_sync(0xffffffffu, ns) ? 8u : 0u;
         }
-        const uint32_t all2 = vote_round(1, it, bits);
-        keep[0] = (j == 0) || (all2 & 2u);
-        if (BATCH == 2) keep[BATCH - 1] = keep[0] ? (all2 & 4u) != 0 : (all2 & 8u) != 0;
-        if (leader)
-#pragma unroll
-          for (int t = 0; t < BATCH; ++t)
-            if (t < nb) publish(j + t, keep[t]);
+        return bits;
+      };
+      bool exact = DENSE || j == 0;
+      if (!DENSE) {
+        // ---- first vote, against the running max this warpgroup last saw (a lower
+        // bound of the current one: what it skips stays skipped)
+        m_run = fmaxf(m_run, st_rows[row].x);
+        uint32_t bits = okw ? 0u : 1u;
+        if (okw && !exact) bits |= vote_bits(m_run);
+        const uint32_t all = vote_round(rnd++, bits);
+        if (all & 1u) { ok = false; break; }
+        if (!exact && (all & 10u) == 0) {
+          // every page of the group is skipped: settled without the other warpgroup
+          if (leader) {
+            if (slog)
+              for (int t = 0; t < nb; ++t) slog[j + t] = 1;
+            mbar_arrive(b_sfree(sb));
+          }
+          mark_settled(g);
+          continue;
+        }
+        exact = true;
       }
+      // ---- exact path: the groups before this one are settled; take their state
+      bool oks = okw && (g == 0 || wait_settled(g - 1));
+      if (oks) {
+        __threadfence_block();
+        const float sr = st_rows[row].x, sf = st_rows[row].y;
+        if (sf != m_ref) {  // the base only moves up: bring this warpgroup's l along
+          if (m_ref != -INFINITY) l *= ex2_approx(m_ref - sf);
+          m_ref = sf;
+        }
+        m_run = sr;
+      }
+      // kept pages before this group: every earlier queue entry is published, and
+      // the count is read before the vote barrier, ahead of this group's publishing
+      const int c0 = DENSE ? j : *kq_count;
+      bool keep[GP];
+      if (DENSE) {
+        if (!oks) { ok = false; break; }
 #pragma unroll
-      for (int t = 0; t < BATCH; ++t)
-        if (t < nb && keep[t] && !fail) kept_page(sv[t], mloc[t], key0[t]);
+        for (int t = 0; t < GP; ++t) keep[t] = t < nb;
+      } else {
+        uint32_t bits = oks ? vote_bits(m_run) : 1u;
+        const uint32_t all = vote_round(rnd++, bits);
+        if (all & 1u) { ok = false; break; }
+        keep[0] = (j == 0) || (all & 2u);
+        if (GP == 2) keep[GP - 1] = nb == 2 && (keep[0] ? (all & 4u) != 0 : (all & 8u) != 0);
+      }
+      // ---- state after this group's decisions: running max, and the exponent base
+      // (with the O rescale factor) of each kept page
+      float mb[GP], alpha[GP];
+      bool rany[GP];
+      int nk = 0, lastk = -1;
+#pragma unroll
+      for (int t = 0; t < GP; ++t) {
+        mb[t] = m_ref;
+        alpha[t] = 1.f;
+        rany[t] = false;
+        if (t < nb && keep[t]) {
+          const float m_new = fmaxf(m_run, mloc[t]);
+          m_run = m_new;
+          const bool resc = (m_ref != -INFINITY) && (m_new > m_ref + kRescaleLog2);
+          alpha[t] = resc ? ex2_approx(m_ref - m_new) : 1.f;
+          rany[t] = __any_sync(0xffffffffu, resc);
+          if (m_new != -INFINITY && (m_ref == -INFINITY || resc)) m_ref = m_new;
+          mb[t] = m_ref;
+          ++nk;
+          lastk = t;
+        }
+      }
+      if (nk > 0) {
+        st_rows[row].x = m_run;
+        st_rows[row].y = m_ref;
+      }
+      if (!DENSE && leader) {
+        int c = c0;
+#pragma unroll
+        for (int t = 0; t < GP; ++t)
+          if (t < nb) {
+            if (slog) slog[j + t] = keep[t] ? 0 : 1;
+            if (keep[t]) {
+              if (j + t > 0) publish_v(c, czp[t]);
+              publish_info(c, (sb * 128 + t * P) | ((t == lastk ? 1 : 0) << 15));
+              ++c;
+            }
+          }
+        if (nk == 0) mbar_arrive(b_sfree(sb));  // nothing kept: the S buffer goes back now
+      }
+      mark_settled(g);
+      // ---- P of the kept pages; their PV follows in list order
+      int c = c0;
+#pragma unroll 1
+      for (int t = 0; t < nb; ++t) {
+        const bool k1 = t > 0;  // (scalar selects keep one copy of the page code)
+        if (!(k1 ? keep[GP - 1] : keep[0])) continue;
+        if (!fail && !kept_page(sb * 128 + t * P, k1 ? key0[GP - 1] : key0[0],
+                                k1 ? mb[GP - 1] : mb[0], k1 ? rany[GP - 1] : rany[0],
+                                k1 ? alpha[GP - 1] : alpha[0], c))
+          fail = true;
+        ++c;
+      }
+      if (DENSE && fail) { ok = false; break; }
     }
-    // ---- epilogue: O / l -> bf16 (each warpgroup its half of the columns), LSE
-    if (ok && !fail && ci > 0)
-      fail = !__all_sync(0xffffffffu, wait(b_pempty((ci - 1) % C::PS), ((ci - 1) / C::PS) & 1));
-    if (ok) {  // all softmax warps are here together: exchange the half-row sums
-      hsum[hw * 128 + row] = l;
-      named_bar_sync(1, 256);
-      l += hsum[(hw ^ 1) * 128 + row];
+    if (leader) {  // the second warpgroup to finish closes the queue
+      __threadfence_block();
+      if (atomicAdd(wg_done, 1) == 1 && !DENSE) *kq_final = *kq_count;
     }
+    // ---- epilogue: both warpgroups' row sums to one base, O / l -> bf16, LSE
+    fin_rows[wg * 128 + row].x = l;
+    fin_rows[wg * 128 + row].y = m_ref;
+    __threadfence_block();
+    named_bar_sync(3, 256);
+    const float ol = fin_rows[(wg ^ 1) * 128 + row].x, om = fin_rows[(wg ^ 1) * 128 + row].y;
+    const float M = fmaxf(m_ref, om);
+    float lt = 0.f;
+    if (m_ref != -INFINITY) lt += l * ex2_approx(m_ref - M);
+    if (om != -INFINITY) lt += ol * ex2_approx(om - M);
+    const int cfin = DENSE ? n_list : *kq_count;
+    int hv = 0;
+    if (lane == 0) hv = (*abort_flag == 0 && cfin > 0) ? 1 : 0;
+    bool have = __shfl_sync(0xffffffffu, hv, 0) != 0;
+    if (have) have = wait_warp(b_pvdone((cfin - 1) % C::PD), ((cfin - 1) / C::PD) & 1);
     tc_fence_after();
-    const float inv = l > 0.f ? 1.f / l : 0.f;
-    __nv_bfloat16* orow = prm.out + (bh * prm.seq_len + grow) * D + hw * HD;
+    const float inv = (have && lt > 0.f) ? 1.f / lt : 0.f;
+    constexpr int HD = D / 2;  // each warpgroup writes half of the columns
+    __nv_bfloat16* orow = prm.out + (bh * prm.seq_len + grow) * D + wg * HD;
 #pragma unroll
-    for (int c = 0; c < HD / 32; ++c) {
+    for (int k = 0; k < HD / 32; ++k) {
       uint32_t r[32];
-      if (ok && !fail && ci > 0) {
-        tmem_ld32(t_row + C::COL_O + hw * HD + c * 32, r);
+      if (have) {
+        tmem_ld32(t_row + C::COL_O + wg * HD + k * 32, r);
       } else {
 #pragma unroll
         for (int e = 0; e < 32; ++e) r[e] = 0u;
@@ -609,23 +825,23 @@ __global__ void __launch_bounds__(384, 1)
                                                     __uint_as_float(r[2 * e + 1]) * inv);
           w[e] = *reinterpret_cast<uint32_t*>(&v2);
         }
-        uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+        uint4* dst = reinterpret_cast<uint4*>(orow + k * 32);
         dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
         dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
         dst[2] = make_uint4(w[8], w[9], w[10], w[11]);
         dst[3] = make_uint4(w[12], w[13], w[14], w[15]);
       }
     }
-    if (hw == 0 && row_valid && prm.lse)
+    if (wg == 0 && row_valid && prm.lse)
       prm.lse[bh * prm.seq_len + grow] =
-          l > 0.f ? (m_ref + log2f(l)) * 0.69314718055994531f : -INFINITY;
-    if (!DENSE && leader && prm.computed) prm.computed[bh * prm.num_q_blocks + qb] = ci;
+          (have && lt > 0.f) ? (M + log2f(lt)) * 0.69314718055994531f : -INFINITY;
+    if (!DENSE && wg == 0 && leader && prm.computed) prm.computed[bh * prm.num_q_blocks + qb] = cfin;
   }
 
   // ---- teardown
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) {
+  if (warp == 3) {
     __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);
