@@ -379,87 +379,88 @@ __global__ void __launch_bounds__(384, 1)
   } else if (warp == 3) {
     if (lane == 0) {
       // ================= MMA issuer: QK^T per group, PV per kept page =============
+      // (a lean loop: it shares its scheduler with two softmax warps)
       constexpr uint32_t ID_FULL = idesc_bf16_f32(128, 128, 0);
       constexpr uint32_t ID_PAGE = idesc_bf16_f32(128, P, 0);  // a lone last page
       constexpr uint32_t ID_PV = idesc_bf16_f32(128, D, 1);
+      // descriptors of the tile bases; a 16-byte aligned offset below 256 KB adds to
+      // the start-address field directly
+      const uint64_t dq = smem_desc_sw128(sQ, 16, 1024);
+      const uint64_t dk = smem_desc_sw128(sK, 16, 1024);
+      const uint64_t dv = smem_desc_sw128(sV, P * 128, 1024);
       bool ok = wait(b_q, 0);
-      int g = 0, c = 0, pv_end = DENSE ? n_list : -1;
-      uint64_t t_idle = globaltimer_ns();
-      uint32_t spins = 0, nap = 32;
+      int g = 0, c = 0, pv_end = DENSE ? n_list : -1, seen = 0;
+      int ks = 0, sbuf = 0;
+      uint32_t kpar = 0, spar = 0;  // phase parities of k_full[ks] and s_free[sbuf]
+      uint64_t t_idle = 0;
+      uint32_t idle = 0, nap = 32;
       while (ok) {
-        bool did = false;
-        if (g < n_groups) {
-          const int ks = g % C::KG, sbuf = g % C::SBG;
-          if (mbar_test_wait(b_kfull(ks), (g / C::KG) & 1) &&
-              (g < C::SBG || mbar_test_wait(b_sfree(sbuf), ((g / C::SBG) - 1) & 1))) {
-            tc_fence_after();
-            const uint32_t id = (g * GP + GP <= n_list) ? ID_FULL : ID_PAGE;
+        // QK^T first: an issue blocks this thread while the tensor core works
+        // through it, so the next group is tried straight away
+        if (g < n_groups && mbar_test_wait(b_kfull(ks), kpar) &&
+            (g < C::SBG || mbar_test_wait(b_sfree(sbuf), spar))) {
+          tc_fence_after();
+          const uint32_t id = (g * GP + GP <= n_list) ? ID_FULL : ID_PAGE;
+          const uint64_t dks = dk + ((uint32_t)ks * C::KG_BYTES >> 4);
 #pragma unroll
-            for (int k = 0; k < D / 16; ++k) {
-              const uint64_t a =
-                  smem_desc_sw128(sQ + (k >> 2) * (C::QB * 128) + (k & 3) * 32, 16, 1024);
-              const uint64_t bd = smem_desc_sw128(
-                  sK + ks * C::KG_BYTES + (k >> 2) * (GP * P * 128) + (k & 3) * 32, 16, 1024);
-              mma_bf16_ss(tmem + sbuf * 128, a, bd, id, k > 0 ? 1u : 0u);
-            }
-            mma_commit(b_kempty(ks));
-            mma_commit(b_sfull(sbuf));
-            ++g;
-            did = true;
-          }
+          for (int k = 0; k < D / 16; ++k)
+            mma_bf16_ss(tmem + sbuf * 128, dq + (((k >> 2) * (C::QB * 128) + (k & 3) * 32) >> 4),
+                        dks + (((k >> 2) * (GP * P * 128) + (k & 3) * 32) >> 4), id, k > 0 ? 1u : 0u);
+          mma_commit(b_kempty(ks));
+          mma_commit(b_sfull(sbuf));
+          ++g;
+          if (++ks == C::KG) { ks = 0; kpar ^= 1u; }
+          if (++sbuf == C::SBG) sbuf = 0;
+          if (g > C::SBG && sbuf == 0) spar ^= 1u;  // s_free waits start at group SBG, parity 0
+          idle = 0;
+          nap = 32;
+          continue;
         }
-        if (!DENSE && pv_end < 0) {
+        if (!DENSE && pv_end < 0 && c >= seen) {
           const int f = *kq_final;  // read before the count: the count is final once f >= 0
+          seen = *kq_count;
           if (f >= 0) pv_end = f;
         }
-        if (pv_end < 0 || c < pv_end) {
-          bool avail = true;
+        if ((DENSE || c < seen) && (pv_end < 0 || c < pv_end)) {
           int col, lastg;
           if (DENSE) {
             const int t = c % GP;
             col = ((c / GP) % C::SBG) * 128 + t * P;
             lastg = (t == GP - 1 || c == n_list - 1) ? 1 : 0;
           } else {
-            avail = *kq_count > c;
-            int info = 0;
-            if (avail) {
-              __threadfence_block();
-              info = kq[c % C::KQ].y;
-            }
+            __threadfence_block();
+            const int info = kq[c % C::KQ].y;
             col = info & 0x7fff;
             lastg = info >> 15;
           }
-          const int vs = c % C::VS, pf = c % C::PF;
-          if (avail && mbar_test_wait(b_vfull(vs), (c / C::VS) & 1) &&
-              mbar_test_wait(b_pfull(pf), (c / C::PF) & 1)) {
+          const int vs = c % C::VS;
+          if (mbar_test_wait(b_vfull(vs), (c / C::VS) & 1) &&
+              mbar_test_wait(b_pfull(c % C::PF), (c / C::PF) & 1)) {
             tc_fence_after();
+            const uint64_t dvs = dv + ((uint32_t)vs * C::KV_BYTES >> 4);
 #pragma unroll
-            for (int k = 0; k < P / 16; ++k) {
-              const uint64_t bd =
-                  smem_desc_sw128(sV + vs * C::KV_BYTES + k * 16 * 128, P * 128, 1024);
-              mma_bf16_ts(tmem + C::COL_O, tmem + col + k * 8, bd, ID_PV,
+            for (int k = 0; k < P / 16; ++k)
+              mma_bf16_ts(tmem + C::COL_O, tmem + col + k * 8, dvs + ((k * 16 * 128) >> 4), ID_PV,
                           (c > 0 || k > 0) ? 1u : 0u);
-            }
             mma_commit(b_vempty(vs));
             mma_commit(b_pvdone(c % C::PD));
             if (lastg) mma_commit(b_sfree(col >> 7));  // the group's S buffer goes back
             ++c;
             *pv_pos = c;  // queue entry c - 1 has been read
-            did = true;
+            idle = 0;
+            nap = 32;
+            continue;
           }
         }
         if (g >= n_groups && pv_end >= 0 && c >= pv_end) break;
-        if (did) {
-          t_idle = globaltimer_ns();
-          spins = 0;
-          nap = 32;
-        } else {
-          if (*abort_flag) break;
-          if ((++spins & 15u) == 0 && timed_out(t_idle)) {
-            give_up();
-            break;
-          }
-          __nanosleep(nap);  // back off while idle: polling takes issue slots
+        if (idle++ == 0) t_idle = globaltimer_ns();
+        if (*abort_flag) break;
+        if ((idle & 15u) == 0 && timed_out(t_idle)) {
+          give_up();
+          break;
+        }
+        if (idle > 2) {  // back off while idle: polling takes issue slots
+          __nanosleep(nap);
           nap = min(nap * 2, 256u);
         }
       }
