@@ -12,12 +12,13 @@
 //   warps 0, 1  K producers: group g is loaded by warp g % 2 into ring slot
 //               g % KG, so two TMA streams run side by side (warp 0 also loads
 //               Q).  The physical page comes from the page table; no multicast.
-//   warp 2      V producer: loads V of the kept pages only, once the vote has
-//               kept them, so a skipped page costs its K tile and its share of
-//               one QK^T, nothing more.
-//   warp 3      MMA issuer (one thread, polling): QK^T of the next group when
-//               its K tile and an S buffer are ready, PV of the next kept page
-//               when its P and V are ready.
+//   warp 2      V loads and PV (one thread): loads V of the kept pages only,
+//               once the vote has kept them (up to VS pages ahead), so a skipped
+//               page costs its K tile and its share of one QK^T, nothing more;
+//               then O += P_c V_c with P read from TMEM.
+//   warp 3      QK^T issuer (one thread); allocates TMEM.  An MMA issue blocks its
+//               thread while the tensor core works, so QK^T and PV have a thread
+//               each.
 //   warps 4-7,  softmax, two warpgroups taking the groups in turn (even groups
 //   8-11        warpgroup 0, odd groups warpgroup 1).  Thread (warp % 4, lane)
 //               owns query row 32 (warp % 4) + lane, which is its TMEM lane,
@@ -37,9 +38,10 @@
 //               always kept.  For kept pages each thread writes
 //               P = exp2(s - m_ref) (bf16) for its row over the page's S
 //               columns; m_ref, the exponent base, moves only when the running
-//               max passes it by more than 2^8 (O and l are then rescaled),
-//               which keeps the result exact.
-// Kept pages reach the V producer and the MMA issuer through a shared-memory
+//               max passes it by more than 2^32 (O and l are then rescaled),
+//               which keeps the result exact: P <= 2^32 stays well inside the
+//               range of bf16, and l and O inside fp32.
+// Kept pages reach the V/PV thread through a shared-memory
 // queue that carries each page's TMA coordinate and P location; the
 // consumers' progress counters give it back-pressure.  Every wait is bounded: on
 // timeout the CTA records COSA_ERR_TIMEOUT in the status word, drains what it
@@ -86,8 +88,8 @@ struct TcCfg {
   static constexpr uint32_t OFF_K = OFF_Q + Q_BYTES;
   static constexpr uint32_t OFF_V = OFF_K + KG * KG_BYTES;
   static constexpr uint32_t OFF_BAR = OFF_V + VS * KV_BYTES;
-  // q, k_full/empty, v_full/empty, s_full/free, p_full, pv_done, done
-  static constexpr int NBAR = 1 + 2 * KG + 2 * VS + 2 * SBG + PF + PD + 1;
+  // q, k_full/empty, v_full/empty, s_full/free, p_full, pv_done, done (QK), done (PV)
+  static constexpr int NBAR = 1 + 2 * KG + 2 * VS + 2 * SBG + PF + PD + 2;
   static constexpr uint32_t OFF_MISC = (OFF_BAR + NBAR * 8 + 127) & ~127u;  // vector-aligned
   // misc: +0 TMEM address, +4 abort flag, +8 kept count (P location published),
   //       +12 final kept count (-1 while the votes run), +16 V progress,
@@ -109,7 +111,9 @@ struct TcCfg {
   static_assert(M_STATE + 128 * 8 <= M_SETTLED && M_SETTLED + 8 * 4 <= M_FIN, "state rows and flags fit");
 };
 
-constexpr float kRescaleLog2 = 8.0f;  // m_ref trails the running max by < 2^8
+// m_ref trails the running max by < 2^32: a rescale waits for the PV before it,
+// so it is kept rare; P = exp2(s - m_ref) <= 2^32, l <= 2^32 * keys, all in range
+constexpr float kRescaleLog2 = 32.0f;
 
 template <int D, int P, bool DENSE>
 __global__ void __launch_bounds__(384, 1)
@@ -135,7 +139,8 @@ __global__ void __launch_bounds__(384, 1)
   auto b_pvdone = [&](int s) {
     return bar + 8u * (1 + 2 * C::KG + 2 * C::VS + 2 * C::SBG + C::PF + s);
   };
-  const uint32_t b_done = bar + 8u * (C::NBAR - 1);
+  const uint32_t b_done = bar + 8u * (C::NBAR - 2);
+  const uint32_t b_done_pv = bar + 8u * (C::NBAR - 1);
   uint8_t* misc = sg + C::OFF_MISC;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(misc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 4);
@@ -194,6 +199,7 @@ __global__ void __launch_bounds__(384, 1)
     for (int s = 0; s < C::PF; ++s) mbar_init(b_pfull(s), 4);
     for (int s = 0; s < C::PD; ++s) mbar_init(b_pvdone(s), 1);
     mbar_init(b_done, 1);
+    mbar_init(b_done_pv, 1);
     *abort_flag = 0;
     *kq_count = 0;
     *kq_final = -1;
@@ -233,12 +239,11 @@ __global__ void __launch_bounds__(384, 1)
   auto timed_out = [&](uint64_t t0) {
     return *(volatile int*)&g_status == COSA_ERR_TIMEOUT || globaltimer_ns() - t0 > tmo;
   };
-  // bounded blocking wait on an mbarrier phase; false on timeout or abort.  The
-  // suspend hint lets a waiting warp sleep instead of taking issue slots.
+  // bounded blocking wait on an mbarrier phase; false on timeout or abort
   auto wait = [&](uint32_t bar_addr, uint32_t parity) -> bool {
     if (mbar_try_wait(bar_addr, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
-    while (!mbar_try_wait_sleep(bar_addr, parity, 20000u)) {
+    while (!mbar_try_wait(bar_addr, parity)) {
       if (*abort_flag) return false;
       if (timed_out(t0)) {
         give_up();
@@ -330,139 +335,113 @@ __global__ void __launch_bounds__(384, 1)
                globaltimer_ns() - t0 < tmo) {}
     }
   } else if (warp == 2) {
-    // ================= V producer: kept pages in list order ======================
-    if (lane == 0) prefetch_tmap(&tm_v);
-    int last = -1;
-    bool ok = true;
-    int cz_l = 0;
-    for (int c = 0; ok; ++c) {
-      int cz;
-      if (DENSE) {
-        if (c >= n_list) break;
-        if ((c & 31) == 0) cz_l = c + lane < n_list ? coord_of(c + lane) : 0;
-        cz = __shfl_sync(0xffffffffu, cz_l, c & 31);
-      } else {
-        int r = 0, e = 0;
-        if (lane == 0) {
-          r = kept_ready(vq_count, c);
-          if (r > 0) {
-            __threadfence_block();
-            e = kq[c % C::KQ].x;
-            *v_pos = c + 1;  // queue entry c has been read
-          }
+    if (lane == 0) {
+      // ================= V loads and PV, kept pages in list order =================
+      // V tiles are loaded ahead (up to VS pages) as the kept pages become known;
+      // PV of page c follows once its P and V are in place.
+      prefetch_tmap(&tm_v);
+      constexpr uint32_t ID_PV = idesc_bf16_f32(128, D, 1);
+      const uint64_t dv = smem_desc_sw128(sV, P * 128, 1024);
+      int nv = 0;                          // V loads issued
+      int c = 0;                           // PV issued
+      int pv_end = DENSE ? n_list : -1;    // kept pages in all (once known)
+      bool ok = true;
+      // issue the V load of kept page nv (its slot is free)
+      auto load_v = [&]() {
+        int cz;
+        if (DENSE) {
+          cz = coord_of(nv);
+        } else {
+          __threadfence_block();
+          cz = kq[nv % C::KQ].x;
+          *v_pos = nv + 1;  // queue entry nv has been read
         }
-        r = __shfl_sync(0xffffffffu, r, 0);
-        if (r < 0) ok = false;
-        if (r <= 0) break;
-        cz = __shfl_sync(0xffffffffu, e, 0);
-      }
-      const int s = c % C::VS;
-      if (c >= C::VS) {
-        ok = wait_warp(b_vempty(s), ((c / C::VS) - 1) & 1);
-        if (!ok) break;
-      }
-      if (lane == 0) {
+        const int s = nv % C::VS;
         mbar_arrive_expect_tx(b_vfull(s), C::KV_BYTES);
 #pragma unroll
         for (int kb = 0; kb < D / 64; ++kb)
           tma_load_3d(sV + s * C::KV_BYTES + kb * (P * 128), &tm_v, b_vfull(s), kb * 64, 0, cz);
+        ++nv;
+      };
+      auto v_known = [&](int x) { return DENSE ? x < n_list : *vq_count > x; };
+      while (ok) {
+        // ---- kept page c known (or the list ended)?
+        if (!DENSE && pv_end < 0) {
+          const int r = kept_ready(kq_count, c);
+          if (r < 0) break;
+          if (r == 0) pv_end = *kq_final;
+        }
+        if (pv_end >= 0 && c >= pv_end) break;
+        // ---- its V, and the following ones while slots are free (no waiting)
+        if (nv == c) {
+          if (c >= C::VS && !wait(b_vempty(c % C::VS), ((c / C::VS) - 1) & 1)) break;
+          load_v();
+        }
+        while (nv < c + C::VS && v_known(nv) &&
+               (nv < C::VS || mbar_test_wait(b_vempty(nv % C::VS), ((nv / C::VS) - 1) & 1)))
+          load_v();
+        // ---- PV of page c
+        int col, lastg;
+        if (DENSE) {
+          const int t = c % GP;
+          col = ((c / GP) % C::SBG) * 128 + t * P;
+          lastg = (t == GP - 1 || c == n_list - 1) ? 1 : 0;
+        } else {
+          __threadfence_block();
+          const int info = kq[c % C::KQ].y;
+          col = info & 0x7fff;
+          lastg = info >> 15;
+        }
+        const int vs = c % C::VS;
+        if (!wait(b_vfull(vs), (c / C::VS) & 1)) break;
+        if (!wait(b_pfull(c % C::PF), (c / C::PF) & 1)) break;
+        tc_fence_after();
+        const uint64_t dvs = dv + ((uint32_t)vs * C::KV_BYTES >> 4);
+#pragma unroll
+        for (int k = 0; k < P / 16; ++k)
+          mma_bf16_ts(tmem + C::COL_O, tmem + col + k * 8, dvs + ((k * 16 * 128) >> 4), ID_PV,
+                      (c > 0 || k > 0) ? 1u : 0u);
+        mma_commit(b_vempty(vs));
+        mma_commit(b_pvdone(c % C::PD));
+        if (lastg) mma_commit(b_sfree(col >> 7));  // the group's S buffer goes back
+        ++c;
+        *pv_pos = c;  // queue entry c - 1 has been read
       }
-      last = c;
-      __syncwarp();
-    }
-    if (lane == 0 && *abort_flag) {
+      // every issued PV completes before teardown frees TMEM; V loads never consumed
+      // (abort only) land before the CTA leaves
+      mma_commit(b_done_pv);
       const uint64_t t0 = globaltimer_ns();
-      for (int c = last; c >= 0 && c > last - C::VS; --c)
-        while (!mbar_try_wait(b_vfull(c % C::VS), (c / C::VS) & 1) &&
-               globaltimer_ns() - t0 < tmo) {}
+      while (!mbar_try_wait(b_done_pv, 0) && globaltimer_ns() - t0 < tmo) {}
+      for (int x = c; x < nv; ++x)
+        while (!mbar_try_wait(b_vfull(x % C::VS), (x / C::VS) & 1) && globaltimer_ns() - t0 < tmo) {}
     }
   } else if (warp == 3) {
     if (lane == 0) {
-      // ================= MMA issuer: QK^T per group, PV per kept page =============
-      // (a lean loop: it shares its scheduler with two softmax warps)
+      // ================= QK^T issuer, one group of 128 keys at a time =============
       constexpr uint32_t ID_FULL = idesc_bf16_f32(128, 128, 0);
       constexpr uint32_t ID_PAGE = idesc_bf16_f32(128, P, 0);  // a lone last page
-      constexpr uint32_t ID_PV = idesc_bf16_f32(128, D, 1);
       // descriptors of the tile bases; a 16-byte aligned offset below 256 KB adds to
       // the start-address field directly
       const uint64_t dq = smem_desc_sw128(sQ, 16, 1024);
       const uint64_t dk = smem_desc_sw128(sK, 16, 1024);
-      const uint64_t dv = smem_desc_sw128(sV, P * 128, 1024);
       bool ok = wait(b_q, 0);
-      int g = 0, c = 0, pv_end = DENSE ? n_list : -1, seen = 0;
       int ks = 0, sbuf = 0;
       uint32_t kpar = 0, spar = 0;  // phase parities of k_full[ks] and s_free[sbuf]
-      uint64_t t_idle = 0;
-      uint32_t idle = 0, nap = 32;
-      while (ok) {
-        // QK^T first: an issue blocks this thread while the tensor core works
-        // through it, so the next group is tried straight away
-        if (g < n_groups && mbar_test_wait(b_kfull(ks), kpar) &&
-            (g < C::SBG || mbar_test_wait(b_sfree(sbuf), spar))) {
-          tc_fence_after();
-          const uint32_t id = (g * GP + GP <= n_list) ? ID_FULL : ID_PAGE;
-          const uint64_t dks = dk + ((uint32_t)ks * C::KG_BYTES >> 4);
+      for (int g = 0; ok && g < n_groups; ++g) {
+        if (!wait(b_kfull(ks), kpar)) break;
+        if (g >= C::SBG && !wait(b_sfree(sbuf), spar)) break;
+        tc_fence_after();
+        const uint32_t id = (g * GP + GP <= n_list) ? ID_FULL : ID_PAGE;
+        const uint64_t dks = dk + ((uint32_t)ks * C::KG_BYTES >> 4);
 #pragma unroll
-          for (int k = 0; k < D / 16; ++k)
-            mma_bf16_ss(tmem + sbuf * 128, dq + (((k >> 2) * (C::QB * 128) + (k & 3) * 32) >> 4),
-                        dks + (((k >> 2) * (GP * P * 128) + (k & 3) * 32) >> 4), id, k > 0 ? 1u : 0u);
-          mma_commit(b_kempty(ks));
-          mma_commit(b_sfull(sbuf));
-          ++g;
-          if (++ks == C::KG) { ks = 0; kpar ^= 1u; }
-          if (++sbuf == C::SBG) sbuf = 0;
-          if (g > C::SBG && sbuf == 0) spar ^= 1u;  // s_free waits start at group SBG, parity 0
-          idle = 0;
-          nap = 32;
-          continue;
-        }
-        if (!DENSE && pv_end < 0 && c >= seen) {
-          const int f = *kq_final;  // read before the count: the count is final once f >= 0
-          seen = *kq_count;
-          if (f >= 0) pv_end = f;
-        }
-        if ((DENSE || c < seen) && (pv_end < 0 || c < pv_end)) {
-          int col, lastg;
-          if (DENSE) {
-            const int t = c % GP;
-            col = ((c / GP) % C::SBG) * 128 + t * P;
-            lastg = (t == GP - 1 || c == n_list - 1) ? 1 : 0;
-          } else {
-            __threadfence_block();
-            const int info = kq[c % C::KQ].y;
-            col = info & 0x7fff;
-            lastg = info >> 15;
-          }
-          const int vs = c % C::VS;
-          if (mbar_test_wait(b_vfull(vs), (c / C::VS) & 1) &&
-              mbar_test_wait(b_pfull(c % C::PF), (c / C::PF) & 1)) {
-            tc_fence_after();
-            const uint64_t dvs = dv + ((uint32_t)vs * C::KV_BYTES >> 4);
-#pragma unroll
-            for (int k = 0; k < P / 16; ++k)
-              mma_bf16_ts(tmem + C::COL_O, tmem + col + k * 8, dvs + ((k * 16 * 128) >> 4), ID_PV,
-                          (c > 0 || k > 0) ? 1u : 0u);
-            mma_commit(b_vempty(vs));
-            mma_commit(b_pvdone(c % C::PD));
-            if (lastg) mma_commit(b_sfree(col >> 7));  // the group's S buffer goes back
-            ++c;
-            *pv_pos = c;  // queue entry c - 1 has been read
-            idle = 0;
-            nap = 32;
-            continue;
-          }
-        }
-        if (g >= n_groups && pv_end >= 0 && c >= pv_end) break;
-        if (idle++ == 0) t_idle = globaltimer_ns();
-        if (*abort_flag) break;
-        if ((idle & 15u) == 0 && timed_out(t_idle)) {
-          give_up();
-          break;
-        }
-        if (idle > 2) {  // back off while idle: polling takes issue slots
-          __nanosleep(nap);
-          nap = min(nap * 2, 256u);
-        }
+        for (int k = 0; k < D / 16; ++k)
+          mma_bf16_ss(tmem + sbuf * 128, dq + (((k >> 2) * (C::QB * 128) + (k & 3) * 32) >> 4),
+                      dks + (((k >> 2) * (GP * P * 128) + (k & 3) * 32) >> 4), id, k > 0 ? 1u : 0u);
+        mma_commit(b_kempty(ks));
+        mma_commit(b_sfull(sbuf));
+        if (++ks == C::KG) { ks = 0; kpar ^= 1u; }
+        if (++sbuf == C::SBG) sbuf = 0;
+        if (g + 1 > C::SBG && sbuf == 0) spar ^= 1u;  // s_free waits start at group SBG
       }
       // every issued MMA completes before teardown frees TMEM
       mma_commit(b_done);
@@ -523,7 +502,7 @@ __global__ void __launch_bounds__(384, 1)
       return mx;
     };
     // leader: publish kept page c to the queue: its TMA coordinate (for the V
-    // producer), then its P column and last-of-group flag (for the MMA issuer)
+    // load), then its P column and last-of-group flag (for the PV issue)
     auto bounded_until = [&](volatile int* pos, int c) {
       if (c < C::KQ) return;
       const uint64_t t0 = globaltimer_ns();
