@@ -34,6 +34,25 @@ METRIC = "128K causal prefill attention ms & effective TFLOP/s; % of bf16 tensor
 WORKLOAD = "gqa-128k"
 
 
+# DRAM traffic (read + write) of one OSK launch at gqa-128k, from one ncu capture
+# (profiles/osk_attention_gqa-128k_traffic.md).  It describes the kernel source the
+# capture ran, identified by the hash below; any other source reports null.
+OSK_TRAFFIC = {"workload": "gqa-128k", "bytes": 2691085312, "source_sha256_16": "954522110e670352"}
+
+
+def _osk_traffic(workload: str):
+    import hashlib
+    h = hashlib.sha256()
+    csrc = os.path.join(os.path.dirname(os.path.abspath(__file__)), "block_sparse_long_kap_b200",
+                        "csrc")
+    for f in ("attn_tc.cuh", "tc_ptx.cuh", "common.cuh"):
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(fh.read())
+    if workload != OSK_TRAFFIC["workload"] or h.hexdigest()[:16] != OSK_TRAFFIC["source_sha256_16"]:
+        return None
+    return OSK_TRAFFIC["bytes"]
+
+
 def _peaks():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -323,7 +342,8 @@ def main():
         "roofline": {"kernel": "osk_attention", "bound": "tensor", "achieved": achieved,
                      "peak": peak_tflops, "unit": "TFLOP/s", "frac": achieved / peak_tflops,
                      "peak_source": f"{peak_src} bf16 sustained (kernel timed inside the step loop)",
-                     "traffic": None,
+                     "traffic": _osk_traffic(args.workload),
+                     "traffic_unit": "bytes per launch (DRAM read + write, ncu)",
                      "work": "visited FLOP = 2*Bq*P*D*(visited pages + computed pages) per launch"},
         "breakdown_ms": {"kap_select": statistics.mean(kap_ms), "osk_attention": osk_avg_ms},
         "budgets": {"kap_kept_frac": steps_visited / n_b_total,
