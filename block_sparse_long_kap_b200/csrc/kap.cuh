@@ -178,8 +178,10 @@ __global__ void __launch_bounds__(ORDER_THREADS) kap_order_kernel(
     float* __restrict__ scores_out, uint8_t* __restrict__ hrm_out, int32_t* __restrict__ order,
     int32_t* __restrict__ count, int num_q_heads, int num_q_blocks, int num_pages, int q_block,
     int page_size, float budget, int sink, int ascending, int k_cap) {
-  extern __shared__ unsigned long long keys[];  // [npow2], then the ascending flags
+  extern __shared__ unsigned long long keys[];  // [npow2] by page, then [npow2] kept keys
   __shared__ int warp_sums[32];
+  __shared__ int hist_s[256];
+  __shared__ int sel_s[3];
   __shared__ float m_s[8];
   __shared__ int arg_s[8];
   const int qb = num_q_blocks - 1 - blockIdx.x;
@@ -243,62 +245,114 @@ __global__ void __launch_bounds__(ORDER_THREADS) kap_order_kernel(
       if (hrm_out) hrm_out[row * num_pages + p] = 0;
     }
   __syncthreads();
-  // bitonic sort, descending
-  for (int kk = 2; kk <= npow2; kk <<= 1) {
-    for (int j = kk >> 1; j > 0; j >>= 1) {
-      for (int i = threadIdx.x; i < npow2; i += blockDim.x) {
-        int ixj = i ^ j;
-        if (ixj > i) {
-          unsigned long long a = keys[i], c = keys[ixj];
-          bool desc = (i & kk) == 0;
-          if (desc ? (a < c) : (a > c)) { keys[i] = c; keys[ixj] = a; }
+  // ---- threshold: the quota-th largest key among the pages that are not forced,
+  // by radix select over 8-bit digits (keys are unique: the page is in the low bits).
+  // Selected = forced pages + non-forced pages with (key >> thr_shift) >= thr_prefix.
+  const int n_nf = n_b - n_f;
+  unsigned long long thr_prefix = 0ull;
+  int thr_shift = 64;  // 64: no non-forced page (quota <= 0); -1: every one
+  if (quota >= n_nf) {
+    thr_shift = -1;
+  } else if (quota > 0) {
+    int r = quota;  // rank (1 = largest) still to find inside the current bucket
+    unsigned long long prefix = 0ull;
+    for (int shift = 56;; shift -= 8) {
+      for (int i = threadIdx.x; i < 256; i += blockDim.x) hist_s[i] = 0;
+      __syncthreads();
+      for (int p0 = 0; p0 < n_b; p0 += blockDim.x) {
+        const int p = p0 + threadIdx.x;
+        int bin = -1;
+        if (p < n_b && !(p < sink || p >= first_diag)) {
+          const unsigned long long key = keys[p];
+          if (shift == 56 || (key >> (shift + 8)) == prefix) bin = (int)((key >> shift) & 255ull);
         }
+        // warp-aggregated: many keys share their leading digits
+        const unsigned peers = __match_any_sync(0xffffffffu, bin);
+        if (bin >= 0 && (threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(&hist_s[bin], __popc(peers));
+      }
+      __syncthreads();
+      if (threadIdx.x < 32) {
+        // lane l holds bins 255 - 8 l ... 248 - 8 l (largest digits first)
+        const int lane = threadIdx.x;
+        int c[8], sum = 0;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          c[e] = hist_s[255 - 8 * lane - e];
+          sum += c[e];
+        }
+        int incl = sum;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int y = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += y;
+        }
+        int run = incl - sum;
+        if (run < r && r <= incl) {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            if (run + c[e] >= r) {
+              sel_s[0] = 255 - 8 * lane - e;  // the digit holding rank r
+              sel_s[1] = r - run;             // its rank inside that digit
+              sel_s[2] = c[e];                // keys with that digit
+              break;
+            }
+            run += c[e];
+          }
+        }
+      }
+      __syncthreads();
+      const int bin = sel_s[0];
+      r = sel_s[1];
+      prefix = (prefix << 8) | (unsigned long long)bin;
+      if (sel_s[2] == r || shift == 0) {  // the whole digit is taken, or the key is exact
+        thr_prefix = prefix;
+        thr_shift = shift;
+        break;
       }
       __syncthreads();
     }
   }
-  // selection over the sorted list: forced pages always, others while quota lasts
-  const int per = (npow2 + blockDim.x - 1) / blockDim.x;
+  auto selected = [&](int p) -> bool {
+    if (p < sink || p >= first_diag) return true;
+    if (thr_shift < 0) return true;
+    if (thr_shift >= 64) return false;
+    return (keys[p] >> thr_shift) >= thr_prefix;
+  };
+  // ---- compaction in page order (contiguous chunks per thread)
+  const int per = (n_b + blockDim.x - 1) / blockDim.x;
   const int beg = threadIdx.x * per;
-  int nf_local = 0;
-  for (int i = beg; i < beg + per && i < n_b; ++i) {
-    int page = 0x7fffffff - (int)(keys[i] & 0x7fffffffull);
-    bool forced = page < sink || page >= first_diag;
-    nf_local += !forced;
-  }
-  int nf_before = block_excl_scan(nf_local, warp_sums, nullptr);
   int sel_local = 0;
-  for (int i = beg; i < beg + per && i < n_b; ++i) {
-    int page = 0x7fffffff - (int)(keys[i] & 0x7fffffffull);
-    bool forced = page < sink || page >= first_diag;
-    bool sel = forced || (nf_before < quota);
-    if (!forced) ++nf_before;
-    sel_local += sel;
-    keys[i] = sel ? (unsigned long long)page : ~0ull;  // page id or "dropped"
-  }
+  for (int p = beg; p < beg + per && p < n_b; ++p) sel_local += selected(p);
   int total = 0;
-  int out_before = block_excl_scan(sel_local, warp_sums, &total);
+  int pos = block_excl_scan(sel_local, warp_sums, &total);
   int32_t* orow = order + row * k_cap;
-  if (!ascending) {
-    for (int i = beg; i < beg + per && i < n_b; ++i) {
-      if (keys[i] != ~0ull) orow[out_before++] = (int32_t)keys[i];
-    }
+  if (ascending) {
+    for (int p = beg; p < beg + per && p < n_b; ++p)
+      if (selected(p)) orow[pos++] = p;
   } else {
-    // list the kept pages by page id: flag array over pages, then compact
+    // kept keys only, then a bitonic sort (descending) of those
+    unsigned long long* kept = keys + npow2;
+    int m = 1;
+    while (m < total) m <<= 1;
+    for (int p = beg; p < beg + per && p < n_b; ++p)
+      if (selected(p)) kept[pos++] = keys[p];
+    for (int i = total + threadIdx.x; i < m; i += blockDim.x) kept[i] = 0ull;  // below every key
     __syncthreads();
-    int* flag = reinterpret_cast<int*>(keys + npow2);
-    for (int p = threadIdx.x; p < n_b; p += blockDim.x) flag[p] = 0;
-    __syncthreads();
-    for (int i = beg; i < beg + per && i < n_b; ++i)
-      if (keys[i] != ~0ull) flag[(int)keys[i]] = 1;
-    __syncthreads();
-    const int perp = (n_b + blockDim.x - 1) / blockDim.x;
-    const int bp = threadIdx.x * perp;
-    int cnt = 0;
-    for (int p = bp; p < bp + perp && p < n_b; ++p) cnt += flag[p];
-    int pos = block_excl_scan(cnt, warp_sums, nullptr);
-    for (int p = bp; p < bp + perp && p < n_b; ++p)
-      if (flag[p]) orow[pos++] = p;
+    for (int kk = 2; kk <= m; kk <<= 1) {
+      for (int j = kk >> 1; j > 0; j >>= 1) {
+        for (int i = threadIdx.x; i < m; i += blockDim.x) {
+          const int ixj = i ^ j;
+          if (ixj > i) {
+            const unsigned long long x = kept[i], y = kept[ixj];
+            const bool desc = (i & kk) == 0;
+            if (desc ? (x < y) : (x > y)) { kept[i] = y; kept[ixj] = x; }
+          }
+        }
+        __syncthreads();
+      }
+    }
+    for (int i = threadIdx.x; i < total; i += blockDim.x)
+      orow[i] = 0x7fffffff - (int)(kept[i] & 0x7fffffffull);
   }
   for (int j = total + threadIdx.x; j < k_cap; j += blockDim.x) orow[j] = -1;
   if (threadIdx.x == 0) {
