@@ -75,9 +75,11 @@ struct TcCfg {
   static constexpr uint32_t Q_BYTES = QB * D * 2;
   static constexpr uint32_t KV_BYTES = P * D * 2; // one page of K or of V
   static constexpr uint32_t KG_BYTES = GP * KV_BYTES;
-  static constexpr int KG = (D == 128) ? 3 : 4;   // K ring slots (groups)
-  static constexpr int VS0 = (int)(65536u / KV_BYTES);
-  static constexpr int VS = VS0 > 6 ? 6 : VS0;    // V ring slots (pages)
+  // Shared memory goes to the K ring first: every group streams K, only kept pages
+  // stream V.  D = 128, P = 64: Q 32 KB + K 4 x 32 KB + V 2 x 16 KB = 192 KB;
+  // P = 128: Q 32 KB + K 3 x 32 KB + V 2 x 32 KB = 192 KB; D = 64: 16 + 96 + 32 KB.
+  static constexpr int KG = (D == 128) ? (P == 64 ? 4 : 3) : 6;  // K ring slots (groups)
+  static constexpr int VS = (P == 64 || D == 64) ? (int)(32768u / KV_BYTES) : 2;  // V slots
   static constexpr int SBG = 3;                   // S group buffers in TMEM, 128 columns each
   static constexpr int COL_O = SBG * 128;         // O accumulator (D columns)
   static constexpr int PF = 8;                    // P-ready barrier ring (kept pages)
@@ -427,21 +429,37 @@ __global__ void __launch_bounds__(384, 1)
       bool ok = wait(b_q, 0);
       int ks = 0, sbuf = 0;
       uint32_t kpar = 0, spar = 0;  // phase parities of k_full[ks] and s_free[sbuf]
+      // The tensor core's queue is short: an issue returns when little of the group
+      // is left to run, so whether the next group can go is tested while the last
+      // MMAs of this one are still queued, and then it goes without a wait.
+      bool next_ready = false;
       for (int g = 0; ok && g < n_groups; ++g) {
-        if (!wait(b_kfull(ks), kpar)) break;
-        if (g >= C::SBG && !wait(b_sfree(sbuf), spar)) break;
+        if (!next_ready) {
+          if (!wait(b_kfull(ks), kpar)) break;
+          if (g >= C::SBG && !wait(b_sfree(sbuf), spar)) break;
+        }
         tc_fence_after();
         const uint32_t id = (g * GP + GP <= n_list) ? ID_FULL : ID_PAGE;
         const uint64_t dks = dk + ((uint32_t)ks * C::KG_BYTES >> 4);
+        // ring positions of the next group
+        const int ks1 = ks + 1 == C::KG ? 0 : ks + 1, sb1 = sbuf + 1 == C::SBG ? 0 : sbuf + 1;
+        const uint32_t kpar1 = ks + 1 == C::KG ? kpar ^ 1u : kpar;
+        const uint32_t spar1 = (g + 1 > C::SBG && sb1 == 0) ? spar ^ 1u : spar;
+        next_ready = false;
 #pragma unroll
-        for (int k = 0; k < D / 16; ++k)
+        for (int k = 0; k < D / 16; ++k) {
+          if (k == D / 16 - 2 && g + 1 < n_groups)
+            next_ready = mbar_test_wait(b_kfull(ks1), kpar1) &&
+                         (g + 1 < C::SBG || mbar_test_wait(b_sfree(sb1), spar1));
           mma_bf16_ss(tmem + sbuf * 128, dq + (((k >> 2) * (C::QB * 128) + (k & 3) * 32) >> 4),
                       dks + (((k >> 2) * (GP * P * 128) + (k & 3) * 32) >> 4), id, k > 0 ? 1u : 0u);
+        }
         mma_commit(b_kempty(ks));
         mma_commit(b_sfull(sbuf));
-        if (++ks == C::KG) { ks = 0; kpar ^= 1u; }
-        if (++sbuf == C::SBG) sbuf = 0;
-        if (g + 1 > C::SBG && sbuf == 0) spar ^= 1u;  // s_free waits start at group SBG
+        ks = ks1;
+        kpar = kpar1;
+        sbuf = sb1;
+        spar = spar1;
       }
       // every issued MMA completes before teardown frees TMEM
       mma_commit(b_done);
