@@ -37,7 +37,7 @@ WORKLOAD = "gqa-128k"
 # DRAM traffic (read + write) of one OSK launch at gqa-128k, from one ncu capture
 # (profiles/osk_attention_gqa-128k_traffic.md).  It describes the kernel source the
 # capture ran, identified by the hash below; any other source reports null.
-OSK_TRAFFIC = {"workload": "gqa-128k", "bytes": 2691085312, "source_sha256_16": "954522110e670352"}
+OSK_TRAFFIC = {"workload": "gqa-128k", "bytes": 2696647168, "source_sha256_16": "d90fe6367aa99c01"}
 
 
 def _osk_traffic(workload: str):
