@@ -1,5 +1,4 @@
-// Ordered-Skipping Kernel (and dense causal attention) on the sm_100a tensor
-// cores: TMA page loads through the page table, tcgen05.mma into TMEM, one
+// Ordered-Skipping Kernel on the sm_100a tensor cores: TMA page loads through the page table, tcgen05.mma into TMEM, one
 // query row per TMEM lane.  (gist.science/pt "CoSA" technical summary,
 // §2.3 "Estágio 2: OSK": mask-skipped pages are never loaded, "KV page
 // remapping"; in-kernel skip from the page's local max vs the running max;
@@ -28,8 +27,7 @@
 //               running max only grows, so a page skipped against an older
 //               value is skipped against the current one, and an all-skip group
 //               is settled without waiting for the other warpgroup.  A group
-//               with a page that may be kept (and the first group, and every
-//               group of dense attention) waits until the groups before it are
+//               with a page that may be kept (and the first group) waits until the groups before it are
 //               settled, reads the exact running max and exponent base of every
 //               row from shared memory and votes again; its pages are then
 //               published in list order.  One barrier round among the 128
@@ -117,7 +115,7 @@ struct TcCfg {
 // so it is kept rare; P = exp2(s - m_ref) <= 2^32, l <= 2^32 * keys, all in range
 constexpr float kRescaleLog2 = 32.0f;
 
-template <int D, int P, bool DENSE>
+template <int D, int P>
 __global__ void __launch_bounds__(384, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const TcParams prm) {
@@ -176,7 +174,7 @@ __global__ void __launch_bounds__(384, 1)
   const int n_causal = causal_pages(qb, prm.q_block, P);
   int n_list = n_causal;
   const int32_t* olist = nullptr;
-  if (!DENSE) {
+  {
     olist = prm.order + (bh * prm.num_q_blocks + qb) * prm.k_cap;
     n_list = min(max(prm.count[bh * prm.num_q_blocks + qb], 0), prm.k_cap);
     int bad = 0;
@@ -188,7 +186,7 @@ __global__ void __launch_bounds__(384, 1)
   }
   const int n_groups = (n_list + GP - 1) / GP;
   const int32_t* ptab = prm.page_table + (long long)b * prm.pages_per_seq;
-  auto page_at = [&](int j) { return DENSE ? j : __ldg(olist + j); };
+  auto page_at = [&](int j) { return __ldg(olist + j); };
   // TMA z coordinate of a logical page in the [phys page][kv head] pools
   auto coord_of = [&](int page) { return __ldg(ptab + page) * prm.num_kv_heads + hk; };
 
@@ -346,18 +344,13 @@ __global__ void __launch_bounds__(384, 1)
       const uint64_t dv = smem_desc_sw128(sV, P * 128, 1024);
       int nv = 0;                          // V loads issued
       int c = 0;                           // PV issued
-      int pv_end = DENSE ? n_list : -1;    // kept pages in all (once known)
+      int pv_end = -1;                     // kept pages in all (once known)
       bool ok = true;
       // issue the V load of kept page nv (its slot is free)
       auto load_v = [&]() {
-        int cz;
-        if (DENSE) {
-          cz = coord_of(nv);
-        } else {
-          __threadfence_block();
-          cz = kq[nv % C::KQ].x;
-          *v_pos = nv + 1;  // queue entry nv has been read
-        }
+        __threadfence_block();
+        const int cz = kq[nv % C::KQ].x;
+        *v_pos = nv + 1;  // queue entry nv has been read
         const int s = nv % C::VS;
         mbar_arrive_expect_tx(b_vfull(s), C::KV_BYTES);
 #pragma unroll
@@ -365,10 +358,10 @@ __global__ void __launch_bounds__(384, 1)
           tma_load_3d(sV + s * C::KV_BYTES + kb * (P * 128), &tm_v, b_vfull(s), kb * 64, 0, cz);
         ++nv;
       };
-      auto v_known = [&](int x) { return DENSE ? x < n_list : *vq_count > x; };
+      auto v_known = [&](int x) { return *vq_count > x; };
       while (ok) {
         // ---- kept page c known (or the list ended)?
-        if (!DENSE && pv_end < 0) {
+        if (pv_end < 0) {
           const int r = kept_ready(kq_count, c);
           if (r < 0) break;
           if (r == 0) pv_end = *kq_final;
@@ -383,17 +376,9 @@ __global__ void __launch_bounds__(384, 1)
                (nv < C::VS || mbar_test_wait(b_vempty(nv % C::VS), ((nv / C::VS) - 1) & 1)))
           load_v();
         // ---- PV of page c
-        int col, lastg;
-        if (DENSE) {
-          const int t = c % GP;
-          col = ((c / GP) % C::SBG) * 128 + t * P;
-          lastg = (t == GP - 1 || c == n_list - 1) ? 1 : 0;
-        } else {
-          __threadfence_block();
-          const int info = kq[c % C::KQ].y;
-          col = info & 0x7fff;
-          lastg = info >> 15;
-        }
+        __threadfence_block();
+        const int info = kq[c % C::KQ].y;
+        const int col = info & 0x7fff, lastg = info >> 15;
         const int vs = c % C::VS;
         if (!wait(b_vfull(vs), (c / C::VS) & 1)) break;
         if (!wait(b_pfull(c % C::PF), (c / C::PF) & 1)) break;
@@ -488,7 +473,7 @@ __global__ void __launch_bounds__(384, 1)
         fb = base;
         const int jl = base + lane;
         pid_l = jl < n_list ? page_at(jl) : 0;
-        if (!DENSE && lead_warp) cz_l = jl < n_list ? coord_of(pid_l) : 0;
+        if (lead_warp) cz_l = jl < n_list ? coord_of(pid_l) : 0;
       }
       cz = __shfl_sync(0xffffffffu, cz_l, j & 31);
       return __shfl_sync(0xffffffffu, pid_l, j & 31);
@@ -541,7 +526,7 @@ __global__ void __launch_bounds__(384, 1)
       __threadfence_block();
       *kq_count = c + 1;
     };
-    uint8_t* slog = (!DENSE && prm.skip_log) ? prm.skip_log + (bh * prm.num_q_blocks + qb) * prm.k_cap
+    uint8_t* slog = prm.skip_log ? prm.skip_log + (bh * prm.num_q_blocks + qb) * prm.k_cap
                                              : nullptr;
     // kept page c: P = exp2(s * scale - mb) (bf16 pairs) written over the page's first
     // P / 2 S columns, after the O rescale by alpha when this page moved the base
@@ -631,7 +616,7 @@ __global__ void __launch_bounds__(384, 1)
       if (lane == 0) settled[wg * 4 + q4] = g;
     };
     // the first listed page is always kept: its V can go out before any vote
-    if (!DENSE && wg == 0 && n_list > 0) {
+    if (wg == 0 && n_list > 0) {
       int cz0;
       fetch(0, cz0);
       if (leader) publish_v(0, cz0);
@@ -681,8 +666,8 @@ __global__ void __launch_bounds__(384, 1)
         }
         return bits;
       };
-      bool exact = DENSE || j == 0;
-      if (!DENSE) {
+      {
+        const bool exact = j == 0;  // the first listed page is always kept
         // ---- first vote, against the running max this warpgroup last saw (a lower
         // bound of the current one: what it skips stays skipped)
         m_run = fmaxf(m_run, st_rows[row].x);
@@ -700,7 +685,6 @@ __global__ void __launch_bounds__(384, 1)
           mark_settled(g);
           continue;
         }
-        exact = true;
       }
       // ---- exact path: the groups before this one are settled; take their state
       bool oks = okw && (g == 0 || wait_settled(g - 1));
@@ -715,13 +699,9 @@ __global__ void __launch_bounds__(384, 1)
       }
       // kept pages before this group: every earlier queue entry is published, and
       // the count is read before the vote barrier, ahead of this group's publishing
-      const int c0 = DENSE ? j : *kq_count;
+      const int c0 = *kq_count;
       bool keep[GP];
-      if (DENSE) {
-        if (!oks) { ok = false; break; }
-#pragma unroll
-        for (int t = 0; t < GP; ++t) keep[t] = t < nb;
-      } else {
+      {
         uint32_t bits = oks ? vote_bits(m_run) : 1u;
         const uint32_t all = vote_round(rnd++, bits);
         if (all & 1u) { ok = false; break; }
@@ -754,7 +734,7 @@ __global__ void __launch_bounds__(384, 1)
         st_rows[row].x = m_run;
         st_rows[row].y = m_ref;
       }
-      if (!DENSE && leader) {
+      if (leader) {
         int c = c0;
 #pragma unroll
         for (int t = 0; t < GP; ++t)
@@ -781,11 +761,10 @@ __global__ void __launch_bounds__(384, 1)
           fail = true;
         ++c;
       }
-      if (DENSE && fail) { ok = false; break; }
     }
     if (leader) {  // the second warpgroup to finish closes the queue
       __threadfence_block();
-      if (atomicAdd(wg_done, 1) == 1 && !DENSE) *kq_final = *kq_count;
+      if (atomicAdd(wg_done, 1) == 1) *kq_final = *kq_count;
     }
     // ---- epilogue: both warpgroups' row sums to one base, O / l -> bf16, LSE
     fin_rows[wg * 128 + row].x = l;
@@ -797,7 +776,7 @@ __global__ void __launch_bounds__(384, 1)
     float lt = 0.f;
     if (m_ref != -INFINITY) lt += l * ex2_approx(m_ref - M);
     if (om != -INFINITY) lt += ol * ex2_approx(om - M);
-    const int cfin = DENSE ? n_list : *kq_count;
+    const int cfin = *kq_count;
     int hv = 0;
     if (lane == 0) hv = (*abort_flag == 0 && cfin > 0) ? 1 : 0;
     bool have = __shfl_sync(0xffffffffu, hv, 0) != 0;
@@ -833,7 +812,7 @@ __global__ void __launch_bounds__(384, 1)
     if (wg == 0 && row_valid && prm.lse)
       prm.lse[bh * prm.seq_len + grow] =
           (have && lt > 0.f) ? (M + log2f(lt)) * 0.69314718055994531f : -INFINITY;
-    if (!DENSE && wg == 0 && leader && prm.computed) prm.computed[bh * prm.num_q_blocks + qb] = cfin;
+    if (wg == 0 && leader && prm.computed) prm.computed[bh * prm.num_q_blocks + qb] = cfin;
   }
 
   // ---- teardown

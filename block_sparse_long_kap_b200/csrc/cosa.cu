@@ -12,6 +12,7 @@
 #include "kap.cuh"
 #include "kap_tc.cuh"
 #include "attn_tc.cuh"
+#include "attn_dense.cuh"
 
 using namespace cosa;
 
@@ -251,7 +252,7 @@ cosa_status_t launch_kap(const cosa_shape_t* s, const cosa_kap_params_t* k, cons
   return launch_order(s, k, true, nullptr, nullptr, pm, scores, hrm, order, count, k_cap, st);
 }
 
-template <int D, int P, bool DENSE>
+template <int D, int P>
 cosa_status_t launch_tc_t(const cosa_shape_t* s, const TcParams& prm, const void* q,
                           const void* k_pool, const void* v_pool, int grid, cudaStream_t st) {
   using Cfg = TcCfg<D, P>;
@@ -261,7 +262,7 @@ cosa_status_t launch_tc_t(const cosa_shape_t* s, const TcParams& prm, const void
   if (!make_map(&mq, q, D, s->seq_len, BH, s->q_block) ||
       !make_map(&mk, k_pool, D, P, PZ, P) || !make_map(&mv, v_pool, D, P, PZ, P))
     return COSA_ERR_CUDA;
-  auto kern = attn_tc_kernel<D, P, DENSE>;
+  auto kern = attn_tc_kernel<D, P>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)Cfg::SMEM_ALLOC) != cudaSuccess)
     return COSA_ERR_CUDA;
@@ -269,14 +270,33 @@ cosa_status_t launch_tc_t(const cosa_shape_t* s, const TcParams& prm, const void
   return last_launch();
 }
 
-template <bool DENSE>
-cosa_status_t launch_attn(const cosa_shape_t* s, const TcParams& prm, const void* q,
-                          const void* k_pool, const void* v_pool, int grid, cudaStream_t st) {
+template <int D, int P>
+cosa_status_t launch_dense_t(const cosa_shape_t* s, const TcParams& prm, const void* q,
+                             const void* k_pool, const void* v_pool, int grid, cudaStream_t st) {
+  using Cfg = DenseCfg<D, P>;
+  CUtensorMap mq, mk, mv;
+  const long long BH = (long long)s->batch * s->num_q_heads;
+  const long long PZ = (long long)s->num_phys_pages * s->num_kv_heads;
+  // Q in 64-row boxes: a 128-row tile past the end of the sequence loads its
+  // first half only
+  if (!make_map(&mq, q, D, s->seq_len, BH, 64) || !make_map(&mk, k_pool, D, P, PZ, P) ||
+      !make_map(&mv, v_pool, D, P, PZ, P))
+    return COSA_ERR_CUDA;
+  auto kern = attn_dense_kernel<D, P>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)Cfg::SMEM_ALLOC) != cudaSuccess)
+    return COSA_ERR_CUDA;
+  kern<<<grid, Cfg::NT, Cfg::SMEM_ALLOC, st>>>(mq, mk, mv, prm);
+  return last_launch();
+}
+
+cosa_status_t launch_osk(const cosa_shape_t* s, const TcParams& prm, const void* q,
+                         const void* k_pool, const void* v_pool, int grid, cudaStream_t st) {
   const int D = s->head_dim, P = s->page_size;
-  if (D == 128 && P == 64) return launch_tc_t<128, 64, DENSE>(s, prm, q, k_pool, v_pool, grid, st);
-  if (D == 128 && P == 128) return launch_tc_t<128, 128, DENSE>(s, prm, q, k_pool, v_pool, grid, st);
-  if (D == 64 && P == 64) return launch_tc_t<64, 64, DENSE>(s, prm, q, k_pool, v_pool, grid, st);
-  if (D == 64 && P == 128) return launch_tc_t<64, 128, DENSE>(s, prm, q, k_pool, v_pool, grid, st);
+  if (D == 128 && P == 64) return launch_tc_t<128, 64>(s, prm, q, k_pool, v_pool, grid, st);
+  if (D == 128 && P == 128) return launch_tc_t<128, 128>(s, prm, q, k_pool, v_pool, grid, st);
+  if (D == 64 && P == 64) return launch_tc_t<64, 64>(s, prm, q, k_pool, v_pool, grid, st);
+  if (D == 64 && P == 128) return launch_tc_t<64, 128>(s, prm, q, k_pool, v_pool, grid, st);
   return COSA_ERR_UNSUPPORTED;
 }
 
@@ -452,8 +472,7 @@ cosa_status_t cosa_osk_attention(const cosa_shape_t* shape, const cosa_osk_param
   p.log2_eps = osk->eps > 0.f ? log2f(osk->eps) : -INFINITY;
   const long long grid = (long long)shape->batch * shape->num_q_heads * (shape->seq_len / shape->q_block);
   if (grid > 0x7fffffffll) return COSA_ERR_UNSUPPORTED;
-  return launch_attn<false>(shape, p, q, k_pool, v_pool, (int)grid,
-                            reinterpret_cast<cudaStream_t>(stream));
+  return launch_osk(shape, p, q, k_pool, v_pool, (int)grid, reinterpret_cast<cudaStream_t>(stream));
 }
 
 cosa_status_t cosa_dense_attention(const cosa_shape_t* shape, const void* q, const void* k_pool,
@@ -466,10 +485,17 @@ cosa_status_t cosa_dense_attention(const cosa_shape_t* shape, const void* q, con
       reinterpret_cast<uintptr_t>(v_pool) % 16 || reinterpret_cast<uintptr_t>(out) % 16)
     return COSA_ERR_INVALID_ARG;
   TcParams p = make_params(shape, out, lse, page_table);
-  const long long grid = (long long)shape->batch * shape->num_q_heads * (shape->seq_len / shape->q_block);
+  // one CTA per pair of 128-row query tiles (the q-block size plays no part)
+  const long long grid =
+      (long long)shape->batch * shape->num_q_heads * ((shape->seq_len + 255) / 256);
   if (grid > 0x7fffffffll) return COSA_ERR_UNSUPPORTED;
-  return launch_attn<true>(shape, p, q, k_pool, v_pool, (int)grid,
-                           reinterpret_cast<cudaStream_t>(stream));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int D = shape->head_dim, P = shape->page_size;
+  if (D == 128 && P == 64) return launch_dense_t<128, 64>(shape, p, q, k_pool, v_pool, (int)grid, st);
+  if (D == 128 && P == 128) return launch_dense_t<128, 128>(shape, p, q, k_pool, v_pool, (int)grid, st);
+  if (D == 64 && P == 64) return launch_dense_t<64, 64>(shape, p, q, k_pool, v_pool, (int)grid, st);
+  if (D == 64 && P == 128) return launch_dense_t<64, 128>(shape, p, q, k_pool, v_pool, (int)grid, st);
+  return COSA_ERR_UNSUPPORTED;
 }
 
 cosa_status_t cosa_get_status(cosa_stream_t stream) {

@@ -285,6 +285,58 @@ __device__ __forceinline__ void reg_tie32(uint32_t* r) {
       :
       : "memory");
 }
+// Issue a 64-column TMEM load without waiting; tmem_ld_wait64 completes it.
+#define COSA_R8(i) "=r"(r[i]), "=r"(r[i + 1]), "=r"(r[i + 2]), "=r"(r[i + 3]), \
+                   "=r"(r[i + 4]), "=r"(r[i + 5]), "=r"(r[i + 6]), "=r"(r[i + 7])
+__device__ __forceinline__ void tmem_ld64_async(uint32_t taddr, uint32_t* r) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x64.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,"
+      "%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,"
+      "%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63}, [%64];"
+      : COSA_R8(0), COSA_R8(8), COSA_R8(16), COSA_R8(24), COSA_R8(32), COSA_R8(40),
+        COSA_R8(48), COSA_R8(56)
+      : "r"(taddr)
+      : "memory");
+}
+#undef COSA_R8
+// Wait for outstanding TMEM loads, tying two 64-register destinations to the wait.
+#define COSA_T8(a, i) "+r"(a[i]), "+r"(a[i + 1]), "+r"(a[i + 2]), "+r"(a[i + 3]), \
+                      "+r"(a[i + 4]), "+r"(a[i + 5]), "+r"(a[i + 6]), "+r"(a[i + 7])
+__device__ __forceinline__ void tmem_ld_wait64x2(uint32_t* a, uint32_t* b) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;"
+               : COSA_T8(a, 0), COSA_T8(a, 8), COSA_T8(a, 16), COSA_T8(a, 24), COSA_T8(a, 32),
+                 COSA_T8(a, 40), COSA_T8(a, 48), COSA_T8(a, 56)
+               :
+               : "memory");
+  asm volatile(""
+               : COSA_T8(b, 0), COSA_T8(b, 8), COSA_T8(b, 16), COSA_T8(b, 24), COSA_T8(b, 32),
+                 COSA_T8(b, 40), COSA_T8(b, 48), COSA_T8(b, 56)
+               :
+               : "memory");
+}
+#undef COSA_T8
+// Issue a 16-column TMEM load without waiting; tmem_ld_wait16 completes it.
+__device__ __forceinline__ void tmem_ld16_async(uint32_t taddr, uint32_t* r) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_ld_wait16(uint32_t* r) {
+  asm volatile(
+      "tcgen05.wait::ld.sync.aligned;"
+      : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]),
+        "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]),
+        "+r"(r[14]), "+r"(r[15])
+      :
+      : "memory");
+}
 __device__ __forceinline__ void tmem_st_wait() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }

@@ -321,10 +321,14 @@ def test_osk_infinite_eps_with_page0_first():
 # dense
 # ---------------------------------------------------------------------------
 @pytest.mark.parametrize("case", ["tiny-2k", "gqa-4k", "wide-head-4k-p128", "gqa-2k-bq64",
-                                  "single-qblock", "single-page"])
+                                  "single-qblock", "single-page", "ragged-320", "ragged-448"])
 def test_dense_parity(case):
+    # the dense kernel takes query rows in pairs of 128-row tiles: N = 64 and 320 end
+    # on a 64-row first tile, 448 on a 64-row second tile with a 64-key diagonal block
     extra = {"single-qblock": W.small_workload("gqa-32k", 128, 2, 1, planted_frac=0.0),
-             "single-page": W.small_workload("gqa-32k", 64, 2, 1, q_block=64, planted_frac=0.0)}
+             "single-page": W.small_workload("gqa-32k", 64, 2, 1, q_block=64, planted_frac=0.0),
+             "ragged-320": W.small_workload("gqa-32k", 320, 4, 2, q_block=64, planted_frac=0.0),
+             "ragged-448": W.small_workload("gqa-32k", 448, 3, 1, q_block=64, planted_frac=0.0)}
     wl = extra[case] if case in extra else OSK_CASES[case][0]
     x = W.make_inputs(wl, seed=10)
     xd = to_dev(x)
