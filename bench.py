@@ -37,7 +37,7 @@ WORKLOAD = "gqa-128k"
 # DRAM traffic (read + write) of one OSK launch at gqa-128k, from one ncu capture
 # (profiles/osk_attention_gqa-128k_traffic.md).  It describes the kernel source the
 # capture ran, identified by the hash below; any other source reports null.
-OSK_TRAFFIC = {"workload": "gqa-128k", "bytes": 2696647168, "source_sha256_16": "d90fe6367aa99c01"}
+OSK_TRAFFIC = {"workload": "gqa-128k", "bytes": 2697283328, "source_sha256_16": "a2dc99f33d35e459"}
 
 
 def _osk_traffic(workload: str):
@@ -64,24 +64,64 @@ def _peaks():
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+    """SM clocks and clock-event (throttle) reasons of this process's GPU, sampled every
+    10 ms during the timed region through NVML (read-only queries), nvidia-smi if NVML
+    cannot be used."""
+    REASONS = (("hw_slowdown", 0x8), ("sw_thermal_slowdown", 0x20), ("hw_thermal_slowdown", 0x40),
+               ("sw_power_cap", 0x4))
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, device_index: int):
-        self.idx = device_index
+    def __init__(self, torch_device: int):
+        self.dev = torch_device
+        self.samples = []       # (sm MHz, max MHz, reason names)
         self.proc = None
         self.lines = []
+        self._stop = threading.Event()
+        self._t = None
+        self.source = None
+
+    def _nvml_handle(self):
+        import pynvml
+        import torch
+        pynvml.nvmlInit()
+        props = torch.cuda.get_device_properties(self.dev)
+        try:
+            return pynvml, pynvml.nvmlDeviceGetHandleByUUID("GPU-" + str(props.uuid))
+        except Exception:
+            bus = f"{props.pci_domain_id:08x}:{props.pci_bus_id:02x}:{props.pci_device_id:02x}.0"
+            return pynvml, pynvml.nvmlDeviceGetHandleByPciBusId(bus)
 
     def start(self):
         try:
+            nv, h = self._nvml_handle()
+            mx = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+
+            def poll():
+                while not self._stop.is_set():
+                    try:
+                        sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+                        bits = nv.nvmlDeviceGetCurrentClocksThrottleReasons(h)
+                        self.samples.append((float(sm), float(mx),
+                                             [n for n, b in self.REASONS if bits & b]))
+                    except Exception:
+                        pass
+                    self._stop.wait(0.01)
+            self._t = threading.Thread(target=poll, daemon=True)
+            self._t.start()
+            self.source = "nvml"
+            return
+        except Exception:
+            pass
+        try:
             self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.FIELDS}",
+                ["nvidia-smi", f"--id={self.dev}", f"--query-gpu={self.FIELDS}",
                  "--format=csv,noheader,nounits", "-lms", "100"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self._t = threading.Thread(target=self._read, daemon=True)
             self._t.start()
+            self.source = "nvidia-smi"
         except Exception:
             self.proc = None
 
@@ -90,29 +130,34 @@ class ClockSampler:
             self.lines.append(line.strip())
 
     def stop(self):
-        if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except Exception:
-            self.proc.kill()
-        sm, mx, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
-            parts = [p.strip() for p in ln.split(",")]
-            if len(parts) < 9:
-                continue
+        if self.source == "nvml":
+            self._stop.set()
+            self._t.join(timeout=1)
+        elif self.proc is not None:
+            self.proc.terminate()
             try:
-                sm.append(float(parts[1]))
-                mx = float(parts[2])
-            except ValueError:
-                continue
-            for n, v in zip(names, parts[5:9]):
-                if v.lower().startswith("active"):
-                    reasons.add(n)
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
-                "reasons": sorted(reasons), "samples": len(sm)}
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+            for ln in self.lines:
+                parts = [p.strip() for p in ln.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm, mx = float(parts[1]), float(parts[2])
+                except ValueError:
+                    continue
+                self.samples.append((sm, mx, [n for n, v in zip(names, parts[5:9])
+                                              if v.lower().startswith("active")]))
+        else:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["clock query unavailable"],
+                    "samples": 0}
+        sm = [x[0] for x in self.samples]
+        reasons = sorted({r for x in self.samples for r in x[2]})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": self.samples[-1][1] if self.samples else None,
+                "reasons": reasons, "samples": len(sm), "source": self.source}
 
 
 def _cpu_cores():
@@ -296,8 +341,7 @@ def main():
     assert C.cosa_get_status(stream) == 0
 
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
-    clocks = ClockSampler(torch.cuda.current_device() if "CUDA_VISIBLE_DEVICES" not in os.environ
-                          else local)
+    clocks = ClockSampler(torch.cuda.current_device())
     barrier()
     torch.cuda.synchronize(dev)
     clocks.start()
