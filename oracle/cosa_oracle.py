@@ -42,7 +42,7 @@ __all__ = [
     "gather_logical", "kap_pool_queries", "kap_pool_keys", "kap_block_scores",
     "kap_maxnorm_hrm", "rank_key", "kap_order_from_scores", "kap_select_block",
     "kap_select", "kap_order", "osk_block", "osk_attention", "dense_rows",
-    "dense_attention",
+    "dense_attention", "kap_group_scores", "kap_select_group", "expand_group_order",
 ]
 
 NEG_INF = -math.inf
@@ -285,6 +285,79 @@ def kap_order(scores: np.ndarray, hrm: np.ndarray, *, page_size: int, q_block: i
                 order[b, h, qb, :len(o)] = o
                 count[b, h, qb] = len(o)
     return order, count
+
+
+# ----------------------------------------------------------------------------
+# Group-shared selection: one ordered list per (b, h_kv, q-block) for the G
+# query heads that read the same KV head.  The pages do not describe it; the
+# readings are:
+#   S_group[p]   = max over the G heads of that head's MaxNorm score S_h[p]
+#                  (a page one head ranks highly stays high for the group),
+#   HRM_group[p] = 1 when the page holds a row max of any head's rows,
+# then the same forced pages, budget, key and order as per-head selection
+# ([TS §2.2]).  Every head of the group then runs the per-head OSK skip rule
+# on the shared list (osk_block, unchanged).
+# ----------------------------------------------------------------------------
+def kap_group_scores(S_heads: np.ndarray, hrm_heads: np.ndarray):
+    """Aggregate per-head MaxNorm scores [G][n_b] and HRM flags [G][n_b] of one
+    (b, h_kv, q-block) into the group's (S float64 [n_b], hrm uint8 [n_b])."""
+    S = np.max(np.asarray(S_heads, dtype=np.float64), axis=0)
+    hrm = (np.asarray(hrm_heads) != 0).any(axis=0).astype(np.uint8)
+    return S, hrm
+
+
+def kap_select_group(q: np.ndarray, k_pool: np.ndarray, page_table: np.ndarray, *,
+                     num_kv_heads: int, page_size: int, q_block: int, q_sub: int,
+                     k_sub: int, scale: float, budget: float, sink_pages: int,
+                     groups: Optional[Sequence] = None,
+                     qblocks: Optional[Sequence[int]] = None):
+    """Group-shared KAP over a whole problem (or a subset of (b, h_kv) groups /
+    q-blocks).  Each head's S and HRM come from the per-head steps
+    (kap_select_block); kap_group_scores aggregates them; kap_order_from_scores
+    selects and orders.  Returns dict with order int32 [B][H_kv][nQB][k_cap]
+    (-1 padded), count int32 [B][H_kv][nQB], S float64 and hrm uint8
+    [B][H_kv][nQB][nP] (zero past n_b)."""
+    B, Hq, N, D = q.shape
+    G = Hq // num_kv_heads
+    nP, nQB = N // page_size, N // q_block
+    kc = k_cap(N, q_block, page_size, sink_pages, budget)
+    order = np.full((B, num_kv_heads, nQB, kc), -1, dtype=np.int32)
+    count = np.zeros((B, num_kv_heads, nQB), dtype=np.int32)
+    S_all = np.zeros((B, num_kv_heads, nQB, nP), dtype=np.float64)
+    hrm_all = np.zeros((B, num_kv_heads, nQB, nP), dtype=np.uint8)
+    if groups is None:
+        groups = [(b, hk) for b in range(B) for hk in range(num_kv_heads)]
+    if qblocks is None:
+        qblocks = range(nQB)
+    for (b, hk) in groups:
+        k_log = gather_logical(k_pool, page_table, b, hk, N)
+        khat = kap_pool_keys(k_log, page_size, k_sub)
+        q_heads = [np.asarray(q[b, hk * G + g], dtype=np.float64) for g in range(G)]
+        for qb in qblocks:
+            Sh, Hh = [], []
+            for g in range(G):
+                _, S_g, h_g, _ = kap_select_block(q_heads[g], None, qb, q_block=q_block,
+                                                  page_size=page_size, q_sub=q_sub, k_sub=k_sub,
+                                                  scale=scale, budget=budget,
+                                                  sink_pages=sink_pages, khat=khat)
+                Sh.append(S_g)
+                Hh.append(h_g)
+            S, hr = kap_group_scores(np.stack(Sh), np.stack(Hh))
+            o = kap_order_from_scores(S, hr, qb, q_block, page_size, budget, sink_pages)
+            order[b, hk, qb, :len(o)] = o
+            count[b, hk, qb] = len(o)
+            S_all[b, hk, qb, :len(S)] = S
+            hrm_all[b, hk, qb, :len(hr)] = hr
+    return {"order": order, "count": count, "S": S_all, "hrm": hrm_all, "k_cap": kc}
+
+
+def expand_group_order(order_g: np.ndarray, count_g: np.ndarray, num_q_heads: int):
+    """Per-head lists [B][H_q][nQB][k_cap] from group lists [B][H_kv][nQB][k_cap]:
+    head h reads the list of its KV head h // G (for osk_attention)."""
+    B, Hkv = count_g.shape[:2]
+    G = num_q_heads // Hkv
+    hk = np.arange(num_q_heads) // G
+    return order_g[:, hk], count_g[:, hk]
 
 
 # ----------------------------------------------------------------------------

@@ -398,3 +398,124 @@ def test_osk_sink_plus_local_budget_is_local_sink_mask():
             torch.from_numpy(q[rows])[None], torch.from_numpy(k)[None], torch.from_numpy(v)[None],
             attn_mask=mask[None], scale=scale)[0].numpy()
         np.testing.assert_allclose(out, want, rtol=0, atol=1e-12)
+
+
+# --------------------------------------------------------------------------
+# group-shared selection: reductions and invariances
+# --------------------------------------------------------------------------
+def _group_problem(G=3, seed=11, N=256, D=16, P=16, Bq=32):
+    wl = W.small_workload("gqa-32k", N, num_q_heads=2 * G, num_kv_heads=2, head_dim=D, page_size=P,
+                          q_block=Bq, planted_frac=0.05, shuffle_pages=True)
+    x = W.make_inputs(wl, seed=seed)
+    return wl, x["q"].float().numpy(), x["k_pool"].float().numpy(), x["page_table"].numpy()
+
+
+def _kw(wl):
+    return dict(num_kv_heads=wl.num_kv_heads, page_size=wl.page_size, q_block=wl.q_block,
+                q_sub=wl.q_block // 4, k_sub=wl.page_size // 2, scale=1 / math.sqrt(wl.head_dim),
+                budget=0.3, sink_pages=1)
+
+
+def test_group_selection_with_one_head_per_group_is_per_head_selection():
+    wl = W.small_workload("gqa-32k", 256, num_q_heads=2, num_kv_heads=2, head_dim=16, page_size=16,
+                          q_block=32, planted_frac=0.05)
+    x = W.make_inputs(wl, seed=3)
+    args = (x["q"].float().numpy(), x["k_pool"].float().numpy(), x["page_table"].numpy())
+    g = O.kap_select_group(*args, **_kw(wl))
+    h = O.kap_select(*args, **_kw(wl))
+    assert np.array_equal(g["order"], h["order"]) and np.array_equal(g["count"], h["count"])
+    np.testing.assert_array_equal(g["S"], h["S"])
+
+
+def test_group_selection_does_not_depend_on_head_order():
+    wl, q, kp, pt = _group_problem()
+    base = O.kap_select_group(q, kp, pt, **_kw(wl))
+    G = 3
+    perm = np.concatenate([hk * G + np.random.default_rng(hk).permutation(G) for hk in range(2)])
+    other = O.kap_select_group(q[:, perm], kp, pt, **_kw(wl))
+    assert np.array_equal(base["order"], other["order"])
+
+
+def test_group_selection_of_identical_heads_is_each_heads_selection():
+    wl, q, kp, pt = _group_problem()
+    G = 3
+    q2 = q.copy()
+    for hk in range(2):
+        q2[:, hk * G + 1: hk * G + G] = q2[:, hk * G: hk * G + 1]
+    g = O.kap_select_group(q2, kp, pt, **_kw(wl))
+    h = O.kap_select(q2, kp, pt, **_kw(wl))
+    for hq in range(2 * G):
+        assert np.array_equal(g["order"][:, hq // G], h["order"][:, hq])
+
+
+def test_group_aggregate_with_a_dominant_head_follows_it():
+    """If one head's scores and HRM flags dominate the others' page by page, the
+    group list is that head's list (selection and order only depend on the key)."""
+    rng = np.random.default_rng(9)
+    Bq, P, sink = 16, 8, 1
+    for trial in range(40):
+        qb = int(rng.integers(1, 6))
+        n_b = O.causal_pages(qb, Bq, P)
+        G = int(rng.integers(2, 5))
+        S0 = rng.random(n_b)
+        h0 = (rng.random(n_b) < 0.3).astype(np.uint8)
+        Sh = [S0] + [S0 * rng.random(n_b) for _ in range(G - 1)]
+        Hh = [h0] + [h0 * (rng.random(n_b) < 0.5) for _ in range(G - 1)]
+        S, hr = O.kap_group_scores(np.stack(Sh), np.stack(Hh))
+        budget = float(rng.choice([0.25, 0.5, 1.0]))
+        got = O.kap_order_from_scores(S, hr, qb, Bq, P, budget, sink)
+        want = O.kap_order_from_scores(S0, h0, qb, Bq, P, budget, sink)
+        assert got.tolist() == want.tolist()
+
+
+def test_group_selection_is_best_subset_brute_force():
+    """Exhaustive check on tiny blocks: the group list is the best k_b-subset
+    (forced pages included) under (any head flags it, largest head score, lower
+    page) compared lexicographically, listed in that order."""
+    rng = np.random.default_rng(12)
+    Bq, P, sink = 16, 8, 1
+    for trial in range(40):
+        qb = int(rng.integers(0, 6))
+        n_b = O.causal_pages(qb, Bq, P)
+        G = int(rng.integers(1, 4))
+        Sh = rng.random((G, n_b)).astype(np.float32).astype(np.float64)
+        Hh = (rng.random((G, n_b)) < 0.2).astype(np.uint8)
+        S, hr = O.kap_group_scores(Sh, Hh)
+        budget = float(rng.choice([0.3, 0.5, 0.75]))
+        order = O.kap_order_from_scores(S, hr, qb, Bq, P, budget, sink)
+        forced = set(O.forced_pages(qb, Bq, P, sink))
+        k_b = O.budget_count(qb, Bq, P, sink, budget)
+
+        def tup(p):
+            return (int(any(Hh[g, p] for g in range(G))), max(float(Sh[g, p]) for g in range(G)), -p)
+        free = [p for p in range(n_b) if p not in forced]
+        best = None
+        for combo in itertools.combinations(free, k_b - len(forced)):
+            cand = sorted((tup(p) for p in combo), reverse=True)
+            if best is None or cand > best[0]:
+                best = (cand, set(combo) | forced)
+        assert set(order.tolist()) == best[1]
+        assert [tup(p) for p in order] == sorted((tup(p) for p in order), reverse=True)
+
+
+def test_group_planted_pages_come_first():
+    """Two query heads share a KV head whose planted pages every query of the
+    last 256 rows is drawn towards: the group list opens with them."""
+    wl = W.small_workload("tiny-2k", 2048, num_q_heads=4, num_kv_heads=2)
+    x = W.make_inputs(wl, seed=0)
+    r = O.kap_select_group(x["q"].float().numpy(), x["k_pool"].float().numpy(),
+                           x["page_table"].numpy(), num_kv_heads=2, page_size=64, q_block=64,
+                           q_sub=16, k_sub=16, scale=1 / math.sqrt(64), budget=0.25, sink_pages=1)
+    nQB = wl.seq_len // wl.q_block
+    for hk in range(2):
+        planted = set(x["planted"][0, hk].tolist())
+        for qb in range(nQB - 256 // wl.q_block, nQB):
+            assert set(r["order"][0, hk, qb, :3].tolist()) == planted
+
+
+def test_expand_group_order_maps_heads_to_their_kv_head():
+    og = np.arange(2 * 3 * 4 * 5, dtype=np.int32).reshape(2, 3, 4, 5)
+    cg = np.arange(2 * 3 * 4, dtype=np.int32).reshape(2, 3, 4)
+    o, c = O.expand_group_order(og, cg, 6)
+    for h in range(6):
+        assert np.array_equal(o[:, h], og[:, h // 2]) and np.array_equal(c[:, h], cg[:, h // 2])
