@@ -19,6 +19,7 @@ __all__ = [
     "cosa_status_string", "cosa_version", "cosa_kap_kcap", "cosa_kap_workspace_size",
     "cosa_kap_select", "cosa_kap_select_noalloc", "cosa_kap_order", "cosa_osk_attention",
     "cosa_dense_attention", "cosa_get_status", "EXPORTED_SYMBOLS", "NOALLOC_SCRATCH_BYTES",
+    "cosa_kap_select_group",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -27,7 +28,7 @@ library_path = os.path.join(_HERE, "libcosa.so")
 EXPORTED_SYMBOLS = (
     "cosa_status_string", "cosa_version", "cosa_kap_kcap", "cosa_kap_workspace_size",
     "cosa_kap_select", "cosa_kap_select_noalloc", "cosa_kap_order", "cosa_osk_attention",
-    "cosa_dense_attention", "cosa_get_status",
+    "cosa_dense_attention", "cosa_get_status", "cosa_kap_select_group",
 )
 
 # Largest workspace the allocation-free Stage-1 entry point accepts (cosa.h).
@@ -137,6 +138,7 @@ def lib():
     L.cosa_kap_workspace_size.argtypes = [P(_Shape), P(_Kap), P(sz)]
     L.cosa_kap_select.argtypes = [P(_Shape), P(_Kap), vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
     L.cosa_kap_select_noalloc.argtypes = [P(_Shape), P(_Kap), vp, vp, vp, vp, vp, vp, vp, vp]
+    L.cosa_kap_select_group.argtypes = [P(_Shape), P(_Kap), vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
     L.cosa_kap_order.argtypes = [P(_Shape), P(_Kap), vp, vp, vp, vp, vp]
     L.cosa_osk_attention.argtypes = [P(_Shape), P(_Osk), vp, vp, vp, vp, vp, vp, i32, vp, vp, vp,
                                      vp, vp]
@@ -230,6 +232,33 @@ def cosa_kap_select(shape: Shape, kap: KapParams, q, k_pool, page_table, order, 
                                  _ptr(page_table), _ptr(order), _ptr(count), _ptr(scores),
                                  _ptr(hrm), _ptr(workspace), nbytes, _stream(stream)),
            "cosa_kap_select")
+
+
+def cosa_kap_select_group(shape: Shape, kap: KapParams, q, k_pool, page_table, order, count,
+                          workspace, scores=None, hrm=None, stream=None) -> None:
+    """Stage 1 with one list per KV head (group-shared selection): order
+    [B][H_kv][nQB][k_cap], count [B][H_kv][nQB]; scores / hrm, when given,
+    [B][H_kv][nQB][nP]."""
+    import torch
+    s, k = shape.c(), kap.c(shape)
+    B, Hq, Hk, N, D = shape.batch, shape.num_q_heads, shape.num_kv_heads, shape.seq_len, shape.head_dim
+    kc = cosa_kap_kcap(shape, kap)
+    _expect(q, "q", torch.bfloat16, (B, Hq, N, D))
+    _expect(k_pool, "k_pool", torch.bfloat16, _kv_shape(shape))
+    _expect(page_table, "page_table", torch.int32, (B, s.pages_per_seq))
+    _expect(order, "order", torch.int32, (B, Hk, shape.num_q_blocks, kc))
+    _expect(count, "count", torch.int32, (B, Hk, shape.num_q_blocks))
+    if scores is not None:
+        _expect(scores, "scores", torch.float32, (B, Hk, shape.num_q_blocks, shape.num_pages))
+    if hrm is not None:
+        _expect(hrm, "hrm", torch.uint8, (B, Hk, shape.num_q_blocks, shape.num_pages))
+    if workspace is None or not workspace.is_cuda:
+        raise ValueError("workspace must be a CUDA tensor")
+    nbytes = workspace.numel() * workspace.element_size()
+    _check(lib().cosa_kap_select_group(ctypes.byref(s), ctypes.byref(k), _ptr(q), _ptr(k_pool),
+                                       _ptr(page_table), _ptr(order), _ptr(count), _ptr(scores),
+                                       _ptr(hrm), _ptr(workspace), nbytes, _stream(stream)),
+           "cosa_kap_select_group")
 
 
 def cosa_kap_select_noalloc(shape: Shape, kap: KapParams, q, k_pool, page_table, order, count,

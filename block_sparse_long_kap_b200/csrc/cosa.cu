@@ -166,17 +166,19 @@ cosa_status_t launch_score_tc(const ScoreParams& prm, const CUtensorMap* maps, i
 cosa_status_t launch_order(const cosa_shape_t* s, const cosa_kap_params_t* k, bool from_a,
                            const float* scores, const uint8_t* hrm, const KapPageMax& pm,
                            float* scores_out, uint8_t* hrm_out, int32_t* order, int32_t* count,
-                           int k_cap, cudaStream_t st) {
+                           int k_cap, cudaStream_t st, bool group = false) {
   const int N = s->seq_len, P = s->page_size, Bq = s->q_block, nP = N / P, nQB = N / Bq;
   int npow2 = 1;
   while (npow2 < nP) npow2 <<= 1;
   const size_t smem = (size_t)npow2 * 8 * 2;  // keys by page, then the kept keys
   if (smem > 200 * 1024) return COSA_ERR_UNSUPPORTED;
-  auto kern = from_a ? kap_order_kernel<true> : kap_order_kernel<false>;
+  if (from_a && (group ? pm.group : 1) * pm.R > ORDER_MAX_ROWS) return COSA_ERR_UNSUPPORTED;
+  auto kern = !from_a ? kap_order_kernel<false, false>
+                      : (group ? kap_order_kernel<true, true> : kap_order_kernel<true, false>);
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
       cudaSuccess)
     return COSA_ERR_CUDA;
-  dim3 grid(nQB, s->batch * s->num_q_heads);
+  dim3 grid(nQB, s->batch * (group ? s->num_kv_heads : s->num_q_heads));
   kern<<<grid, ORDER_THREADS, smem, st>>>(scores, hrm, pm, scores_out, hrm_out, order, count,
                                           s->num_q_heads, nQB, nP, Bq, P, k->budget,
                                           k->sink_pages, k->ascending, k_cap);
@@ -187,7 +189,7 @@ template <int D>
 cosa_status_t launch_kap(const cosa_shape_t* s, const cosa_kap_params_t* k, const void* q,
                          const void* k_pool, const int32_t* page_table, int32_t* order,
                          int32_t* count, float* scores, uint8_t* hrm, const KapLayout& L,
-                         uint8_t* ws, int k_cap, cudaStream_t st) {
+                         uint8_t* ws, int k_cap, cudaStream_t st, bool group = false) {
   const int B = s->batch, Hq = s->num_q_heads, Hk = s->num_kv_heads, N = s->seq_len;
   const int P = s->page_size, Bq = s->q_block, nP = N / P, nQB = N / Bq;
   const int R = Bq / k->q_sub, T = P / k->k_sub, G = Hq / Hk;
@@ -249,7 +251,8 @@ cosa_status_t launch_kap(const cosa_shape_t* s, const cosa_kap_params_t* k, cons
   pm.num_kv_heads = Hk;
   pm.group = G;
   pm.R = R;
-  return launch_order(s, k, true, nullptr, nullptr, pm, scores, hrm, order, count, k_cap, st);
+  return launch_order(s, k, true, nullptr, nullptr, pm, scores, hrm, order, count, k_cap, st,
+                      group);
 }
 
 template <int D, int P>
@@ -410,6 +413,30 @@ cosa_status_t cosa_kap_select(const cosa_shape_t* shape, const cosa_kap_params_t
                            k_cap, st);
   return launch_kap<64>(shape, kap, q, k_pool, page_table, order, count, scores, hrm, L, ws, k_cap,
                         st);
+}
+
+cosa_status_t cosa_kap_select_group(const cosa_shape_t* shape, const cosa_kap_params_t* kap,
+                                    const void* q, const void* k_pool, const int32_t* page_table,
+                                    int32_t* order, int32_t* count, float* scores, uint8_t* hrm,
+                                    void* workspace, size_t workspace_bytes, cosa_stream_t stream) {
+  cosa_status_t e = check_shape(shape);
+  if (e != COSA_OK) return e;
+  if ((e = check_kap(shape, kap)) != COSA_OK) return e;
+  if (kap->ascending) return COSA_ERR_UNSUPPORTED;
+  if (!q || !k_pool || !page_table || !order || !count) return COSA_ERR_INVALID_ARG;
+  KapLayout L = kap_layout(shape, kap);
+  if (!workspace || workspace_bytes < L.total) return COSA_ERR_WORKSPACE;
+  if (reinterpret_cast<uintptr_t>(workspace) % 256) return COSA_ERR_WORKSPACE;
+  if (reinterpret_cast<uintptr_t>(q) % 16 || reinterpret_cast<uintptr_t>(k_pool) % 16)
+    return COSA_ERR_INVALID_ARG;
+  const int k_cap = kcap_of(shape, kap);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* ws = reinterpret_cast<uint8_t*>(workspace);
+  if (shape->head_dim == 128)
+    return launch_kap<128>(shape, kap, q, k_pool, page_table, order, count, scores, hrm, L, ws,
+                           k_cap, st, true);
+  return launch_kap<64>(shape, kap, q, k_pool, page_table, order, count, scores, hrm, L, ws, k_cap,
+                        st, true);
 }
 
 cosa_status_t cosa_kap_select_noalloc(const cosa_shape_t* shape, const cosa_kap_params_t* kap,

@@ -134,7 +134,10 @@ __global__ void __launch_bounds__(256) kap_pool_kernel(
 
 // ---------------------------------------------------------------------------
 // K3: MaxNorm + HRM (from the page maxima) or caller-given scores, then
-// selection + ordering.  grid.x = nQB (heaviest first), grid.y = B * H_q.
+// selection + ordering.  grid.x = nQB (heaviest first), grid.y = B * H_q, or
+// B * H_kv in group mode: one list for the G query heads of a KV head, from
+// S[p] = max over the heads of each head's MaxNorm score and HRM[p] = any head's
+// flag (the group-shared selection; the pages describe per-head selection only).
 // key = hrm << 63 | float_bits(S) << 31 | (2^31 - 1 - page): larger is better.
 // ---------------------------------------------------------------------------
 constexpr int ORDER_THREADS = 512;
@@ -172,7 +175,9 @@ struct KapPageMax {
   int num_kv_heads, group, R;
 };
 
-template <bool FROM_A>
+constexpr int ORDER_MAX_ROWS = 64;  // representative rows read by one CTA (G * R in group mode)
+
+template <bool FROM_A, bool GROUP>
 __global__ void __launch_bounds__(ORDER_THREADS) kap_order_kernel(
     const float* __restrict__ scores, const uint8_t* __restrict__ hrm, KapPageMax pm,
     float* __restrict__ scores_out, uint8_t* __restrict__ hrm_out, int32_t* __restrict__ order,
@@ -182,8 +187,8 @@ __global__ void __launch_bounds__(ORDER_THREADS) kap_order_kernel(
   __shared__ int warp_sums[32];
   __shared__ int hist_s[256];
   __shared__ int sel_s[3];
-  __shared__ float m_s[8];
-  __shared__ int arg_s[8];
+  __shared__ float m_s[ORDER_MAX_ROWS];
+  __shared__ int arg_s[ORDER_MAX_ROWS];
   const int qb = num_q_blocks - 1 - blockIdx.x;
   const int bhq = blockIdx.y;
   const long long row = (long long)bhq * num_q_blocks + qb;
@@ -196,17 +201,27 @@ __global__ void __launch_bounds__(ORDER_THREADS) kap_order_kernel(
   while (npow2 < n_b) npow2 <<= 1;
 
   const float* arow = nullptr;
+  const int n_heads = GROUP ? pm.group : 1;  // heads whose rows this CTA reads
   if (FROM_A) {
-    const int b = bhq / num_q_heads, h = bhq % num_q_heads;
-    const int hk = h / pm.group, g = h % pm.group;
+    int b, hk, g;
+    if (GROUP) {
+      b = bhq / pm.num_kv_heads;
+      hk = bhq % pm.num_kv_heads;
+      g = 0;
+    } else {
+      b = bhq / num_q_heads;
+      const int h = bhq % num_q_heads;
+      hk = h / pm.group;
+      g = h % pm.group;
+    }
     const int GR = pm.group * pm.R;
     const long long slab = (long long)b * pm.num_kv_heads + hk;
     const long long rep0 = (slab * num_q_blocks + qb) * GR + (long long)g * pm.R;
     arow = pm.a + slab * GR * cum_pages(num_q_blocks, q_block, page_size) +
            (long long)GR * cum_pages(qb, q_block, page_size) + (long long)g * pm.R * n_b;
-    if (threadIdx.x < pm.R) {
-      m_s[threadIdx.x] = pm.row_max[rep0 + threadIdx.x];
-      arg_s[threadIdx.x] = pm.row_arg[rep0 + threadIdx.x];
+    for (int t = threadIdx.x; t < n_heads * pm.R; t += blockDim.x) {
+      m_s[t] = pm.row_max[rep0 + t];
+      arg_s[t] = pm.row_arg[rep0 + t];
     }
     __syncthreads();
   }
@@ -219,14 +234,18 @@ __global__ void __launch_bounds__(ORDER_THREADS) kap_order_kernel(
       float sv;
       int flag;
       if (FROM_A) {
-        // MaxNorm: S[p] = mean_r exp(a[r][p] - m_r); HRM: p is some row's first maximum
+        // MaxNorm: S[p] = mean_r exp(a[r][p] - m_r); HRM: p is some row's first
+        // maximum (group mode: the largest head score, any head's flag)
         sv = 0.f;
         flag = 0;
-        for (int r = 0; r < pm.R; ++r) {
-          sv += expf(arow[(long long)r * n_b + p] - m_s[r]);
-          flag |= (arg_s[r] == p);
+        for (int g = 0; g < n_heads; ++g) {
+          float sg = 0.f;
+          for (int r = g * pm.R; r < (g + 1) * pm.R; ++r) {
+            sg += expf(arow[(long long)r * n_b + p] - m_s[r]);
+            flag |= (arg_s[r] == p);
+          }
+          sv = fmaxf(sv, sg * invR);
         }
-        sv *= invR;
       } else {
         sv = srow[p];
         flag = hrow[p] != 0;

@@ -137,6 +137,22 @@ cosa_status_t cosa_kap_select(const cosa_shape_t* shape, const cosa_kap_params_t
                               int32_t* order, int32_t* count, float* scores, uint8_t* hrm,
                               void* workspace, size_t workspace_bytes, cosa_stream_t stream);
 
+/* Stage 1 with one list per KV head: the G query heads that read KV head h_kv
+ * share one ordered list per q-block (the group-shared selection; the pages
+ * describe per-head selection only, this is the next step after it).  Every
+ * step up to the per-head MaxNorm scores S_h[p] and flags HRM_h[p] is that of
+ * cosa_kap_select; then
+ *   S[p] = max over the group's heads of S_h[p], HRM[p] = OR of HRM_h[p],
+ * and the same forced pages, budget, key and order.  order is
+ * int32 [B][H_kv][nQB][k_cap] (-1 padded), count int32 [B][H_kv][nQB]; scores /
+ * hrm (may be NULL) get the group's S and flags, [B][H_kv][nQB][nP].  Same
+ * workspace as cosa_kap_select.  kap->ascending must be 0
+ * (COSA_ERR_UNSUPPORTED otherwise); G * (q_block / q_sub) > 64 is unsupported. */
+cosa_status_t cosa_kap_select_group(const cosa_shape_t* shape, const cosa_kap_params_t* kap,
+                                    const void* q, const void* k_pool, const int32_t* page_table,
+                                    int32_t* order, int32_t* count, float* scores, uint8_t* hrm,
+                                    void* workspace, size_t workspace_bytes, cosa_stream_t stream);
+
 /* Largest workspace (cosa_kap_workspace_size) that cosa_kap_select_noalloc
  * accepts: 128 MiB, enough for a 32K-token layer with 32 query heads. */
 #define COSA_KAP_NOALLOC_SCRATCH_BYTES (128u << 20)
