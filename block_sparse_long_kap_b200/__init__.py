@@ -19,7 +19,7 @@ __all__ = [
     "cosa_status_string", "cosa_version", "cosa_kap_kcap", "cosa_kap_workspace_size",
     "cosa_kap_select", "cosa_kap_select_noalloc", "cosa_kap_order", "cosa_osk_attention",
     "cosa_dense_attention", "cosa_get_status", "EXPORTED_SYMBOLS", "NOALLOC_SCRATCH_BYTES",
-    "cosa_kap_select_group",
+    "cosa_kap_select_group", "cosa_osk_attention_group",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -28,7 +28,7 @@ library_path = os.path.join(_HERE, "libcosa.so")
 EXPORTED_SYMBOLS = (
     "cosa_status_string", "cosa_version", "cosa_kap_kcap", "cosa_kap_workspace_size",
     "cosa_kap_select", "cosa_kap_select_noalloc", "cosa_kap_order", "cosa_osk_attention",
-    "cosa_dense_attention", "cosa_get_status", "cosa_kap_select_group",
+    "cosa_dense_attention", "cosa_get_status", "cosa_kap_select_group", "cosa_osk_attention_group",
 )
 
 # Largest workspace the allocation-free Stage-1 entry point accepts (cosa.h).
@@ -143,6 +143,8 @@ def lib():
     L.cosa_osk_attention.argtypes = [P(_Shape), P(_Osk), vp, vp, vp, vp, vp, vp, i32, vp, vp, vp,
                                      vp, vp]
     L.cosa_dense_attention.argtypes = [P(_Shape), vp, vp, vp, vp, vp, vp, vp]
+    L.cosa_osk_attention_group.argtypes = [P(_Shape), P(_Osk), vp, vp, vp, vp, vp, vp, i32, vp, vp,
+                                           vp, vp, vp]
     L.cosa_get_status.argtypes = [vp]
     for name in EXPORTED_SYMBOLS:
         if name not in ("cosa_status_string", "cosa_version"):
@@ -325,6 +327,36 @@ def cosa_osk_attention(shape: Shape, osk: OskParams, q, k_pool, v_pool, page_tab
                                     _ptr(v_pool), _ptr(page_table), _ptr(order), _ptr(count), kc,
                                     _ptr(out), _ptr(lse), _ptr(computed), _ptr(skip_log),
                                     _stream(stream)), "cosa_osk_attention")
+
+
+def cosa_osk_attention_group(shape: Shape, osk: OskParams, q, k_pool, v_pool, page_table, order,
+                             count, out, lse=None, computed=None, skip_log=None,
+                             stream=None) -> None:
+    """Stage 2 over group-shared lists: order [B][H_kv][nQB][k_cap], count
+    [B][H_kv][nQB]; every query head runs its own skip rule on its KV head's list."""
+    import torch
+    s, o = shape.c(), osk.c()
+    B, Hq, Hk, N, D = shape.batch, shape.num_q_heads, shape.num_kv_heads, shape.seq_len, shape.head_dim
+    if order is None or order.dim() != 4:
+        raise ValueError("order must be int32 [B][H_kv][nQB][k_cap]")
+    kc = int(order.shape[-1])
+    _expect(q, "q", torch.bfloat16, (B, Hq, N, D))
+    _expect(k_pool, "k_pool", torch.bfloat16, _kv_shape(shape))
+    _expect(v_pool, "v_pool", torch.bfloat16, _kv_shape(shape))
+    _expect(page_table, "page_table", torch.int32, (B, s.pages_per_seq))
+    _expect(order, "order", torch.int32, (B, Hk, shape.num_q_blocks, kc))
+    _expect(count, "count", torch.int32, (B, Hk, shape.num_q_blocks))
+    _expect(out, "out", torch.bfloat16, (B, Hq, N, D))
+    if lse is not None:
+        _expect(lse, "lse", torch.float32, (B, Hq, N))
+    if computed is not None:
+        _expect(computed, "computed", torch.int32, (B, Hq, shape.num_q_blocks))
+    if skip_log is not None:
+        _expect(skip_log, "skip_log", torch.uint8, (B, Hq, shape.num_q_blocks, kc))
+    _check(lib().cosa_osk_attention_group(ctypes.byref(s), ctypes.byref(o), _ptr(q), _ptr(k_pool),
+                                          _ptr(v_pool), _ptr(page_table), _ptr(order), _ptr(count),
+                                          kc, _ptr(out), _ptr(lse), _ptr(computed), _ptr(skip_log),
+                                          _stream(stream)), "cosa_osk_attention_group")
 
 
 def cosa_dense_attention(shape: Shape, q, k_pool, v_pool, page_table, out, lse=None,

@@ -13,6 +13,7 @@
 #include "kap_tc.cuh"
 #include "attn_tc.cuh"
 #include "attn_dense.cuh"
+#include "attn_gqa.cuh"
 
 using namespace cosa;
 
@@ -293,6 +294,24 @@ cosa_status_t launch_dense_t(const cosa_shape_t* s, const TcParams& prm, const v
   return last_launch();
 }
 
+template <int D, int P>
+cosa_status_t launch_pair_t(const cosa_shape_t* s, const TcParams& prm, const void* q,
+                            const void* k_pool, const void* v_pool, int grid, cudaStream_t st) {
+  using Cfg = PairCfg<D, P>;
+  CUtensorMap mq, mk, mv;
+  const long long BH = (long long)s->batch * s->num_q_heads;
+  const long long PZ = (long long)s->num_phys_pages * s->num_kv_heads;
+  if (!make_map(&mq, q, D, s->seq_len, BH, s->q_block) || !make_map(&mk, k_pool, D, P, PZ, P) ||
+      !make_map(&mv, v_pool, D, P, PZ, P))
+    return COSA_ERR_CUDA;
+  auto kern = attn_pair_kernel<D, P>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)Cfg::SMEM_ALLOC) != cudaSuccess)
+    return COSA_ERR_CUDA;
+  kern<<<grid, Cfg::NT, Cfg::SMEM_ALLOC, st>>>(mq, mk, mv, prm);
+  return last_launch();
+}
+
 cosa_status_t launch_osk(const cosa_shape_t* s, const TcParams& prm, const void* q,
                          const void* k_pool, const void* v_pool, int grid, cudaStream_t st) {
   const int D = s->head_dim, P = s->page_size;
@@ -500,6 +519,40 @@ cosa_status_t cosa_osk_attention(const cosa_shape_t* shape, const cosa_osk_param
   const long long grid = (long long)shape->batch * shape->num_q_heads * (shape->seq_len / shape->q_block);
   if (grid > 0x7fffffffll) return COSA_ERR_UNSUPPORTED;
   return launch_osk(shape, p, q, k_pool, v_pool, (int)grid, reinterpret_cast<cudaStream_t>(stream));
+}
+
+cosa_status_t cosa_osk_attention_group(const cosa_shape_t* shape, const cosa_osk_params_t* osk,
+                                       const void* q, const void* k_pool, const void* v_pool,
+                                       const int32_t* page_table, const int32_t* order,
+                                       const int32_t* count, int32_t k_cap, void* out, float* lse,
+                                       int32_t* computed, uint8_t* skip_log, cosa_stream_t stream) {
+  cosa_status_t e = check_shape(shape);
+  if (e != COSA_OK) return e;
+  if (!osk || !(osk->eps >= 0.f)) return COSA_ERR_INVALID_ARG;
+  if (!q || !k_pool || !v_pool || !page_table || !order || !count || !out)
+    return COSA_ERR_INVALID_ARG;
+  if (k_cap <= 0 || k_cap > shape->seq_len / shape->page_size) return COSA_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(q) % 16 || reinterpret_cast<uintptr_t>(k_pool) % 16 ||
+      reinterpret_cast<uintptr_t>(v_pool) % 16 || reinterpret_cast<uintptr_t>(out) % 16)
+    return COSA_ERR_INVALID_ARG;
+  TcParams p = make_params(shape, out, lse, page_table);
+  p.order = order;
+  p.count = count;
+  p.computed = computed;
+  p.skip_log = skip_log;
+  p.k_cap = k_cap;
+  p.log2_eps = osk->eps > 0.f ? log2f(osk->eps) : -INFINITY;
+  const int G = shape->num_q_heads / shape->num_kv_heads;
+  const long long grid = (long long)shape->batch * shape->num_kv_heads *
+                         (shape->seq_len / shape->q_block) * ((G + 1) / 2);
+  if (grid > 0x7fffffffll) return COSA_ERR_UNSUPPORTED;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int D = shape->head_dim, P = shape->page_size;
+  if (D == 128 && P == 64) return launch_pair_t<128, 64>(shape, p, q, k_pool, v_pool, (int)grid, st);
+  if (D == 128 && P == 128) return launch_pair_t<128, 128>(shape, p, q, k_pool, v_pool, (int)grid, st);
+  if (D == 64 && P == 64) return launch_pair_t<64, 64>(shape, p, q, k_pool, v_pool, (int)grid, st);
+  if (D == 64 && P == 128) return launch_pair_t<64, 128>(shape, p, q, k_pool, v_pool, (int)grid, st);
+  return COSA_ERR_UNSUPPORTED;
 }
 
 cosa_status_t cosa_dense_attention(const cosa_shape_t* shape, const void* q, const void* k_pool,

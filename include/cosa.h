@@ -203,6 +203,19 @@ cosa_status_t cosa_osk_attention(const cosa_shape_t* shape, const cosa_osk_param
                                  const int32_t* count, int32_t k_cap, void* out, float* lse,
                                  int32_t* computed, uint8_t* skip_log, cosa_stream_t stream);
 
+/* Stage 2 over group-shared lists (cosa_kap_select_group): every query head h
+ * runs the per-head skip rule and online softmax of cosa_osk_attention on the
+ * list of its KV head h / G; the result equals cosa_osk_attention given each
+ * head its KV head's list.  Two query heads of a KV head run in one CTA and
+ * share every K tile load.  order int32 [B][H_kv][nQB][k_cap], count int32
+ * [B][H_kv][nQB]; out, lse, computed (int32 [B][H_q][nQB]) and skip_log (uint8
+ * [B][H_q][nQB][k_cap]) as for cosa_osk_attention. */
+cosa_status_t cosa_osk_attention_group(const cosa_shape_t* shape, const cosa_osk_params_t* osk,
+                                       const void* q, const void* k_pool, const void* v_pool,
+                                       const int32_t* page_table, const int32_t* order,
+                                       const int32_t* count, int32_t k_cap, void* out, float* lse,
+                                       int32_t* computed, uint8_t* skip_log, cosa_stream_t stream);
+
 /* Dense causal attention over the same paged cache (every causal page in page
  * order, no skipping): the comparison point for the sparse path's speedup.
  * lse may be NULL. */
