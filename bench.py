@@ -160,6 +160,24 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(sm), "source": self.source}
 
 
+def max_over_ranks(v: float, world: int, device) -> float:
+    """The largest of the ranks' values (every rank gets it); each rank times its
+    own shard, and the job takes as long as the slowest."""
+    if world <= 1:
+        return v
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def weak_value(world: int, flop_per_rank: float, ms: float) -> float:
+    """Whole-job TFLOP/s when every rank runs its own layer (weak scaling): all
+    ranks' work over the slowest rank's time."""
+    return world * flop_per_rank / (ms * 1e-3) / 1e12
+
+
 def _cpu_cores():
     try:
         return len(os.sched_getaffinity(0))
@@ -296,7 +314,7 @@ def main():
     dev = torch.device("cuda", local)
     if world > 1:
         import datetime
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=dev)
 
     wl = W.WORKLOADS[args.workload]
@@ -330,12 +348,6 @@ def main():
         if world > 1:
             dist.barrier()
 
-    def max_over_ranks(v: float) -> float:
-        if world == 1:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
 
     if args.dense_only:
         dense_flop = 4.0 * B * Hq * D * N * (N + 1) / 2
@@ -379,14 +391,14 @@ def main():
     torch.cuda.synchronize(dev)
     barrier()
     clk = clocks.stop()
-    total_ms = max_over_ranks(t_start.elapsed_time(t_end))
+    total_ms = max_over_ranks(t_start.elapsed_time(t_end), world, dev)
     kap_ms = [e[0].elapsed_time(e[1]) for e in evs]
     osk_ms = [e[1].elapsed_time(e[2]) for e in evs]
     assert C.cosa_get_status(stream) == 0
 
     ms_per_step = total_ms / args.steps
     dense_flop = wl.dense_flops()
-    value = world * dense_flop / (ms_per_step * 1e-3) / 1e12
+    value = weak_value(world, dense_flop, ms_per_step)
 
     # algorithmic work of the dominant kernel (OSK) for the roofline
     cnt = count.to(torch.int64)
@@ -427,6 +439,44 @@ def main():
         "budgets": {"kap_kept_frac": steps_visited / n_b_total,
                     "osk_computed_frac": steps_computed / n_b_total},
     }
+    # ---- end to end through the C-ABI with host buffers (every rank, every N) ---
+    def e2e_leg():
+        qh = x["q"].cpu().pin_memory()
+        kh = x["k_pool"].cpu().pin_memory()
+        vh = x["v_pool"].cpu().pin_memory()
+        pth = x["page_table"].cpu().pin_memory()
+        outh = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        qd, kd, vd, ptd = (torch.empty_like(x["q"]), torch.empty_like(x["k_pool"]),
+                           torch.empty_like(x["v_pool"]), torch.empty_like(x["page_table"]))
+        e2e_steps = max(1, min(args.steps, 3))
+
+        def e2e_step():
+            qd.copy_(qh, non_blocking=True)
+            kd.copy_(kh, non_blocking=True)
+            vd.copy_(vh, non_blocking=True)
+            ptd.copy_(pth, non_blocking=True)
+            C.cosa_kap_select(shape, kap, qd, kd, ptd, order, count, ws, stream=stream)
+            C.cosa_osk_attention(shape, osk, qd, kd, vd, ptd, order, count, out, stream=stream)
+            outh.copy_(out, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize(dev)
+        barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(e2e_steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier()
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, world, dev)
+        h2d = sum(t.numel() * t.element_size() for t in (qh, kh, vh, pth))
+        d2h = outh.numel() * outh.element_size()
+        return {"value": weak_value(world, dense_flop, e2e_ms), "unit": "TFLOP/s",
+                "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+    if world > 1:
+        line["e2e"] = e2e_leg()
     if args.no_extras or world > 1:
         if rank == 0:
             print(json.dumps(line), flush=True)
@@ -474,39 +524,58 @@ def main():
                       "speedup_vs_dense": dense_ms / (ms + statistics.mean(kap_ms))})
     line["eps_sweep"] = sweep
 
-    # ---- end to end through the C-ABI with host buffers ---------------------
-    qh = x["q"].cpu().pin_memory()
-    kh = x["k_pool"].cpu().pin_memory()
-    vh = x["v_pool"].cpu().pin_memory()
-    pth = x["page_table"].cpu().pin_memory()
-    outh = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-    qd, kd, vd, ptd = (torch.empty_like(x["q"]), torch.empty_like(x["k_pool"]),
-                       torch.empty_like(x["v_pool"]), torch.empty_like(x["page_table"]))
-    e2e_steps = max(1, min(args.steps, 3))
+    # ---- group-shared selection: one list per KV head and q-block (KAP group +
+    # OSK over head pairs), same budget and eps; quality against the dense output
+    Hk = wl.num_kv_heads
+    og = torch.empty(B, Hk, shape.num_q_blocks, kc, dtype=torch.int32, device=dev)
+    cg = torch.empty(B, Hk, shape.num_q_blocks, dtype=torch.int32, device=dev)
+    outg = torch.empty_like(out)
+    compg = torch.empty_like(computed)
 
-    def e2e_step():
-        qd.copy_(qh, non_blocking=True)
-        kd.copy_(kh, non_blocking=True)
-        vd.copy_(vh, non_blocking=True)
-        ptd.copy_(pth, non_blocking=True)
-        C.cosa_kap_select(shape, kap, qd, kd, ptd, order, count, ws, stream=stream)
-        C.cosa_osk_attention(shape, osk, qd, kd, vd, ptd, order, count, out, stream=stream)
-        outh.copy_(out, non_blocking=True)
+    def gstep(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        C.cosa_kap_select_group(shape, kap, x["q"], x["k_pool"], x["page_table"], og, cg, ws,
+                                stream=stream)
+        if ev is not None:
+            ev[1].record(stream)
+        C.cosa_osk_attention_group(shape, osk, x["q"], x["k_pool"], x["v_pool"], x["page_table"],
+                                   og, cg, outg, computed=compg, stream=stream)
+        if ev is not None:
+            ev[2].record(stream)
 
-    e2e_step()
+    for _ in range(args.warmup):
+        gstep()
     torch.cuda.synchronize(dev)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(e2e_steps):
-        e2e_step()
-    e1.record(stream)
+    gevs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    for i in range(args.steps):
+        gstep(gevs[i])
     torch.cuda.synchronize(dev)
-    e2e_ms = e0.elapsed_time(e1) / e2e_steps
-    h2d = sum(t.numel() * t.element_size() for t in (qh, kh, vh, pth))
-    d2h = outh.numel() * outh.element_size()
-    line["e2e"] = {"value": dense_flop / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
-                   "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
-    del qh, kh, vh, outh
+    assert C.cosa_get_status(stream) == 0
+    g_kap = statistics.mean(e[0].elapsed_time(e[1]) for e in gevs)
+    g_osk = statistics.mean(e[1].elapsed_time(e[2]) for e in gevs)
+    g_ms = g_kap + g_osk
+    # the per-head output at this eps, for the same quality measure
+    C.cosa_osk_attention(shape, osk, x["q"], x["k_pool"], x["v_pool"], x["page_table"], order,
+                         count, out, computed=computed, stream=stream)
+    torch.cuda.synchronize(dev)
+    dref = dense_out.float()
+
+    def rel_l2(a):
+        return float((a.float() - dref).norm() / dref.norm())
+
+    G_ = Hq // Hk
+    vis_g = G_ * int(cg.to(torch.int64).sum().item())
+    comp_g = int(compg.to(torch.int64).sum().item())
+    vis_tf = tile * (vis_g + comp_g) / (g_osk * 1e-3) / 1e12
+    line["group_shared"] = {
+        "kap_ms": g_kap, "osk_ms": g_osk, "ms": g_ms, "tflops": dense_flop / (g_ms * 1e-3) / 1e12,
+        "speedup_vs_dense": dense_ms / g_ms, "speedup_vs_per_head": ms_per_step / g_ms,
+        "visited_tflops": vis_tf, "visited_frac_vs_burst": vis_tf / burst,
+        "kap_kept_frac": vis_g / n_b_total, "osk_computed_frac": comp_g / n_b_total,
+        "rel_l2_vs_dense": rel_l2(outg), "per_head_rel_l2_vs_dense": rel_l2(out)}
+
+    line["e2e"] = e2e_leg()
 
     # ---- CPU oracle on a bounded sample of the same workload ----------------
     xh = {"q": x["q"][:, :1].cpu(), "k_pool": x["k_pool"][:, :1].cpu(),
