@@ -115,3 +115,29 @@ def test_null_pointers_and_bad_eps_rejected_before_launch():
                                16, 1 << 40, None) == 5
     # null shape
     assert lib.cosa_dense_attention(None, 16, 16, 16, 16, 16, None, None) == 1
+
+
+def test_group_entry_points_reject_bad_arguments_before_launch():
+    lib = C.lib()
+    shp = C.Shape(1, 4, 2, 1024, 128, 64, 128)
+    s = shp.c()
+    k = C.KapParams().c(shp)
+    o = C._Osk(1e-4)
+    # null q / negative eps / k_cap out of range / misaligned output
+    assert lib.cosa_osk_attention_group(ctypes.byref(s), ctypes.byref(o), None, 16, 16, 16, 16, 16,
+                                        4, 16, None, None, None, None) == 1
+    ob = C._Osk(-1.0)
+    assert lib.cosa_osk_attention_group(ctypes.byref(s), ctypes.byref(ob), 16, 16, 16, 16, 16, 16,
+                                        4, 16, None, None, None, None) == 1
+    assert lib.cosa_osk_attention_group(ctypes.byref(s), ctypes.byref(o), 16, 16, 16, 16, 16, 16,
+                                        0, 16, None, None, None, None) == 1
+    assert lib.cosa_osk_attention_group(ctypes.byref(s), ctypes.byref(o), 16, 16, 16, 16, 16, 16,
+                                        4, 24, None, None, None, None) == 1
+    # workspace missing / too small; ascending lists unsupported in group mode
+    assert lib.cosa_kap_select_group(ctypes.byref(s), ctypes.byref(k), 16, 16, 16, 16, 16, None,
+                                     None, None, 0, None) == 5
+    assert lib.cosa_kap_select_group(ctypes.byref(s), ctypes.byref(k), 16, 16, 16, 16, 16, None,
+                                     None, 256, 100, None) == 5
+    ka = C.KapParams(ascending=True).c(shp)
+    assert lib.cosa_kap_select_group(ctypes.byref(s), ctypes.byref(ka), 16, 16, 16, 16, 16, None,
+                                     None, 256, 1 << 40, None) == 2
