@@ -171,7 +171,8 @@ cosa_status_t launch_order(const cosa_shape_t* s, const cosa_kap_params_t* k, bo
   const int N = s->seq_len, P = s->page_size, Bq = s->q_block, nP = N / P, nQB = N / Bq;
   int npow2 = 1;
   while (npow2 < nP) npow2 <<= 1;
-  const size_t smem = (size_t)npow2 * 8 * 2;  // keys by page, then the kept keys
+  // keys by page, then the kept keys (at least one warp's worth for the register sort)
+  const size_t smem = (size_t)(npow2 + (npow2 < 32 ? 32 : npow2)) * 8;
   if (smem > 200 * 1024) return COSA_ERR_UNSUPPORTED;
   if (from_a && (group ? pm.group : 1) * pm.R > ORDER_MAX_ROWS) return COSA_ERR_UNSUPPORTED;
   auto kern = !from_a ? kap_order_kernel<false, false>

@@ -183,7 +183,7 @@ __global__ void __launch_bounds__(ORDER_THREADS) kap_order_kernel(
     float* __restrict__ scores_out, uint8_t* __restrict__ hrm_out, int32_t* __restrict__ order,
     int32_t* __restrict__ count, int num_q_heads, int num_q_blocks, int num_pages, int q_block,
     int page_size, float budget, int sink, int ascending, int k_cap) {
-  extern __shared__ unsigned long long keys[];  // [npow2] by page, then [npow2] kept keys
+  extern __shared__ unsigned long long keys[];  // [npow2] by page, then max(npow2, 32) kept keys
   __shared__ int warp_sums[32];
   __shared__ int hist_s[256];
   __shared__ int sel_s[3];
@@ -355,10 +355,30 @@ __global__ void __launch_bounds__(ORDER_THREADS) kap_order_kernel(
     while (m < total) m <<= 1;
     for (int p = beg; p < beg + per && p < n_b; ++p)
       if (selected(p)) kept[pos++] = keys[p];
-    for (int i = total + threadIdx.x; i < m; i += blockDim.x) kept[i] = 0ull;  // below every key
+    const int mw = m < 32 ? 32 : m;  // whole warps take part in the register stages
+    for (int i = total + threadIdx.x; i < mw; i += blockDim.x) kept[i] = 0ull;  // below every key
     __syncthreads();
-    for (int kk = 2; kk <= m; kk <<= 1) {
-      for (int j = kk >> 1; j > 0; j >>= 1) {
+    // Bitonic sort, descending.  Stages pairing elements 32 or more apart go through
+    // shared memory; the others pair lanes of one warp and run in registers (element i
+    // is held by lane i % 32 of its warp; the partner of i is i ^ j).
+    auto warp_stages = [&](int k_lo, int k_hi) {
+      for (int i0 = 0; i0 < mw; i0 += blockDim.x) {
+        const int i = i0 + (int)threadIdx.x;
+        if (i >= mw) continue;  // whole warps: mw and blockDim are multiples of 32
+        unsigned long long x = kept[i];
+        for (int kk = k_lo; kk <= k_hi; kk <<= 1)
+          for (int j = (kk >> 1) < 16 ? (kk >> 1) : 16; j > 0; j >>= 1) {
+            const unsigned long long y = __shfl_xor_sync(0xffffffffu, x, j);
+            const bool keep_max = ((i & j) == 0) == ((i & kk) == 0);
+            x = keep_max ? (x > y ? x : y) : (x < y ? x : y);
+          }
+        kept[i] = x;
+      }
+      __syncthreads();
+    };
+    if (m >= 2) warp_stages(2, m < 32 ? m : 32);  // every size up to 32 at once
+    for (int kk = 64; kk <= m; kk <<= 1) {
+      for (int j = kk >> 1; j >= 32; j >>= 1) {
         for (int i = threadIdx.x; i < m; i += blockDim.x) {
           const int ixj = i ^ j;
           if (ixj > i) {
@@ -369,6 +389,7 @@ __global__ void __launch_bounds__(ORDER_THREADS) kap_order_kernel(
         }
         __syncthreads();
       }
+      warp_stages(kk, kk);
     }
     for (int i = threadIdx.x; i < total; i += blockDim.x)
       orow[i] = 0x7fffffff - (int)(kept[i] & 0x7fffffffull);
