@@ -8,16 +8,28 @@
 // Listed pages are taken in list order in groups of 128 keys (two pages of 64
 // keys, or one of 128): one QK^T of N = 128 per group, into one of three S
 // buffers in TMEM.
-//   warps 0, 1  K producers: group g is loaded by warp g % 2 into ring slot
-//               g % KG, so two TMA streams run side by side (warp 0 also loads
-//               Q).  The physical page comes from the page table; no multicast.
+//   warp 0 (1)  Q and K loads: group g into ring slot g % KG; warp 0 loads every
+//               group when there are two QK^T issuers, else warps 0 and 1 take
+//               the groups in turn.  The physical page comes from the page table,
+//               looked up ahead of the copies; no multicast.
 //   warp 2      V loads and PV (one thread): loads V of the kept pages only,
 //               once the vote has kept them (up to VS pages ahead), so a skipped
 //               page costs its K tile and its share of one QK^T, nothing more;
 //               then O += P_c V_c with P read from TMEM.
-//   warp 3      QK^T issuer (one thread); allocates TMEM.  An MMA issue blocks its
-//               thread while the tensor core works, so QK^T and PV have a thread
-//               each.
+//   warps 3, 1  QK^T issuers (one thread each): warp 3 the even groups and warp 1
+//               the odd ones (warp 3 all of them when KG is odd); warp 3 also
+//               allocates TMEM.  An MMA issue blocks its thread until the tensor
+//               core's short queue has room, so what a thread does between two
+//               groups (barrier tests, ring positions) leaves the tensor core
+//               idle unless another thread's MMAs are queued.
+// Barrier phases are waited on by parity, which only tells a phase from the one
+// before it: a waiter must have seen the previous phase of the same barrier
+// complete.  With two issuers the groups no longer complete in order, so the S
+// buffer barriers are kept per group parity: group g reports S full on
+// s_full[g % 3][g % 2], and the group that reuses its buffer (g + 3, the other
+// parity) waits on s_free[g % 3][(g + 1) % 2]; each barrier then serves one
+// thread's groups in order, 6 groups apart.  A K slot serves groups of one
+// parity when KG is even, which is why a single issuer is kept when it is odd.
 //   warps 4-7,  softmax, two warpgroups taking the groups in turn (even groups
 //   8-11        warpgroup 0, odd groups warpgroup 1).  Thread (warp % 4, lane)
 //               owns query row 32 (warp % 4) + lane, which is its TMEM lane,
@@ -79,6 +91,8 @@ struct TcCfg {
   static constexpr int KG = (D == 128) ? (P == 64 ? 4 : 3) : 6;  // K ring slots (groups)
   static constexpr int VS = (P == 64 || D == 64) ? (int)(32768u / KV_BYTES) : 2;  // V slots
   static constexpr int SBG = 3;                   // S group buffers in TMEM, 128 columns each
+  static constexpr bool TWO_QK = KG % 2 == 0;     // two QK^T issuers (K slots of one parity)
+  static constexpr int NPROD = TWO_QK ? 1 : 2;     // K producer warps (warp 1 when free)
   static constexpr int COL_O = SBG * 128;         // O accumulator (D columns)
   static constexpr int PF = 8;                    // P-ready barrier ring (kept pages)
   static constexpr int PD = 8;                    // PV-done barrier ring (kept pages)
@@ -88,27 +102,30 @@ struct TcCfg {
   static constexpr uint32_t OFF_K = OFF_Q + Q_BYTES;
   static constexpr uint32_t OFF_V = OFF_K + KG * KG_BYTES;
   static constexpr uint32_t OFF_BAR = OFF_V + VS * KV_BYTES;
-  // q, k_full/empty, v_full/empty, s_full/free, p_full, pv_done, done (QK), done (PV)
-  static constexpr int NBAR = 1 + 2 * KG + 2 * VS + 2 * SBG + PF + PD + 2;
+  // q, k_full/empty, v_full/empty, s_full/free [SBG][2], p_full, pv_done, done (QK even, odd), done (PV)
+  static constexpr int NBAR = 1 + 2 * KG + 2 * VS + 4 * SBG + PF + PD + 3;
   static constexpr uint32_t OFF_MISC = (OFF_BAR + NBAR * 8 + 127) & ~127u;  // vector-aligned
   // misc: +0 TMEM address, +4 abort flag, +8 kept count (P location published),
   //       +12 final kept count (-1 while the votes run), +16 V progress,
   //       +20 warpgroups finished, +36 PV progress, +40 kept count (TMA coordinate
   //       published), +48 votes [2 wg][2][4], +128 kept queue [KQ] {TMA coordinate,
   //       P column | last << 15}, +640 settled state rows [128] {m_run, m_ref},
-  //       +1664 last settled group per softmax warp [8], +2688 final rows [2][128] {l, m_ref}
+  //       +1664 last settled group per softmax warp [8], +1696 S-ready flag per
+  //       warpgroup [2], +2688 final rows [2][128] {l, m_ref}
   static constexpr uint32_t M_STATE = 640, M_SETTLED = 1664, M_FIN = 2688;
   static constexpr uint32_t MISC_BYTES = M_FIN + 2 * 128 * 8;
   static constexpr uint32_t SMEM = OFF_MISC + MISC_BYTES;
   static constexpr uint32_t SMEM_ALLOC = SMEM + 1024;  // 1024-byte alignment slack
   static_assert(COL_O + D <= TMEM_COLS, "TMEM budget");
   static_assert(VS >= 2 && KG >= 2, "ring depths");
+  static_assert(SBG % 2 == 1, "S buffer barriers per group parity: 2 * SBG groups apart");
   static_assert(PF >= 2 * SBG + 1 && PD >= 2 * SBG + 1, "barrier rings cover the kept pages in flight");
   static_assert(SMEM_ALLOC <= 227 * 1024, "shared memory budget");
   static_assert(OFF_MISC % 128 == 0, "16-byte vector access to the vote words");
   static_assert(KV_BYTES % 1024 == 0, "tiles stay 1024-byte aligned for the 128-byte swizzle");
   static_assert(48 + 64 <= 128 && 128 + 8 * KQ <= M_STATE, "vote words and kept queue fit");
-  static_assert(M_STATE + 128 * 8 <= M_SETTLED && M_SETTLED + 8 * 4 <= M_FIN, "state rows and flags fit");
+  static_assert(M_STATE + 128 * 8 <= M_SETTLED && M_SETTLED + 8 * 4 + 2 * 4 <= M_FIN,
+                "state rows and flags fit");
 };
 
 // m_ref trails the running max by < 2^32: a rescale waits for the PV before it,
@@ -116,7 +133,7 @@ struct TcCfg {
 constexpr float kRescaleLog2 = 32.0f;
 
 template <int D, int P>
-__global__ void __launch_bounds__(384, 1)
+__global__ void __launch_bounds__(TcCfg<D, P>::NT, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const TcParams prm) {
   using C = TcCfg<D, P>;
@@ -133,13 +150,17 @@ __global__ void __launch_bounds__(384, 1)
   auto b_kempty = [&](int s) { return bar + 8u * (1 + C::KG + s); };
   auto b_vfull = [&](int s) { return bar + 8u * (1 + 2 * C::KG + s); };
   auto b_vempty = [&](int s) { return bar + 8u * (1 + 2 * C::KG + C::VS + s); };
-  auto b_sfull = [&](int s) { return bar + 8u * (1 + 2 * C::KG + 2 * C::VS + s); };
-  auto b_sfree = [&](int s) { return bar + 8u * (1 + 2 * C::KG + 2 * C::VS + C::SBG + s); };
-  auto b_pfull = [&](int s) { return bar + 8u * (1 + 2 * C::KG + 2 * C::VS + 2 * C::SBG + s); };
-  auto b_pvdone = [&](int s) {
-    return bar + 8u * (1 + 2 * C::KG + 2 * C::VS + 2 * C::SBG + C::PF + s);
+  // S buffer s, group parity p (see the note on barrier phases above)
+  auto b_sfull = [&](int s, int p) { return bar + 8u * (1 + 2 * C::KG + 2 * C::VS + 2 * s + p); };
+  auto b_sfree = [&](int s, int p) {
+    return bar + 8u * (1 + 2 * C::KG + 2 * C::VS + 2 * C::SBG + 2 * s + p);
   };
-  const uint32_t b_done = bar + 8u * (C::NBAR - 2);
+  auto b_pfull = [&](int s) { return bar + 8u * (1 + 2 * C::KG + 2 * C::VS + 4 * C::SBG + s); };
+  auto b_pvdone = [&](int s) {
+    return bar + 8u * (1 + 2 * C::KG + 2 * C::VS + 4 * C::SBG + C::PF + s);
+  };
+  const uint32_t b_done = bar + 8u * (C::NBAR - 3);      // QK^T, even groups
+  const uint32_t b_done_odd = bar + 8u * (C::NBAR - 2);  // QK^T, odd groups
   const uint32_t b_done_pv = bar + 8u * (C::NBAR - 1);
   uint8_t* misc = sg + C::OFF_MISC;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(misc);
@@ -152,6 +173,7 @@ __global__ void __launch_bounds__(384, 1)
   volatile int* vq_count = reinterpret_cast<volatile int*>(misc + 40);
   volatile int* votes = reinterpret_cast<volatile int*>(misc + 48);     // [2][2][4]
   volatile int* settled = reinterpret_cast<volatile int*>(misc + C::M_SETTLED);  // [8]
+  volatile int* s_ok = reinterpret_cast<volatile int*>(misc + C::M_SETTLED + 32);  // [2]
   volatile int2* kq = reinterpret_cast<volatile int2*>(misc + 128);     // [KQ]
   volatile float2* st_rows = reinterpret_cast<volatile float2*>(misc + C::M_STATE);  // [128]
   volatile float2* fin_rows = reinterpret_cast<volatile float2*>(misc + C::M_FIN);    // [2][128]
@@ -195,10 +217,12 @@ __global__ void __launch_bounds__(384, 1)
     mbar_init(b_q, 1);
     for (int s = 0; s < C::KG; ++s) { mbar_init(b_kfull(s), 1); mbar_init(b_kempty(s), 1); }
     for (int s = 0; s < C::VS; ++s) { mbar_init(b_vfull(s), 1); mbar_init(b_vempty(s), 1); }
-    for (int s = 0; s < C::SBG; ++s) { mbar_init(b_sfull(s), 1); mbar_init(b_sfree(s), 1); }
+    for (int s = 0; s < C::SBG; ++s)
+      for (int p = 0; p < 2; ++p) { mbar_init(b_sfull(s, p), 1); mbar_init(b_sfree(s, p), 1); }
     for (int s = 0; s < C::PF; ++s) mbar_init(b_pfull(s), 4);
     for (int s = 0; s < C::PD; ++s) mbar_init(b_pvdone(s), 1);
     mbar_init(b_done, 1);
+    mbar_init(b_done_odd, 1);
     mbar_init(b_done_pv, 1);
     *abort_flag = 0;
     *kq_count = 0;
@@ -279,8 +303,8 @@ __global__ void __launch_bounds__(384, 1)
     }
   };
 
-  if (warp < 2) {
-    // ================= K producers: groups g = warp, warp + 2, ... ==============
+  if (warp < C::NPROD) {
+    // ================= Q (warp 0), then K: groups g = warp, warp + NPROD, ... ========
     const int kp = warp;
     if (kp == 0 && lane == 0) {
       prefetch_tmap(&tm_q);
@@ -292,16 +316,27 @@ __global__ void __launch_bounds__(384, 1)
     }
     int last = -1;  // last group this warp issued
     bool ok = true;
-    // lane l holds the coordinate of page l % GP of this warp's group m0 + l / GP
-    for (int m0 = 0; ok && kp + 2 * m0 < n_groups; m0 += 32 / GP) {
-      int cz_l = 0;
-      {
-        const int gl = kp + 2 * (m0 + lane / GP);
-        const int jl = gl * GP + lane % GP;
-        if (gl < n_groups && jl < n_list) cz_l = coord_of(page_at(jl));
-      }
-      for (int mm = 0; mm < 32 / GP; ++mm) {
-        const int g = kp + 2 * (m0 + mm);
+    constexpr int GB = 32 / GP;  // this warp's groups per block of page-table lookups
+    // lane l: the logical page of page l % GP of this warp's group i0 + l / GP (-1 past
+    // the list).  Page ids are read two blocks ahead and TMA coordinates one block
+    // ahead, so the copies never wait on those global loads.
+    auto page_of_lane = [&](int i0) -> int {
+      const int jl = (kp + C::NPROD * (i0 + lane / GP)) * GP + lane % GP;
+      return jl < n_list ? page_at(jl) : -1;
+    };
+    const int n_mine = (n_groups - kp + C::NPROD - 1) / C::NPROD;  // this warp's groups
+    int cz_next;
+    {
+      const int pg0 = page_of_lane(0);
+      cz_next = pg0 >= 0 ? coord_of(pg0) : 0;
+    }
+    int pg_next = GB < n_mine ? page_of_lane(GB) : -1;
+    for (int i0 = 0; ok && i0 < n_mine; i0 += GB) {
+      const int cz_l = cz_next;
+      cz_next = pg_next >= 0 ? coord_of(pg_next) : 0;
+      pg_next = i0 + 2 * GB < n_mine ? page_of_lane(i0 + 2 * GB) : -1;
+      for (int mm = 0; mm < GB; ++mm) {
+        const int g = kp + C::NPROD * (i0 + mm);
         if (g >= n_groups) break;
         const int s = g % C::KG;
         if (g >= C::KG) {
@@ -330,7 +365,7 @@ __global__ void __launch_bounds__(384, 1)
       const uint64_t t0 = globaltimer_ns();
       if (kp == 0)
         while (!mbar_try_wait(b_q, 0) && globaltimer_ns() - t0 < tmo) {}
-      for (int g = last; g >= 0 && g > last - 2 * C::KG; g -= 2)
+      for (int g = last; g >= 0 && g > last - C::NPROD * C::KG; g -= C::NPROD)
         while (!mbar_try_wait(b_kfull(g % C::KG), (g / C::KG) & 1) &&
                globaltimer_ns() - t0 < tmo) {}
     }
@@ -378,7 +413,7 @@ __global__ void __launch_bounds__(384, 1)
         // ---- PV of page c
         __threadfence_block();
         const int info = kq[c % C::KQ].y;
-        const int col = info & 0x7fff, lastg = info >> 15;
+        const int col = info & 0x7fff, lastg = (info >> 15) & 1, gpar = (info >> 16) & 1;
         const int vs = c % C::VS;
         if (!wait(b_vfull(vs), (c / C::VS) & 1)) break;
         if (!wait(b_pfull(c % C::PF), (c / C::PF) & 1)) break;
@@ -390,7 +425,8 @@ __global__ void __launch_bounds__(384, 1)
                       (c > 0 || k > 0) ? 1u : 0u);
         mma_commit(b_vempty(vs));
         mma_commit(b_pvdone(c % C::PD));
-        if (lastg) mma_commit(b_sfree(col >> 7));  // the group's S buffer goes back
+        // the group's S buffer goes back, to the issuer of the group that reuses it
+        if (lastg) mma_commit(b_sfree(col >> 7, gpar ^ 1));
         ++c;
         *pv_pos = c;  // queue entry c - 1 has been read
       }
@@ -402,9 +438,11 @@ __global__ void __launch_bounds__(384, 1)
       for (int x = c; x < nv; ++x)
         while (!mbar_try_wait(b_vfull(x % C::VS), (x / C::VS) & 1) && globaltimer_ns() - t0 < tmo) {}
     }
-  } else if (warp == 3) {
+  } else if (warp == 3 || (C::TWO_QK && warp == 1)) {
     if (lane == 0) {
-      // ================= QK^T issuer, one group of 128 keys at a time =============
+      // ================= QK^T issuers: warp 3 the even groups, warp 1 the odd ones ====
+      const int par = warp == 3 ? 0 : 1;
+      constexpr int step = C::TWO_QK ? 2 : 1;
       constexpr uint32_t ID_FULL = idesc_bf16_f32(128, 128, 0);
       constexpr uint32_t ID_PAGE = idesc_bf16_f32(128, P, 0);  // a lone last page
       // descriptors of the tile bases; a 16-byte aligned offset below 256 KB adds to
@@ -412,46 +450,43 @@ __global__ void __launch_bounds__(384, 1)
       const uint64_t dq = smem_desc_sw128(sQ, 16, 1024);
       const uint64_t dk = smem_desc_sw128(sK, 16, 1024);
       bool ok = wait(b_q, 0);
-      int ks = 0, sbuf = 0;
-      uint32_t kpar = 0, spar = 0;  // phase parities of k_full[ks] and s_free[sbuf]
-      // The tensor core's queue is short: an issue returns when little of the group
-      // is left to run, so whether the next group can go is tested while the last
-      // MMAs of this one are still queued, and then it goes without a wait.
+      // Group g reads K ring slot g % KG (phase g / KG) and writes S buffer g % SBG,
+      // which its previous user, group g - SBG, gave back on s_free[g % SBG][g % 2] in
+      // phase (g - SBG) / (2 SBG).  Whether this thread's next group can go is tested
+      // while the last MMAs of this one are still queued, and then it goes without a
+      // wait.
+      auto sfree_phase = [](int g) { return ((g - C::SBG) / (2 * C::SBG)) & 1; };
       bool next_ready = false;
-      for (int g = 0; ok && g < n_groups; ++g) {
+      for (int g = par; ok && g < n_groups; g += step) {
+        const int ks = g % C::KG, sbuf = g % C::SBG;
         if (!next_ready) {
-          if (!wait(b_kfull(ks), kpar)) break;
-          if (g >= C::SBG && !wait(b_sfree(sbuf), spar)) break;
+          if (!wait(b_kfull(ks), (g / C::KG) & 1)) break;
+          if (g >= C::SBG && !wait(b_sfree(sbuf, g & 1), sfree_phase(g))) break;
         }
         tc_fence_after();
         const uint32_t id = (g * GP + GP <= n_list) ? ID_FULL : ID_PAGE;
         const uint64_t dks = dk + ((uint32_t)ks * C::KG_BYTES >> 4);
-        // ring positions of the next group
-        const int ks1 = ks + 1 == C::KG ? 0 : ks + 1, sb1 = sbuf + 1 == C::SBG ? 0 : sbuf + 1;
-        const uint32_t kpar1 = ks + 1 == C::KG ? kpar ^ 1u : kpar;
-        const uint32_t spar1 = (g + 1 > C::SBG && sb1 == 0) ? spar ^ 1u : spar;
+        const int g2 = g + step;
         next_ready = false;
 #pragma unroll
         for (int k = 0; k < D / 16; ++k) {
-          if (k == D / 16 - 2 && g + 1 < n_groups)
-            next_ready = mbar_test_wait(b_kfull(ks1), kpar1) &&
-                         (g + 1 < C::SBG || mbar_test_wait(b_sfree(sb1), spar1));
+          if (k == D / 16 - 2 && g2 < n_groups)
+            next_ready = mbar_test_wait(b_kfull(g2 % C::KG), (g2 / C::KG) & 1) &&
+                         (g2 < C::SBG || mbar_test_wait(b_sfree(g2 % C::SBG, g2 & 1),
+                                                        sfree_phase(g2)));
           mma_bf16_ss(tmem + sbuf * 128, dq + (((k >> 2) * (C::QB * 128) + (k & 3) * 32) >> 4),
                       dks + (((k >> 2) * (GP * P * 128) + (k & 3) * 32) >> 4), id, k > 0 ? 1u : 0u);
         }
         mma_commit(b_kempty(ks));
-        mma_commit(b_sfull(sbuf));
-        ks = ks1;
-        kpar = kpar1;
-        sbuf = sb1;
-        spar = spar1;
+        mma_commit(b_sfull(sbuf, g & 1));
       }
-      // every issued MMA completes before teardown frees TMEM
-      mma_commit(b_done);
+      // every MMA this thread issued completes before teardown frees TMEM
+      const uint32_t bd = par == 0 ? b_done : b_done_odd;
+      mma_commit(bd);
       const uint64_t t0 = globaltimer_ns();
-      while (!mbar_try_wait(b_done, 0) && globaltimer_ns() - t0 < tmo) {}
+      while (!mbar_try_wait(bd, 0) && globaltimer_ns() - t0 < tmo) {}
     }
-  } else {
+  } else if (warp >= 4) {
     // ================= softmax: two warpgroups taking the groups in turn ========
     const int wg = (warp - 4) >> 2;      // groups g with g % 2 == wg
     const int q4 = warp & 3;             // TMEM lane quarter
@@ -632,8 +667,12 @@ __global__ void __launch_bounds__(384, 1)
         czp[t] = 0;
         key0[t] = t < nb ? fetch(j + t, czp[t]) * P : 0;
       }
-      // ---- row maxima of the group's pages, read from TMEM
-      const bool okw = !fail && wait_warp(b_sfull(sb), (g / C::SBG) & 1);
+      // ---- row maxima of the group's pages, read from TMEM.  One lane waits for S and
+      // the named barrier brings the four warps along together (apart, each warp
+      // waking on its own, the vote barrier waited for the last of them).
+      if (leader) s_ok[wg] = wait(b_sfull(sb, wg), (g / (2 * C::SBG)) & 1) ? 1 : 0;
+      named_bar_sync(1 + wg, 128);
+      const bool okw = !fail && s_ok[wg] != 0;
       if (okw) tc_fence_after();
       // (one copy of the per-page code: the loop is not unrolled)
       float ml0 = -INFINITY, ml1 = -INFINITY;
@@ -680,7 +719,7 @@ __global__ void __launch_bounds__(384, 1)
           if (leader) {
             if (slog)
               for (int t = 0; t < nb; ++t) slog[j + t] = 1;
-            mbar_arrive(b_sfree(sb));
+            mbar_arrive(b_sfree(sb, wg ^ 1));
           }
           mark_settled(g);
           continue;
@@ -742,11 +781,11 @@ __global__ void __launch_bounds__(384, 1)
             if (slog) slog[j + t] = keep[t] ? 0 : 1;
             if (keep[t]) {
               if (j + t > 0) publish_v(c, czp[t]);
-              publish_info(c, (sb * 128 + t * P) | ((t == lastk ? 1 : 0) << 15));
+              publish_info(c, (sb * 128 + t * P) | ((t == lastk ? 1 : 0) << 15) | (wg << 16));
               ++c;
             }
           }
-        if (nk == 0) mbar_arrive(b_sfree(sb));  // nothing kept: the S buffer goes back now
+        if (nk == 0) mbar_arrive(b_sfree(sb, wg ^ 1));  // nothing kept: the S buffer goes back now
       }
       mark_settled(g);
       // ---- P of the kept pages; their PV follows in list order
