@@ -347,15 +347,16 @@ __global__ void __launch_bounds__(TcCfg<D, P>::NT, 1)
         int cz[GP];
 #pragma unroll
         for (int t = 0; t < GP; ++t) cz[t] = __shfl_sync(0xffffffffu, cz_l, mm * GP + t);
-        if (lane == 0) {
-          mbar_arrive_expect_tx(b_kfull(s), (uint32_t)nb * C::KV_BYTES);
+        // lane 0 posts the group's bytes, then lane t copies page t: copies issued from
+        // separate threads stream side by side
+        if (lane == 0) mbar_arrive_expect_tx(b_kfull(s), (uint32_t)nb * C::KV_BYTES);
+        __syncwarp();
+        if (lane < nb) {
+          const int czt = (GP == 2 && lane == 1) ? cz[GP - 1] : cz[0];
 #pragma unroll
-          for (int t = 0; t < GP; ++t)
-            if (t < nb)
-#pragma unroll
-              for (int kb = 0; kb < D / 64; ++kb)
-                tma_load_3d(sK + s * C::KG_BYTES + kb * (GP * P * 128) + t * (P * 128), &tm_k,
-                            b_kfull(s), kb * 64, 0, cz[t]);
+          for (int kb = 0; kb < D / 64; ++kb)
+            tma_load_3d(sK + s * C::KG_BYTES + kb * (GP * P * 128) + lane * (P * 128), &tm_k,
+                        b_kfull(s), kb * 64, 0, czt);
         }
         last = g;
         __syncwarp();
