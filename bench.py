@@ -37,7 +37,7 @@ WORKLOAD = "gqa-128k"
 # DRAM traffic (read + write) of one OSK launch at gqa-128k, from one ncu capture
 # (profiles/osk_attention_gqa-128k_traffic.md).  It describes the kernel source the
 # capture ran, identified by the hash below; any other source reports null.
-OSK_TRAFFIC = {"workload": "gqa-128k", "bytes": 2697283328, "source_sha256_16": "a2dc99f33d35e459"}
+OSK_TRAFFIC = {"workload": "gqa-128k", "bytes": 2695605504, "source_sha256_16": "37ec78a68845158c"}
 
 
 def _osk_traffic(workload: str):
