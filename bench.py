@@ -441,23 +441,20 @@ def main():
     }
     # ---- end to end through the C-ABI with host buffers (every rank, every N) ---
     def e2e_leg():
+        # through the library's host-buffer entry point: every step copies its inputs in
+        # from page-locked host memory and its output back, one KV head at a time, the
+        # copies overlapping the kernels
         qh = x["q"].cpu().pin_memory()
         kh = x["k_pool"].cpu().pin_memory()
         vh = x["v_pool"].cpu().pin_memory()
         pth = x["page_table"].cpu().pin_memory()
         outh = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-        qd, kd, vd, ptd = (torch.empty_like(x["q"]), torch.empty_like(x["k_pool"]),
-                           torch.empty_like(x["v_pool"]), torch.empty_like(x["page_table"]))
+        wsh = torch.empty(C.cosa_attention_host_workspace_size(shape, kap), dtype=torch.uint8,
+                          device=dev)
         e2e_steps = max(1, min(args.steps, 3))
 
         def e2e_step():
-            qd.copy_(qh, non_blocking=True)
-            kd.copy_(kh, non_blocking=True)
-            vd.copy_(vh, non_blocking=True)
-            ptd.copy_(pth, non_blocking=True)
-            C.cosa_kap_select(shape, kap, qd, kd, ptd, order, count, ws, stream=stream)
-            C.cosa_osk_attention(shape, osk, qd, kd, vd, ptd, order, count, out, stream=stream)
-            outh.copy_(out, non_blocking=True)
+            C.cosa_attention_host(shape, kap, osk, qh, kh, vh, pth, outh, wsh, stream=stream)
 
         e2e_step()
         torch.cuda.synchronize(dev)

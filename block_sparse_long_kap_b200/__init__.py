@@ -19,7 +19,8 @@ __all__ = [
     "cosa_status_string", "cosa_version", "cosa_kap_kcap", "cosa_kap_workspace_size",
     "cosa_kap_select", "cosa_kap_select_noalloc", "cosa_kap_order", "cosa_osk_attention",
     "cosa_dense_attention", "cosa_get_status", "EXPORTED_SYMBOLS", "NOALLOC_SCRATCH_BYTES",
-    "cosa_kap_select_group", "cosa_osk_attention_group",
+    "cosa_kap_select_group", "cosa_osk_attention_group", "cosa_attention_host_workspace_size",
+    "cosa_attention_host",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -29,6 +30,7 @@ EXPORTED_SYMBOLS = (
     "cosa_status_string", "cosa_version", "cosa_kap_kcap", "cosa_kap_workspace_size",
     "cosa_kap_select", "cosa_kap_select_noalloc", "cosa_kap_order", "cosa_osk_attention",
     "cosa_dense_attention", "cosa_get_status", "cosa_kap_select_group", "cosa_osk_attention_group",
+    "cosa_attention_host_workspace_size", "cosa_attention_host",
 )
 
 # Largest workspace the allocation-free Stage-1 entry point accepts (cosa.h).
@@ -146,6 +148,8 @@ def lib():
     L.cosa_osk_attention_group.argtypes = [P(_Shape), P(_Osk), vp, vp, vp, vp, vp, vp, i32, vp, vp,
                                            vp, vp, vp]
     L.cosa_get_status.argtypes = [vp]
+    L.cosa_attention_host_workspace_size.argtypes = [P(_Shape), P(_Kap), P(sz)]
+    L.cosa_attention_host.argtypes = [P(_Shape), P(_Kap), P(_Osk), vp, vp, vp, vp, vp, vp, sz, vp]
     for name in EXPORTED_SYMBOLS:
         if name not in ("cosa_status_string", "cosa_version"):
             getattr(L, name).restype = ctypes.c_int
@@ -375,6 +379,47 @@ def cosa_dense_attention(shape: Shape, q, k_pool, v_pool, page_table, out, lse=N
     _check(lib().cosa_dense_attention(ctypes.byref(s), _ptr(q), _ptr(k_pool), _ptr(v_pool),
                                       _ptr(page_table), _ptr(out), _ptr(lse), _stream(stream)),
            "cosa_dense_attention")
+
+
+def cosa_attention_host_workspace_size(shape: Shape, kap: KapParams) -> int:
+    out = ctypes.c_size_t(0)
+    s, k = shape.c(), kap.c(shape)
+    _check(lib().cosa_attention_host_workspace_size(ctypes.byref(s), ctypes.byref(k),
+                                                    ctypes.byref(out)),
+           "cosa_attention_host_workspace_size")
+    return out.value
+
+
+def _expect_host(t, name, dtype, shape):
+    if t is None:
+        raise ValueError(f"{name} is required")
+    if t.dtype != dtype:
+        raise TypeError(f"{name}: dtype {t.dtype}, expected {dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if t.is_cuda:
+        raise ValueError(f"{name} must be a host (CPU) tensor, page-locked for overlap")
+
+
+def cosa_attention_host(shape: Shape, kap: KapParams, osk: OskParams, q, k_pool, v_pool,
+                        page_table, out, workspace, stream=None) -> None:
+    """Both stages from host tensors, pipelined per KV head (copies overlap the kernels)."""
+    import torch
+    s, k, o = shape.c(), kap.c(shape), osk.c()
+    B, Hq, N, D = shape.batch, shape.num_q_heads, shape.seq_len, shape.head_dim
+    _expect_host(q, "q", torch.bfloat16, (B, Hq, N, D))
+    _expect_host(k_pool, "k_pool", torch.bfloat16, _kv_shape(shape))
+    _expect_host(v_pool, "v_pool", torch.bfloat16, _kv_shape(shape))
+    _expect_host(page_table, "page_table", torch.int32, (B, s.pages_per_seq))
+    _expect_host(out, "out", torch.bfloat16, (B, Hq, N, D))
+    if workspace is None or workspace.dtype != torch.uint8 or not workspace.is_cuda:
+        raise ValueError("workspace must be a CUDA uint8 tensor")
+    _check(lib().cosa_attention_host(ctypes.byref(s), ctypes.byref(k), ctypes.byref(o), _ptr(q),
+                                     _ptr(k_pool), _ptr(v_pool), _ptr(page_table), _ptr(out),
+                                     _ptr(workspace), workspace.numel(), _stream(stream)),
+           "cosa_attention_host")
 
 
 def cosa_get_status(stream=None) -> int:

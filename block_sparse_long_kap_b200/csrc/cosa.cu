@@ -374,6 +374,80 @@ cosa_status_t noalloc_scratch_address(void** out) {
   return COSA_OK;
 }
 
+// ---------------------------------------------------------------------------
+// cosa_attention_host: both stages from host buffers, one KV head at a time.
+// Heads are independent in both stages, so KV head c's copies in, its KAP + OSK
+// and the copy of its output back run on three streams: the copies of head c + 1
+// and the read-back of head c - 1 overlap head c's kernels.  The device copies of
+// one head's Q, K, V and output are doubled; the page table, the ordered lists and
+// the KAP workspace are single (the kernels use them in stream order).
+// ---------------------------------------------------------------------------
+size_t al256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+struct HostLayout {
+  cosa_shape_t sub;  // one KV head: H_q = G, H_kv = 1
+  int32_t k_cap;
+  size_t q, kv, ord, cnt, pt, kapws;       // bytes: one head's Q (or O), K (or V) pool, lists
+  size_t set_k, set_v, set_o, set_bytes;   // offsets inside one buffer set (Q at 0)
+  size_t off_set[2], off_ord, off_cnt, off_kapws, total;  // page table at 0
+};
+
+cosa_status_t host_layout(const cosa_shape_t* s, const cosa_kap_params_t* kap, HostLayout* L) {
+  cosa_status_t e = check_shape(s);
+  if (e != COSA_OK) return e;
+  if ((e = check_kap(s, kap)) != COSA_OK) return e;
+  L->sub = *s;
+  L->sub.num_q_heads = s->num_q_heads / s->num_kv_heads;
+  L->sub.num_kv_heads = 1;
+  const cosa_shape_t* u = &L->sub;
+  L->k_cap = kcap_of(u, kap);
+  const size_t nqb = static_cast<size_t>(u->seq_len / u->q_block);
+  const size_t bh = static_cast<size_t>(u->batch) * u->num_q_heads;
+  L->q = bh * u->seq_len * u->head_dim * 2;
+  L->kv = static_cast<size_t>(u->num_phys_pages) * u->page_size * u->head_dim * 2;
+  L->ord = bh * nqb * L->k_cap * 4;
+  L->cnt = bh * nqb * 4;
+  L->pt = static_cast<size_t>(s->batch) * s->pages_per_seq * 4;
+  L->kapws = kap_layout(u, kap).total;
+  L->set_k = al256(L->q);
+  L->set_v = L->set_k + al256(L->kv);
+  L->set_o = L->set_v + al256(L->kv);
+  L->set_bytes = L->set_o + al256(L->q);
+  L->off_set[0] = al256(L->pt);
+  L->off_set[1] = L->off_set[0] + L->set_bytes;
+  L->off_ord = L->off_set[1] + L->set_bytes;
+  L->off_cnt = L->off_ord + al256(L->ord);
+  L->off_kapws = L->off_cnt + al256(L->cnt);
+  L->total = L->off_kapws + al256(L->kapws);
+  return COSA_OK;
+}
+
+// Streams and events of one cosa_attention_host call, released on scope exit (CUDA
+// defers the release of a stream or event until the work queued on it is done).
+struct HostPipe {
+  cudaStream_t in = nullptr, out = nullptr;
+  cudaEvent_t start = nullptr, fin_in = nullptr, fin_out = nullptr;
+  cudaEvent_t loaded[2] = {}, used[2] = {}, drained[2] = {};
+  bool create() {
+    if (cudaStreamCreateWithFlags(&in, cudaStreamNonBlocking) != cudaSuccess ||
+        cudaStreamCreateWithFlags(&out, cudaStreamNonBlocking) != cudaSuccess)
+      return false;
+    cudaEvent_t* evs[] = {&start, &fin_in, &fin_out, &loaded[0], &loaded[1],
+                          &used[0], &used[1], &drained[0], &drained[1]};
+    for (cudaEvent_t* e : evs)
+      if (cudaEventCreateWithFlags(e, cudaEventDisableTiming) != cudaSuccess) return false;
+    return true;
+  }
+  ~HostPipe() {
+    cudaEvent_t evs[] = {start, fin_in, fin_out, loaded[0], loaded[1],
+                         used[0], used[1], drained[0], drained[1]};
+    for (cudaEvent_t e : evs)
+      if (e) cudaEventDestroy(e);
+    if (in) cudaStreamDestroy(in);
+    if (out) cudaStreamDestroy(out);
+  }
+};
+
 }  // namespace
 
 extern "C" {
@@ -594,6 +668,98 @@ cosa_status_t cosa_get_status(cosa_stream_t stream) {
       return COSA_ERR_CUDA;
   }
   return static_cast<cosa_status_t>(v);
+}
+
+cosa_status_t cosa_attention_host_workspace_size(const cosa_shape_t* shape,
+                                                 const cosa_kap_params_t* kap, size_t* bytes) {
+  if (!bytes) return COSA_ERR_INVALID_ARG;
+  HostLayout L;
+  const cosa_status_t e = host_layout(shape, kap, &L);
+  if (e != COSA_OK) return e;
+  *bytes = L.total;
+  return COSA_OK;
+}
+
+cosa_status_t cosa_attention_host(const cosa_shape_t* shape, const cosa_kap_params_t* kap,
+                                  const cosa_osk_params_t* osk, const void* q_host,
+                                  const void* k_pool_host, const void* v_pool_host,
+                                  const int32_t* page_table_host, void* out_host, void* workspace,
+                                  size_t workspace_bytes, cosa_stream_t stream) {
+  HostLayout L;
+  cosa_status_t e = host_layout(shape, kap, &L);
+  if (e != COSA_OK) return e;
+  if (!osk || !(osk->eps >= 0.f)) return COSA_ERR_INVALID_ARG;
+  if (!q_host || !k_pool_host || !v_pool_host || !page_table_host || !out_host)
+    return COSA_ERR_INVALID_ARG;
+  if (!workspace || workspace_bytes < L.total || reinterpret_cast<uintptr_t>(workspace) % 256)
+    return COSA_ERR_WORKSPACE;
+  const int B = shape->batch, Hq = shape->num_q_heads, Hkv = shape->num_kv_heads, G = Hq / Hkv;
+  const size_t head_bytes = static_cast<size_t>(shape->seq_len) * shape->head_dim * 2;  // one (b, h)
+  const size_t page_bytes = static_cast<size_t>(shape->page_size) * shape->head_dim * 2;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  int32_t* pt_d = reinterpret_cast<int32_t*>(ws);
+  int32_t* ord_d = reinterpret_cast<int32_t*>(ws + L.off_ord);
+  int32_t* cnt_d = reinterpret_cast<int32_t*>(ws + L.off_cnt);
+  void* kapws_d = ws + L.off_kapws;
+  const uint8_t* qh = static_cast<const uint8_t*>(q_host);
+  const uint8_t* kh = static_cast<const uint8_t*>(k_pool_host);
+  const uint8_t* vh = static_cast<const uint8_t*>(v_pool_host);
+  uint8_t* oh = static_cast<uint8_t*>(out_host);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  HostPipe pp;
+  if (!pp.create()) return COSA_ERR_CUDA;
+  // the workspace may still be in use by earlier work on the caller's stream
+  bool ok = cudaEventRecord(pp.start, st) == cudaSuccess &&
+            cudaStreamWaitEvent(pp.in, pp.start, 0) == cudaSuccess &&
+            cudaStreamWaitEvent(pp.out, pp.start, 0) == cudaSuccess &&
+            cudaMemcpyAsync(pt_d, page_table_host, L.pt, cudaMemcpyHostToDevice, pp.in) ==
+                cudaSuccess;
+  e = ok ? COSA_OK : COSA_ERR_CUDA;
+  for (int c = 0; e == COSA_OK && c < Hkv; ++c) {
+    const int x = c & 1;
+    uint8_t* set = ws + L.off_set[x];
+    uint8_t *q_d = set, *k_d = set + L.set_k, *v_d = set + L.set_v, *o_d = set + L.set_o;
+    // KV head c in: its G query heads of every sequence, its column of the page pools
+    // (one page-sized row per physical page), once the kernels of head c - 2 are done
+    // with this buffer set
+    ok = c < 2 || cudaStreamWaitEvent(pp.in, pp.used[x], 0) == cudaSuccess;
+    for (int b = 0; ok && b < B; ++b)
+      ok = cudaMemcpyAsync(q_d + static_cast<size_t>(b) * G * head_bytes,
+                           qh + (static_cast<size_t>(b) * Hq + static_cast<size_t>(c) * G) * head_bytes,
+                           G * head_bytes, cudaMemcpyHostToDevice, pp.in) == cudaSuccess;
+    ok = ok &&
+         cudaMemcpy2DAsync(k_d, page_bytes, kh + c * page_bytes, Hkv * page_bytes, page_bytes,
+                           shape->num_phys_pages, cudaMemcpyHostToDevice, pp.in) == cudaSuccess &&
+         cudaMemcpy2DAsync(v_d, page_bytes, vh + c * page_bytes, Hkv * page_bytes, page_bytes,
+                           shape->num_phys_pages, cudaMemcpyHostToDevice, pp.in) == cudaSuccess &&
+         cudaEventRecord(pp.loaded[x], pp.in) == cudaSuccess &&
+         // the kernels wait for the inputs and for the read-back of head c - 2's output
+         cudaStreamWaitEvent(st, pp.loaded[x], 0) == cudaSuccess &&
+         (c < 2 || cudaStreamWaitEvent(st, pp.drained[x], 0) == cudaSuccess);
+    if (!ok) { e = COSA_ERR_CUDA; break; }
+    e = cosa_kap_select(&L.sub, kap, q_d, k_d, pt_d, ord_d, cnt_d, nullptr, nullptr, kapws_d,
+                        L.kapws, stream);
+    if (e != COSA_OK) break;
+    e = cosa_osk_attention(&L.sub, osk, q_d, k_d, v_d, pt_d, ord_d, cnt_d, L.k_cap, o_d, nullptr,
+                           nullptr, nullptr, stream);
+    if (e != COSA_OK) break;
+    // head c's output back to its place in out_host
+    ok = cudaEventRecord(pp.used[x], st) == cudaSuccess &&
+         cudaStreamWaitEvent(pp.out, pp.used[x], 0) == cudaSuccess;
+    for (int b = 0; ok && b < B; ++b)
+      ok = cudaMemcpyAsync(oh + (static_cast<size_t>(b) * Hq + static_cast<size_t>(c) * G) * head_bytes,
+                           o_d + static_cast<size_t>(b) * G * head_bytes, G * head_bytes,
+                           cudaMemcpyDeviceToHost, pp.out) == cudaSuccess;
+    ok = ok && cudaEventRecord(pp.drained[x], pp.out) == cudaSuccess;
+    if (!ok) e = COSA_ERR_CUDA;
+  }
+  // the caller's stream holds until everything queued above (copies included) is done
+  const bool joined = cudaEventRecord(pp.fin_in, pp.in) == cudaSuccess &&
+                      cudaEventRecord(pp.fin_out, pp.out) == cudaSuccess &&
+                      cudaStreamWaitEvent(st, pp.fin_in, 0) == cudaSuccess &&
+                      cudaStreamWaitEvent(st, pp.fin_out, 0) == cudaSuccess;
+  if (e == COSA_OK && !joined) e = COSA_ERR_CUDA;
+  return e;
 }
 
 }  // extern "C"

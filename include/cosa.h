@@ -16,8 +16,11 @@
  *
  * Conventions for every entry point
  *   - All tensor arguments are DEVICE pointers on the current CUDA device,
- *     allocated and owned by the caller; the library allocates no device
- *     memory per call and keeps no pointer after the call is enqueued.
+ *     allocated and owned by the caller (except the *_host arguments of
+ *     cosa_attention_host, which are host memory); the library allocates no
+ *     device memory per call and keeps no pointer after the call is enqueued
+ *     (cosa_attention_host creates two streams and a few events per call and
+ *     hands them back to CUDA before returning).
  *   - Layouts are dense, row-major (last index fastest):
  *       q          bf16  [B][H_q][N][D]
  *       k_pool     bf16  [num_phys_pages][H_kv][P][D]   (one page of one KV head
@@ -222,6 +225,36 @@ cosa_status_t cosa_osk_attention_group(const cosa_shape_t* shape, const cosa_osk
 cosa_status_t cosa_dense_attention(const cosa_shape_t* shape, const void* q, const void* k_pool,
                                    const void* v_pool, const int32_t* page_table, void* out,
                                    float* lse, cosa_stream_t stream);
+
+/* Bytes of device workspace cosa_attention_host needs: the page table, two sets
+ * of one KV head's Q, K pool column, V pool column and output, one KV head's
+ * ordered lists and its cosa_kap_select workspace.  Host-only; no CUDA call. */
+cosa_status_t cosa_attention_host_workspace_size(const cosa_shape_t* shape,
+                                                 const cosa_kap_params_t* kap, size_t* bytes);
+
+/* Both stages end to end from host memory: for every KV head, copy its G query
+ * heads of Q (every sequence) and its column of the K and V page pools to the
+ * device, run cosa_kap_select and cosa_osk_attention on that head alone (shape
+ * with H_q = G, H_kv = 1: heads are independent in both stages, so the result
+ * equals the whole-layer calls), and copy its output back to its place in
+ * out_host.  The copies of the next KV head and the read-back of the previous
+ * one run on two streams of the call's own, overlapping the kernels, which run
+ * on `stream`; `stream` waits for all of it, so synchronising `stream` means the
+ * output is in out_host.  q_host bf16 [B][H_q][N][D], k_pool_host / v_pool_host
+ * bf16 [num_phys_pages][H_kv][P][D], page_table_host int32 [B][pages_per_seq]
+ * and out_host bf16 [B][H_q][N][D] are host memory; page-locked memory lets the
+ * copies overlap the kernels (pageable memory works but the copies serialise).
+ * The host buffers must stay valid and unmodified until `stream` reaches the end
+ * of this call's work.  workspace: device buffer of at least
+ * cosa_attention_host_workspace_size bytes, 256-byte aligned.  Argument errors
+ * return before anything is queued; a failed CUDA call returns COSA_ERR_CUDA
+ * with the work queued so far still joined to `stream`; in-kernel errors go to
+ * the status word as for the stage calls. */
+cosa_status_t cosa_attention_host(const cosa_shape_t* shape, const cosa_kap_params_t* kap,
+                                  const cosa_osk_params_t* osk, const void* q_host,
+                                  const void* k_pool_host, const void* v_pool_host,
+                                  const int32_t* page_table_host, void* out_host, void* workspace,
+                                  size_t workspace_bytes, cosa_stream_t stream);
 
 /* Read (and clear) the current device's status word: COSA_OK, or the first
  * in-kernel error recorded since the last call (e.g. COSA_ERR_TIMEOUT).

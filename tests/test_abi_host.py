@@ -141,3 +141,38 @@ def test_group_entry_points_reject_bad_arguments_before_launch():
     ka = C.KapParams(ascending=True).c(shp)
     assert lib.cosa_kap_select_group(ctypes.byref(s), ctypes.byref(ka), 16, 16, 16, 16, 16, None,
                                      None, 256, 1 << 40, None) == 2
+
+
+def test_host_pipeline_workspace_and_argument_checks():
+    """cosa_attention_host: the workspace holds two sets of one KV head's inputs and
+    output plus that head's lists and KAP workspace; bad arguments return before
+    anything is queued (no CUDA call is made on these paths)."""
+    lib = C.lib()
+    shp = C.Shape(2, 8, 2, 2048, 128, 64, 128)
+    kap = C.KapParams(budget=0.25, q_sub=32, k_sub=16)
+    ws = C.cosa_attention_host_workspace_size(shp, kap)
+    sub = C.Shape(2, 4, 1, 2048, 128, 64, 128)
+    q_head = 2 * 4 * 2048 * 128 * 2
+    kv_head = shp.c().num_phys_pages * 64 * 128 * 2
+    assert ws >= 2 * (2 * q_head + 2 * kv_head) + C.cosa_kap_workspace_size(sub, kap)
+    s, k, o = shp.c(), kap.c(shp), C._Osk(1e-4)
+    # null host buffer, negative eps, missing / small / misaligned workspace
+    assert lib.cosa_attention_host(ctypes.byref(s), ctypes.byref(k), ctypes.byref(o), None, 16, 16,
+                                   16, 16, 256, ws, None) == 1
+    ob = C._Osk(-1.0)
+    assert lib.cosa_attention_host(ctypes.byref(s), ctypes.byref(k), ctypes.byref(ob), 16, 16, 16,
+                                   16, 16, 256, ws, None) == 1
+    assert lib.cosa_attention_host(ctypes.byref(s), ctypes.byref(k), ctypes.byref(o), 16, 16, 16,
+                                   16, 16, None, 0, None) == 5
+    assert lib.cosa_attention_host(ctypes.byref(s), ctypes.byref(k), ctypes.byref(o), 16, 16, 16,
+                                   16, 16, 256, ws - 1, None) == 5
+    assert lib.cosa_attention_host(ctypes.byref(s), ctypes.byref(k), ctypes.byref(o), 16, 16, 16,
+                                   16, 16, 128, ws, None) == 5
+    # invalid shape (H_q not a multiple of H_kv) and null size pointer
+    bad = C.Shape(1, 6, 4, 1024, 128, 64, 128).c()
+    assert lib.cosa_attention_host_workspace_size(ctypes.byref(bad), ctypes.byref(k),
+                                                  ctypes.byref(ctypes.c_size_t(0))) == 1
+    assert lib.cosa_attention_host_workspace_size(ctypes.byref(s), ctypes.byref(k), None) == 1
+    # the binding refuses device-resident host arguments before calling in
+    with pytest.raises((TypeError, ValueError)):
+        C.cosa_attention_host(shp, kap, C.OskParams(1e-4), None, None, None, None, None, None)
