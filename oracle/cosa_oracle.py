@@ -41,7 +41,7 @@ __all__ = [
     "causal_pages", "forced_pages", "budget_count", "k_cap",
     "gather_logical", "kap_pool_queries", "kap_pool_keys", "kap_block_scores",
     "kap_maxnorm_hrm", "rank_key", "kap_order_from_scores", "kap_select_block",
-    "kap_select", "kap_order", "osk_block", "osk_attention", "dense_rows",
+    "kap_select", "kap_order", "osk_block", "osk_block_rules", "osk_attention", "dense_rows",
     "dense_attention", "kap_group_scores", "kap_select_group", "expand_group_order",
 ]
 
@@ -363,10 +363,13 @@ def expand_group_order(order_g: np.ndarray, count_g: np.ndarray, num_q_heads: in
 # ----------------------------------------------------------------------------
 # Stage 2: Ordered-Skipping Kernel  ([TS §2.1], [TS §2.3])
 # ----------------------------------------------------------------------------
-def osk_block(q_rows: np.ndarray, k_log: np.ndarray, v_log: np.ndarray, qb: int,
-              q_block: int, page_size: int, order: Sequence[int], eps: float,
-              scale: float, force: Optional[dict] = None):
-    """Ordered-skipping online-softmax attention for one q-block.
+def osk_block_rules(q_rows: np.ndarray, k_log: np.ndarray, v_log: np.ndarray, qb: int,
+                    q_block: int, page_size: int, order: Sequence[int], eps: float,
+                    scale: float, force: Optional[dict] = None, rule: str = "max",
+                    max_run: Optional[int] = None) -> dict:
+    """Ordered-skipping online-softmax attention for one q-block, under the
+    pages' skip rule (rule="max") or one of two variants the pages do not give
+    (rule="sum", max_run): see the end of this docstring.
 
     Pages are visited in the order given ([ABS] "the order in which KV pages
     are visited in the kernel inner loop"); online-softmax accumulation is
@@ -389,8 +392,18 @@ def osk_block(q_rows: np.ndarray, k_log: np.ndarray, v_log: np.ndarray, qb: int,
     force: optional {step j: bool skipped} overriding the rule at listed steps
     (used by tests to evaluate the alternative at steps whose decision lies
     within rounding of the threshold).
-    Returns (out [Bq][D], lse [Bq], computed int, skip_log uint8 [len(order)],
-    margin float64 [len(order)] = max_i d_i - ln(eps))."""
+
+    Variants (not on the pages; stated here as they are computed):
+      rule="sum": a row's test also weighs the page against the mass the row
+        already holds: the page is skipped iff max_i (d_i + ln P - ln l_i) <
+        ln(eps), l_i the running sum relative to the running max m_i.  Each of
+        the page's at most P visible keys has weight <= e^{d_i} relative to m_i,
+        so a skipped page would have added less than eps * l_i to row i's sum.
+      max_run=r: after r consecutive skipped pages the rest of the list is
+        skipped without being visited (no QK^T, no K load).
+    Returns dict: out [Bq][D], lse [Bq], computed (pages with P V), visited
+    (pages whose QK^T was evaluated), skip uint8 [len(order)], margin float64
+    [len(order)] = the tested maximum minus ln(eps) (NaN past a break)."""
     Bq, D = q_rows.shape
     rows = qb * q_block + np.arange(Bq)
     qf = np.asarray(q_rows, dtype=np.float64)
@@ -402,7 +415,13 @@ def osk_block(q_rows: np.ndarray, k_log: np.ndarray, v_log: np.ndarray, qb: int,
     skip_log = np.zeros(n, dtype=np.uint8)
     margin = np.full(n, np.nan)
     computed = 0
+    visited = 0
+    run = 0
     for j, p in enumerate(order):
+        if max_run is not None and run >= max_run:
+            skip_log[j:] = 1
+            break
+        visited += 1
         keys = int(p) * page_size + np.arange(page_size)
         s = (qf @ k_log[keys].T) * scale
         s = np.where(keys[None, :] > rows[:, None], NEG_INF, s)
@@ -413,6 +432,10 @@ def osk_block(q_rows: np.ndarray, k_log: np.ndarray, v_log: np.ndarray, qb: int,
         d[first_seen] = math.inf
         both = live & (m > NEG_INF)
         d[both] = m_loc[both] - m[both]
+        if rule == "sum":
+            d[both] += math.log(page_size) - np.log(l[both])
+        elif rule != "max":
+            raise ValueError(f"unknown skip rule {rule!r}")
         dmax = d.max() if live.any() else NEG_INF
         if log_eps == NEG_INF or log_eps == math.inf:
             margin[j] = math.inf if log_eps == NEG_INF else NEG_INF
@@ -423,7 +446,9 @@ def osk_block(q_rows: np.ndarray, k_log: np.ndarray, v_log: np.ndarray, qb: int,
             skip = bool(force[j])
         skip_log[j] = 1 if skip else 0
         if skip:
+            run += 1
             continue
+        run = 0
         computed += 1
         m_new = np.maximum(m, m_loc)
         upd = m_new > NEG_INF
@@ -439,17 +464,31 @@ def osk_block(q_rows: np.ndarray, k_log: np.ndarray, v_log: np.ndarray, qb: int,
     seen = l > 0
     out[seen] = o[seen] / l[seen, None]
     lse[seen] = m[seen] + np.log(l[seen])
-    return out, lse, computed, skip_log, margin
+    return {"out": out, "lse": lse, "computed": computed, "visited": visited,
+            "skip": skip_log, "margin": margin}
+
+
+def osk_block(q_rows: np.ndarray, k_log: np.ndarray, v_log: np.ndarray, qb: int,
+              q_block: int, page_size: int, order: Sequence[int], eps: float,
+              scale: float, force: Optional[dict] = None):
+    """The pages' rule for one q-block (osk_block_rules with rule="max", no
+    break).  Returns (out [Bq][D], lse [Bq], computed int, skip_log uint8
+    [len(order)], margin float64 [len(order)] = max_i d_i - ln(eps))."""
+    r = osk_block_rules(q_rows, k_log, v_log, qb, q_block, page_size, order, eps, scale,
+                        force=force)
+    return r["out"], r["lse"], r["computed"], r["skip"], r["margin"]
 
 
 def osk_attention(q: np.ndarray, k_pool: np.ndarray, v_pool: np.ndarray,
                   page_table: np.ndarray, order: np.ndarray, count: np.ndarray, *,
                   num_kv_heads: int, page_size: int, q_block: int, eps: float,
                   scale: float, heads: Optional[Sequence] = None,
-                  qblocks: Optional[Sequence[int]] = None):
+                  qblocks: Optional[Sequence[int]] = None, rule: str = "max",
+                  max_run: Optional[int] = None):
     """OSK over a whole problem (or a subset).  order [B][H_q][nQB][k_cap],
-    count [B][H_q][nQB].  Returns dict with out float64 [B][H_q][N][D],
-    lse [B][H_q][N], computed int32 [B][H_q][nQB], skip uint8
+    count [B][H_q][nQB]; rule / max_run select a skip-rule variant
+    (osk_block_rules).  Returns dict with out float64 [B][H_q][N][D],
+    lse [B][H_q][N], computed and visited int32 [B][H_q][nQB], skip uint8
     [B][H_q][nQB][k_cap], margin float64 [B][H_q][nQB][k_cap]."""
     B, Hq, N, D = q.shape
     G = Hq // num_kv_heads
@@ -458,6 +497,7 @@ def osk_attention(q: np.ndarray, k_pool: np.ndarray, v_pool: np.ndarray,
     out = np.zeros((B, Hq, N, D))
     lse = np.full((B, Hq, N), NEG_INF)
     computed = np.zeros((B, Hq, nQB), dtype=np.int32)
+    visited = np.zeros((B, Hq, nQB), dtype=np.int32)
     skip = np.zeros((B, Hq, nQB, kc), dtype=np.uint8)
     margin = np.full((B, Hq, nQB, kc), np.nan)
     if heads is None:
@@ -474,14 +514,16 @@ def osk_attention(q: np.ndarray, k_pool: np.ndarray, v_pool: np.ndarray,
         for qb in qblocks:
             rows = slice(qb * q_block, (qb + 1) * q_block)
             c = int(count[b, h, qb])
-            o, ls, comp, sk, mg = osk_block(q[b, h, rows], k_log, v_log, qb, q_block,
-                                            page_size, order[b, h, qb, :c], eps, scale)
-            out[b, h, rows] = o
-            lse[b, h, rows] = ls
-            computed[b, h, qb] = comp
-            skip[b, h, qb, :c] = sk
-            margin[b, h, qb, :c] = mg
-    return {"out": out, "lse": lse, "computed": computed, "skip": skip, "margin": margin}
+            r = osk_block_rules(q[b, h, rows], k_log, v_log, qb, q_block, page_size,
+                                order[b, h, qb, :c], eps, scale, rule=rule, max_run=max_run)
+            out[b, h, rows] = r["out"]
+            lse[b, h, rows] = r["lse"]
+            computed[b, h, qb] = r["computed"]
+            visited[b, h, qb] = r["visited"]
+            skip[b, h, qb, :c] = r["skip"]
+            margin[b, h, qb, :c] = r["margin"]
+    return {"out": out, "lse": lse, "computed": computed, "visited": visited, "skip": skip,
+            "margin": margin}
 
 
 # ----------------------------------------------------------------------------

@@ -519,3 +519,89 @@ def test_expand_group_order_maps_heads_to_their_kv_head():
     o, c = O.expand_group_order(og, cg, 6)
     for h in range(6):
         assert np.array_equal(o[:, h], og[:, h // 2]) and np.array_equal(c[:, h], cg[:, h // 2])
+
+
+# ---------------------------------------------------------------------------
+# skip-rule variants (not on the pages): the sum-aware test and the early break
+# ---------------------------------------------------------------------------
+def test_sum_rule_skipped_pages_hold_less_than_eps_of_the_row_mass():
+    """Under rule="sum" a skipped page would have added less than eps times the
+    row's mass so far.  Recompute that mass from the full logit matrix over the
+    pages computed before the skip (not online), and the page's own mass."""
+    q, k, v = _tiny_problem(seed=12, drift=0.3)
+    N, P, Bq, scale = 256, 16, 16, 1 / math.sqrt(8)
+    L = (q @ k.T) * scale
+    L[np.triu(np.ones((N, N), dtype=bool), 1)] = -np.inf
+    rng = np.random.default_rng(13)
+    n_skips = 0
+    for eps in [0.3, 1e-1, 1e-2]:
+        for qb in range(N // Bq):
+            n_b = O.causal_pages(qb, Bq, P)
+            order = rng.permutation(n_b)
+            rows = np.arange(qb * Bq, (qb + 1) * Bq)
+            r = O.osk_block_rules(q[rows], k, v, qb, Bq, P, order, eps, scale, rule="sum")
+            sk = r["skip"]
+            assert sk[0] == 0 and r["computed"] == len(order) - sk.sum()
+            for j in np.nonzero(sk)[0]:
+                done = [order[t] for t in range(j) if sk[t] == 0]
+                cols = np.concatenate([np.arange(pp * P, (pp + 1) * P) for pp in done])
+                M = L[rows][:, cols].max(axis=1)
+                page = L[rows][:, order[j] * P:(order[j] + 1) * P]
+                sees = (page > -np.inf).any(axis=1)
+                assert np.all(M[sees] > -np.inf)          # no row meets its first key here
+                S = np.exp(L[rows][:, cols] - M[:, None]).sum(axis=1)
+                Wp = np.exp(page - M[:, None]).sum(axis=1)
+                assert np.all(Wp[sees] < eps * S[sees] * (1 + 1e-12))
+            n_skips += int(sk.sum())
+    assert n_skips > 0
+
+
+def test_sum_rule_extremes_match_the_pages_rule():
+    """eps = 0 skips nothing and eps = inf keeps only the first page and pages
+    where some row meets its first key, under both rules."""
+    q, k, v = _tiny_problem(seed=14, drift=0.2)
+    N, P, Bq, scale = 256, 16, 16, 1 / math.sqrt(8)
+    rng = np.random.default_rng(15)
+    for qb in range(N // Bq):
+        rows = np.arange(qb * Bq, (qb + 1) * Bq)
+        order = rng.permutation(O.causal_pages(qb, Bq, P))
+        for eps in (0.0, math.inf):
+            a = O.osk_block_rules(q[rows], k, v, qb, Bq, P, order, eps, scale, rule="sum")
+            b = O.osk_block_rules(q[rows], k, v, qb, Bq, P, order, eps, scale, rule="max")
+            assert np.array_equal(a["skip"], b["skip"])
+            np.testing.assert_array_equal(a["out"], b["out"])
+    with pytest.raises(ValueError):
+        O.osk_block_rules(q[:Bq], k, v, 0, Bq, P, [0], 1e-3, scale, rule="mean")
+
+
+def test_early_break_is_the_pages_rule_cut_after_r_skips():
+    """A skipped page changes no state, so with max_run = r the decisions equal
+    the pages' rule up to its first run of r consecutive skips and every later
+    page is skipped unvisited; the output equals the pages' rule with those
+    later pages forced skipped (osk_block's force path)."""
+    q, k, v = _tiny_problem(seed=16, drift=0.3)
+    N, P, Bq, scale = 256, 16, 16, 1 / math.sqrt(8)
+    rng = np.random.default_rng(17)
+    cuts = 0
+    for eps in [1e-1, 1e-2]:
+        for qb in range(N // Bq):
+            rows = np.arange(qb * Bq, (qb + 1) * Bq)
+            order = rng.permutation(O.causal_pages(qb, Bq, P))
+            base = O.osk_block_rules(q[rows], k, v, qb, Bq, P, order, eps, scale)
+            for r in (1, 2, 3):
+                got = O.osk_block_rules(q[rows], k, v, qb, Bq, P, order, eps, scale, max_run=r)
+                sk = base["skip"]
+                t = next((i for i in range(r - 1, len(order)) if sk[i - r + 1:i + 1].all()),
+                         None)
+                want = sk.copy()
+                if t is not None:
+                    want[t + 1:] = 1
+                    cuts += int(t + 1 < len(order))
+                assert np.array_equal(got["skip"], want)
+                assert got["visited"] == (len(order) if t is None else min(t + 1, len(order)))
+                forced = {j: True for j in range(t + 1, len(order))} if t is not None else None
+                out, lse, comp, _, _ = O.osk_block(q[rows], k, v, qb, Bq, P, order, eps, scale,
+                                                   force=forced)
+                np.testing.assert_array_equal(got["out"], out)
+                assert got["computed"] == comp
+    assert cuts > 0
