@@ -572,6 +572,45 @@ def main():
         "kap_kept_frac": vis_g / n_b_total, "osk_computed_frac": comp_g / n_b_total,
         "rel_l2_vs_dense": rel_l2(outg), "per_head_rel_l2_vs_dense": rel_l2(out)}
 
+    # ---- early break (max_run: not part of the pages' method): OSK only, the lists
+    # reused; output against the pages' rule at this eps (in `out`) and against dense
+    def early_break_leg():
+        bout = torch.empty_like(out)
+        bcomp = torch.empty_like(computed)
+        pref = out.float()
+        k_ms = statistics.mean(kap_ms)
+        res = []
+        for r in (16, 8):
+            o3 = C.OskParams(eps=args.eps, max_run=r)
+
+            def run():
+                C.cosa_osk_attention(shape, o3, x["q"], x["k_pool"], x["v_pool"], x["page_table"],
+                                     order, count, bout, computed=bcomp, stream=stream)
+
+            run()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(3):
+                run()
+            e1.record(stream)
+            torch.cuda.synchronize(dev)
+            if C.cosa_get_status(stream) != 0:
+                raise RuntimeError("in-kernel error status")
+            ms = e0.elapsed_time(e1) / 3
+            comp = int(bcomp.to(torch.int64).sum().item())
+            res.append({"max_run": r, "eps": args.eps, "osk_ms": ms, "kap_plus_osk_ms": ms + k_ms,
+                        "tflops": dense_flop / ((ms + k_ms) * 1e-3) / 1e12,
+                        "speedup_vs_dense": dense_ms / (ms + k_ms),
+                        "computed_frac": comp / n_b_total,
+                        "rel_l2_vs_pages_rule": float((bout.float() - pref).norm() / pref.norm()),
+                        "rel_l2_vs_dense": rel_l2(bout)})
+        return res
+
+    try:
+        line["early_break"] = early_break_leg()
+    except Exception as exc:  # an extra leg: report the failure, keep the line
+        line["early_break"] = {"error": repr(exc)}
+
     line["e2e"] = e2e_leg()
 
     # ---- CPU oracle on a bounded sample of the same workload ----------------

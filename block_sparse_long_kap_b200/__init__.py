@@ -65,7 +65,7 @@ class _Kap(ctypes.Structure):
 
 
 class _Osk(ctypes.Structure):
-    _fields_ = [("eps", ctypes.c_float)]
+    _fields_ = [("eps", ctypes.c_float), ("max_run", ctypes.c_int32)]
 
 
 @dataclasses.dataclass
@@ -113,9 +113,10 @@ class KapParams:
 @dataclasses.dataclass
 class OskParams:
     eps: float = 1e-4
+    max_run: int = 0        # > 0: early break after this many consecutive skipped pages
 
     def c(self) -> _Osk:
-        return _Osk(self.eps)
+        return _Osk(self.eps, self.max_run)
 
 
 _lib = None

@@ -74,6 +74,7 @@ struct TcParams {
   uint8_t* skip_log;
   int num_q_heads, num_kv_heads, group, seq_len, num_q_blocks, pages_per_seq, k_cap, q_block;
   float scale_log2, log2_eps;
+  int max_run;  // OSK early break after this many consecutive skipped pages; 0: none
   unsigned long long timeout_ns;
 };
 
@@ -107,11 +108,13 @@ struct TcCfg {
   static constexpr uint32_t OFF_MISC = (OFF_BAR + NBAR * 8 + 127) & ~127u;  // vector-aligned
   // misc: +0 TMEM address, +4 abort flag, +8 kept count (P location published),
   //       +12 final kept count (-1 while the votes run), +16 V progress,
-  //       +20 warpgroups finished, +36 PV progress, +40 kept count (TMA coordinate
+  //       +20 warpgroups finished, +24 first group past an early break, +28 list
+  //       position of the last kept page, +36 PV progress, +40 kept count (TMA coordinate
   //       published), +48 votes [2 wg][2][4], +128 kept queue [KQ] {TMA coordinate,
   //       P column | last << 15}, +640 settled state rows [128] {m_run, m_ref},
   //       +1664 last settled group per softmax warp [8], +1696 S-ready flag per
-  //       warpgroup [2], +2688 final rows [2][128] {l, m_ref}
+  //       warpgroup [2], +1704 last group loaded per K producer warp [2],
+  //       +2688 final rows [2][128] {l, m_ref}
   static constexpr uint32_t M_STATE = 640, M_SETTLED = 1664, M_FIN = 2688;
   static constexpr uint32_t MISC_BYTES = M_FIN + 2 * 128 * 8;
   static constexpr uint32_t SMEM = OFF_MISC + MISC_BYTES;
@@ -124,7 +127,7 @@ struct TcCfg {
   static_assert(OFF_MISC % 128 == 0, "16-byte vector access to the vote words");
   static_assert(KV_BYTES % 1024 == 0, "tiles stay 1024-byte aligned for the 128-byte swizzle");
   static_assert(48 + 64 <= 128 && 128 + 8 * KQ <= M_STATE, "vote words and kept queue fit");
-  static_assert(M_STATE + 128 * 8 <= M_SETTLED && M_SETTLED + 8 * 4 + 2 * 4 <= M_FIN,
+  static_assert(M_STATE + 128 * 8 <= M_SETTLED && M_SETTLED + 8 * 4 + 4 * 4 <= M_FIN,
                 "state rows and flags fit");
 };
 
@@ -169,11 +172,17 @@ __global__ void __launch_bounds__(TcCfg<D, P>::NT, 1)
   volatile int* kq_final = reinterpret_cast<volatile int*>(misc + 12);
   volatile int* v_pos = reinterpret_cast<volatile int*>(misc + 16);
   int* wg_done = reinterpret_cast<int*>(misc + 20);
+  // early break (max_run > 0): groups >= *stop_g lie past it; *kept_last is the list
+  // position of the last kept page, written in list order by the exact path
+  volatile int* stop_g = reinterpret_cast<volatile int*>(misc + 24);
+  volatile int* kept_last = reinterpret_cast<volatile int*>(misc + 28);
   volatile int* pv_pos = reinterpret_cast<volatile int*>(misc + 36);
   volatile int* vq_count = reinterpret_cast<volatile int*>(misc + 40);
   volatile int* votes = reinterpret_cast<volatile int*>(misc + 48);     // [2][2][4]
   volatile int* settled = reinterpret_cast<volatile int*>(misc + C::M_SETTLED);  // [8]
   volatile int* s_ok = reinterpret_cast<volatile int*>(misc + C::M_SETTLED + 32);  // [2]
+  // last group each K producer warp loaded (for the drain after an early break)
+  volatile int* k_last = reinterpret_cast<volatile int*>(misc + C::M_SETTLED + 40);  // [2]
   volatile int2* kq = reinterpret_cast<volatile int2*>(misc + 128);     // [KQ]
   volatile float2* st_rows = reinterpret_cast<volatile float2*>(misc + C::M_STATE);  // [128]
   volatile float2* fin_rows = reinterpret_cast<volatile float2*>(misc + C::M_FIN);    // [2][128]
@@ -231,6 +240,10 @@ __global__ void __launch_bounds__(TcCfg<D, P>::NT, 1)
     *pv_pos = 0;
     *vq_count = 0;
     *wg_done = 0;
+    *stop_g = n_groups;
+    *kept_last = -1;
+    k_last[0] = -1;
+    k_last[1] = -1;
     for (int w = 0; w < 8; ++w) settled[w] = -1;
     for (int r = 0; r < 128; ++r) {
       st_rows[r].x = -INFINITY;
@@ -256,6 +269,7 @@ __global__ void __launch_bounds__(TcCfg<D, P>::NT, 1)
   const uint32_t tmem = *tmem_slot;
 
   const unsigned long long tmo = prm.timeout_ns;
+  const int R = prm.max_run;  // early break after R consecutive skipped pages (0: none)
   auto give_up = [&]() {
     *abort_flag = 1;
     set_status(COSA_ERR_TIMEOUT);
@@ -275,6 +289,21 @@ __global__ void __launch_bounds__(TcCfg<D, P>::NT, 1)
       }
     }
     return true;
+  };
+  // the same for work of group g: 1 done, 0 timeout or abort, 2 group g now lies past an
+  // early break (the phase may never complete: nothing past the break is loaded or issued)
+  auto wait_g = [&](uint32_t bar_addr, uint32_t parity, int g) -> int {
+    if (mbar_try_wait(bar_addr, parity)) return 1;
+    const uint64_t t0 = globaltimer_ns();
+    while (!mbar_try_wait(bar_addr, parity)) {
+      if (g >= *stop_g) return 2;
+      if (*abort_flag) return 0;
+      if (timed_out(t0)) {
+        give_up();
+        return 0;
+      }
+    }
+    return 1;
   };
   // the same, waited on by lane 0 for the whole warp
   auto wait_warp = [&](uint32_t bar_addr, uint32_t parity) -> bool {
@@ -338,10 +367,20 @@ __global__ void __launch_bounds__(TcCfg<D, P>::NT, 1)
       for (int mm = 0; mm < GB; ++mm) {
         const int g = kp + C::NPROD * (i0 + mm);
         if (g >= n_groups) break;
+        // nothing past an early break is loaded (one read for the warp; none without a
+        // break, where the stop never moves)
+        if (R > 0 && __shfl_sync(0xffffffffu, lane == 0 ? *stop_g : 0, 0) <= g) {
+          ok = false;
+          break;
+        }
         const int s = g % C::KG;
         if (g >= C::KG) {
-          ok = wait_warp(b_kempty(s), ((g / C::KG) - 1) & 1);
-          if (!ok) break;
+          int r = 1;
+          if (lane == 0) r = wait_g(b_kempty(s), ((g / C::KG) - 1) & 1, g);
+          if (__shfl_sync(0xffffffffu, r, 0) != 1) {
+            ok = false;
+            break;
+          }
         }
         const int nb = min(GP, n_list - g * GP);
         int cz[GP];
@@ -362,6 +401,7 @@ __global__ void __launch_bounds__(TcCfg<D, P>::NT, 1)
         __syncwarp();
       }
     }
+    if (lane == 0) k_last[kp] = last;
     if (lane == 0 && *abort_flag) {  // drain what was issued and never consumed
       const uint64_t t0 = globaltimer_ns();
       if (kp == 0)
@@ -459,10 +499,11 @@ __global__ void __launch_bounds__(TcCfg<D, P>::NT, 1)
       auto sfree_phase = [](int g) { return ((g - C::SBG) / (2 * C::SBG)) & 1; };
       bool next_ready = false;
       for (int g = par; ok && g < n_groups; g += step) {
+        if (R > 0 && g >= *stop_g) break;  // past an early break: not issued
         const int ks = g % C::KG, sbuf = g % C::SBG;
         if (!next_ready) {
-          if (!wait(b_kfull(ks), (g / C::KG) & 1)) break;
-          if (g >= C::SBG && !wait(b_sfree(sbuf, g & 1), sfree_phase(g))) break;
+          if (wait_g(b_kfull(ks), (g / C::KG) & 1, g) != 1) break;
+          if (g >= C::SBG && wait_g(b_sfree(sbuf, g & 1), sfree_phase(g), g) != 1) break;
         }
         tc_fence_after();
         const uint32_t id = (g * GP + GP <= n_list) ? ID_FULL : ID_PAGE;
@@ -627,7 +668,9 @@ __global__ void __launch_bounds__(TcCfg<D, P>::NT, 1)
     };
     // wait (lane 0 of each warp) until every warp of the other warpgroup has settled
     // group g (all groups before the next one of this warpgroup are then settled)
-    auto wait_settled = [&](int g) -> bool {
+    // (1 done, 0 timeout or abort, 2 group g + 1 lies past an early break: group g may
+    // never be settled, and g + 1 needs no state, all its pages being skipped)
+    auto wait_settled = [&](int g) -> int {
       int okl = 1;
       if (lane == 0) {
         volatile int* o = settled + (wg ^ 1) * 4;
@@ -636,6 +679,7 @@ __global__ void __launch_bounds__(TcCfg<D, P>::NT, 1)
           const uint64_t t0 = globaltimer_ns();
           uint32_t spins = 0, nap = 32;
           while (!done()) {
+            if (g + 1 >= *stop_g) { okl = 2; break; }
             if (*abort_flag) { okl = 0; break; }
             if ((++spins & 15u) == 0 && timed_out(t0)) { give_up(); okl = 0; break; }
             __nanosleep(nap);
@@ -643,7 +687,7 @@ __global__ void __launch_bounds__(TcCfg<D, P>::NT, 1)
           }
         }
       }
-      return __shfl_sync(0xffffffffu, okl, 0) != 0;
+      return __shfl_sync(0xffffffffu, okl, 0);
     };
     // this warp has settled group g (its state rows and queue entries are written)
     auto mark_settled = [&](int g) {
@@ -671,9 +715,14 @@ __global__ void __launch_bounds__(TcCfg<D, P>::NT, 1)
       // ---- row maxima of the group's pages, read from TMEM.  One lane waits for S and
       // the named barrier brings the four warps along together (apart, each warp
       // waking on its own, the vote barrier waited for the last of them).
-      if (leader) s_ok[wg] = wait(b_sfull(sb, wg), (g / (2 * C::SBG)) & 1) ? 1 : 0;
+      // A group past an early break is not waited for (it may never be issued): the
+      // warpgroup stops there.
+      if (leader)
+        s_ok[wg] = (R > 0 && g >= *stop_g) ? 2 : wait_g(b_sfull(sb, wg), (g / (2 * C::SBG)) & 1, g);
       named_bar_sync(1 + wg, 128);
-      const bool okw = !fail && s_ok[wg] != 0;
+      const int s_res = s_ok[wg];
+      if (s_res == 2) break;
+      const bool okw = !fail && s_res != 0;
       if (okw) tc_fence_after();
       // (one copy of the per-page code: the loop is not unrolled)
       float ml0 = -INFINITY, ml1 = -INFINITY;
@@ -721,13 +770,24 @@ __global__ void __launch_bounds__(TcCfg<D, P>::NT, 1)
             if (slog)
               for (int t = 0; t < nb; ++t) slog[j + t] = 1;
             mbar_arrive(b_sfree(sb, wg ^ 1));
+            // early break: once every group before this one is settled, the last kept
+            // page is known; if the skipped run reaches R by the next group's first
+            // page, every later group lies past the break
+            if (R > 0) {
+              volatile int* o = settled + (wg ^ 1) * 4;
+              if (min(min(o[0], o[1]), min(o[2], o[3])) >= g - 1) {
+                __threadfence_block();
+                if ((g + 1) * GP - *kept_last - 1 >= R) atomicMin(const_cast<int*>(stop_g), g + 1);
+              }
+            }
           }
           mark_settled(g);
           continue;
         }
       }
       // ---- exact path: the groups before this one are settled; take their state
-      bool oks = okw && (g == 0 || wait_settled(g - 1));
+      const int wsr = !okw ? 0 : (g == 0 ? 1 : wait_settled(g - 1));
+      const bool oks = wsr == 1;
       if (oks) {
         __threadfence_block();
         const float sr = st_rows[row].x, sf = st_rows[row].y;
@@ -740,13 +800,22 @@ __global__ void __launch_bounds__(TcCfg<D, P>::NT, 1)
       // kept pages before this group: every earlier queue entry is published, and
       // the count is read before the vote barrier, ahead of this group's publishing
       const int c0 = *kq_count;
+      // early break: list position of the last kept page before this group; a page with
+      // R skipped pages right before it, and every page after it, is skipped unvisited
+      const int kl = (R > 0 && oks) ? *kept_last : -1;
       bool keep[GP];
       {
-        uint32_t bits = oks ? vote_bits(m_run) : 1u;
+        // bit 16: page j lies past the break (said by every warp that knows it)
+        uint32_t bits = oks ? vote_bits(m_run) : (wsr == 2 ? 16u : 1u);
+        if (oks && R > 0 && j - kl - 1 >= R) bits |= 16u;
         const uint32_t all = vote_round(rnd++, bits);
         if (all & 1u) { ok = false; break; }
-        keep[0] = (j == 0) || (all & 2u);
-        if (GP == 2) keep[GP - 1] = nb == 2 && (keep[0] ? (all & 4u) != 0 : (all & 8u) != 0);
+        const bool past0 = (all & 16u) != 0;
+        keep[0] = !past0 && ((j == 0) || (all & 2u));
+        if (GP == 2) {
+          const bool past1 = past0 || (R > 0 && !keep[0] && j - kl >= R);
+          keep[GP - 1] = !past1 && nb == 2 && (keep[0] ? (all & 4u) != 0 : (all & 8u) != 0);
+        }
       }
       // ---- state after this group's decisions: running max, and the exponent base
       // (with the O rescale factor) of each kept page
@@ -787,6 +856,11 @@ __global__ void __launch_bounds__(TcCfg<D, P>::NT, 1)
             }
           }
         if (nk == 0) mbar_arrive(b_sfree(sb, wg ^ 1));  // nothing kept: the S buffer goes back now
+        if (R > 0 && oks) {  // early break: the last kept page, and whether the rest is past it
+          const int kl2 = nk > 0 ? j + lastk : kl;
+          if (nk > 0) *kept_last = kl2;
+          if ((g + 1) * GP - kl2 - 1 >= R) atomicMin(const_cast<int*>(stop_g), g + 1);
+        }
       }
       mark_settled(g);
       // ---- P of the kept pages; their PV follows in list order
@@ -804,7 +878,12 @@ __global__ void __launch_bounds__(TcCfg<D, P>::NT, 1)
     }
     if (leader) {  // the second warpgroup to finish closes the queue
       __threadfence_block();
-      if (atomicAdd(wg_done, 1) == 1) *kq_final = *kq_count;
+      if (atomicAdd(wg_done, 1) == 1) {
+        *kq_final = *kq_count;
+        // pages of groups past an early break that no warpgroup reached: skipped
+        if (slog && R > 0)
+          for (int p = *stop_g * GP; p < n_list; ++p) slog[p] = 1;
+      }
     }
     // ---- epilogue: both warpgroups' row sums to one base, O / l -> bf16, LSE
     fin_rows[wg * 128 + row].x = l;
@@ -858,6 +937,25 @@ __global__ void __launch_bounds__(TcCfg<D, P>::NT, 1)
   // ---- teardown
   tc_fence_before();
   __syncthreads();
+  if (R > 0 && tid == 0) {
+    // After an early break some K copies may never have been consumed: wait for the last
+    // copy into every ring slot.  Slot s holds groups s, s + KG, ... in order, each
+    // loaded only after the one before it was read, so its last copy is the largest
+    // loaded group g = s (mod KG), phase g / KG; the producers loaded prefixes of their
+    // groups (group g by warp g % NPROD).
+    const uint64_t t0 = globaltimer_ns();
+    for (int s = 0; s < C::KG; ++s) {
+      int best = -1;
+      for (int kp = 0; kp < C::NPROD; ++kp)
+        for (int g = k_last[kp]; g >= 0 && g > k_last[kp] - C::NPROD * C::KG; g -= C::NPROD)
+          if (g % C::KG == s) {
+            best = max(best, g);
+            break;
+          }
+      if (best >= 0)
+        while (!mbar_try_wait(b_kfull(s), (best / C::KG) & 1) && globaltimer_ns() - t0 < tmo) {}
+    }
+  }
   if (warp == 3) {
     __syncwarp();
     tc_fence_after();

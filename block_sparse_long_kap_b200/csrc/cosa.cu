@@ -338,6 +338,7 @@ TcParams make_params(const cosa_shape_t* s, void* out, float* lse, const int32_t
   p.q_block = s->q_block;
   p.scale_log2 = s->softmax_scale * 1.4426950408889634f;
   p.log2_eps = -INFINITY;
+  p.max_run = 0;
   p.timeout_ns = kWaitTimeoutNs;
   return p;
 }
@@ -577,7 +578,7 @@ cosa_status_t cosa_osk_attention(const cosa_shape_t* shape, const cosa_osk_param
                                  int32_t* computed, uint8_t* skip_log, cosa_stream_t stream) {
   cosa_status_t e = check_shape(shape);
   if (e != COSA_OK) return e;
-  if (!osk || !(osk->eps >= 0.f)) return COSA_ERR_INVALID_ARG;
+  if (!osk || !(osk->eps >= 0.f) || osk->max_run < 0) return COSA_ERR_INVALID_ARG;
   if (!q || !k_pool || !v_pool || !page_table || !order || !count || !out)
     return COSA_ERR_INVALID_ARG;
   if (k_cap <= 0 || k_cap > shape->seq_len / shape->page_size) return COSA_ERR_INVALID_ARG;
@@ -591,6 +592,7 @@ cosa_status_t cosa_osk_attention(const cosa_shape_t* shape, const cosa_osk_param
   p.skip_log = skip_log;
   p.k_cap = k_cap;
   p.log2_eps = osk->eps > 0.f ? log2f(osk->eps) : -INFINITY;
+  p.max_run = osk->max_run;
   const long long grid = (long long)shape->batch * shape->num_q_heads * (shape->seq_len / shape->q_block);
   if (grid > 0x7fffffffll) return COSA_ERR_UNSUPPORTED;
   return launch_osk(shape, p, q, k_pool, v_pool, (int)grid, reinterpret_cast<cudaStream_t>(stream));
@@ -603,7 +605,8 @@ cosa_status_t cosa_osk_attention_group(const cosa_shape_t* shape, const cosa_osk
                                        int32_t* computed, uint8_t* skip_log, cosa_stream_t stream) {
   cosa_status_t e = check_shape(shape);
   if (e != COSA_OK) return e;
-  if (!osk || !(osk->eps >= 0.f)) return COSA_ERR_INVALID_ARG;
+  if (!osk || !(osk->eps >= 0.f) || osk->max_run < 0) return COSA_ERR_INVALID_ARG;
+  if (osk->max_run != 0) return COSA_ERR_UNSUPPORTED;  // the pair kernel has no early break
   if (!q || !k_pool || !v_pool || !page_table || !order || !count || !out)
     return COSA_ERR_INVALID_ARG;
   if (k_cap <= 0 || k_cap > shape->seq_len / shape->page_size) return COSA_ERR_INVALID_ARG;
@@ -688,7 +691,7 @@ cosa_status_t cosa_attention_host(const cosa_shape_t* shape, const cosa_kap_para
   HostLayout L;
   cosa_status_t e = host_layout(shape, kap, &L);
   if (e != COSA_OK) return e;
-  if (!osk || !(osk->eps >= 0.f)) return COSA_ERR_INVALID_ARG;
+  if (!osk || !(osk->eps >= 0.f) || osk->max_run < 0) return COSA_ERR_INVALID_ARG;
   if (!q_host || !k_pool_host || !v_pool_host || !page_table_host || !out_host)
     return COSA_ERR_INVALID_ARG;
   if (!workspace || workspace_bytes < L.total || reinterpret_cast<uintptr_t>(workspace) % 256)

@@ -99,10 +99,16 @@ typedef struct {
 
 /* Ordered-Skipping Kernel parameters (gist.science/pt §2.3). */
 typedef struct {
-  float eps; /* >= 0.  A listed page other than the first is skipped when, for every
-                row of the q-block that sees a key in it, (page max logit - running
-                max) < ln(eps).  0 never skips; +inf skips every page after the
-                first unless some row meets its first visible key there.          */
+  float eps;       /* >= 0.  A listed page other than the first is skipped when, for
+                      every row of the q-block that sees a key in it, (page max logit
+                      - running max) < ln(eps).  0 never skips; +inf skips every page
+                      after the first unless some row meets its first visible key
+                      there.                                                          */
+  int32_t max_run; /* >= 0.  0: the rule above alone (the pages' rule).  r > 0: once
+                      r consecutive listed pages have been skipped, the rest of the
+                      q-block's list is skipped without being visited (no K load,
+                      no QK^T): an early break, not part of the pages' method.
+                      cosa_osk_attention_group supports 0 only.                       */
 } cosa_osk_params_t;
 
 /* Status string for a status code (static storage, never NULL). */

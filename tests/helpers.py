@@ -60,14 +60,15 @@ def gpu_kap(shape: C.Shape, kap: C.KapParams, xd: dict, export=True):
     return order, count, scores, hrm
 
 
-def gpu_osk(shape: C.Shape, eps: float, xd: dict, order: torch.Tensor, count: torch.Tensor):
+def gpu_osk(shape: C.Shape, eps: float, xd: dict, order: torch.Tensor, count: torch.Tensor,
+            max_run: int = 0):
     B, Hq, N, D = shape.batch, shape.num_q_heads, shape.seq_len, shape.head_dim
     dev = xd["q"].device
     out = torch.full((B, Hq, N, D), float("nan"), dtype=torch.bfloat16, device=dev)
     lse = torch.full((B, Hq, N), float("nan"), dtype=torch.float32, device=dev)
     computed = torch.full((B, Hq, shape.num_q_blocks), -7, dtype=torch.int32, device=dev)
     skip = torch.full(tuple(order.shape), 7, dtype=torch.uint8, device=dev)
-    C.cosa_osk_attention(shape, C.OskParams(eps), xd["q"], xd["k_pool"], xd["v_pool"],
+    C.cosa_osk_attention(shape, C.OskParams(eps, max_run), xd["q"], xd["k_pool"], xd["v_pool"],
                          xd["page_table"], order, count, out, lse=lse, computed=computed,
                          skip_log=skip)
     torch.cuda.synchronize()

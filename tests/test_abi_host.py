@@ -176,3 +176,17 @@ def test_host_pipeline_workspace_and_argument_checks():
     # the binding refuses device-resident host arguments before calling in
     with pytest.raises((TypeError, ValueError)):
         C.cosa_attention_host(shp, kap, C.OskParams(1e-4), None, None, None, None, None, None)
+
+
+def test_early_break_argument_checks():
+    """max_run < 0 is an argument error; the group-shared kernel has no early break."""
+    lib = C.lib()
+    shp = C.Shape(1, 4, 2, 1024, 128, 64, 128)
+    s = shp.c()
+    neg = C._Osk(1e-4, -1)
+    assert lib.cosa_osk_attention(ctypes.byref(s), ctypes.byref(neg), 16, 16, 16, 16, 16, 16, 4,
+                                  16, None, None, None, None) == 1
+    brk = C._Osk(1e-4, 4)
+    assert lib.cosa_osk_attention_group(ctypes.byref(s), ctypes.byref(brk), 16, 16, 16, 16, 16,
+                                        16, 4, 16, None, None, None, None) == 2
+    assert C.OskParams(1e-3, 8).c().max_run == 8 and C.OskParams().c().max_run == 0

@@ -343,3 +343,75 @@ def test_dense_parity(case):
 
 def test_status_word_clear_after_runs():
     assert C.cosa_get_status() == 0
+
+
+# ---------------------------------------------------------------------------
+# early break (max_run): not part of the pages' method; parity with the oracle's
+# osk_block_rules(max_run=r)
+# ---------------------------------------------------------------------------
+BREAK_CASES = {  # workload, budget, eps, max_run values (eps large enough that tiles break)
+    "gqa-4k": (W.small_workload("gqa-32k", 4096, 8, 2, shuffle_pages=True), 0.25, 0.5, (2, 3)),
+    "narrow-kv-4k-g7": (W.small_workload("narrow-kv-64k", 4096, 7, 1, batch=2), 0.2, 1e-4, (2, 3)),
+    "wide-head-4k-p128": (W.small_workload("wide-head-128k", 4096, 8, 1), 0.3, 0.5, (2, 3)),
+}
+
+
+@pytest.mark.parametrize("case,r", [(c, r) for c in sorted(BREAK_CASES) for r in BREAK_CASES[c][3]])
+def test_osk_early_break_parity(case, r):
+    """The skip log equals the oracle's decisions page for page: where a decision lies
+    within rounding of the threshold, the oracle takes the kernel's decision there and
+    runs on (the break point moves with it); the first difference always precedes any
+    break, so its margin is defined.  Outputs and LSE then match the oracle run that
+    takes the same decisions, and some tiles do break."""
+    wl, budget, eps, _ = BREAK_CASES[case]
+    x = W.make_inputs(wl, seed=4)
+    xd = to_dev(x)
+    shape = shape_of(wl, x)
+    oa = _oracle_args(wl, x)
+    scale = 1 / math.sqrt(wl.head_dim)
+    sel = O.kap_select(oa["q"], oa["k_pool"], oa["page_table"], num_kv_heads=wl.num_kv_heads,
+                       page_size=wl.page_size, q_block=wl.q_block, q_sub=wl.q_block // 4,
+                       k_sub=16, scale=scale, budget=budget, sink_pages=1)
+    order = torch.from_numpy(sel["order"]).cuda()
+    count = torch.from_numpy(sel["count"]).cuda()
+    out, lse, computed, skip = gpu_osk(shape, eps, xd, order, count, max_run=r)
+    out, lse = np64(out), lse.cpu().numpy()
+    computed, skip = computed.cpu().numpy(), skip.cpu().numpy()
+    want_out = np.zeros_like(out)
+    want_lse = np.full_like(lse, -np.inf)
+    G = wl.num_q_heads // wl.num_kv_heads
+    N, Bq, P = wl.seq_len, wl.q_block, wl.page_size
+    logical = {}
+    n_breaks = n_forced = 0
+    for idx in np.ndindex(*sel["count"].shape):
+        b, h, qb = idx
+        n = int(sel["count"][idx])
+        lst = sel["order"][idx][:n]
+        if (b, h // G) not in logical:
+            logical[(b, h // G)] = (O.gather_logical(oa["k_pool"], oa["page_table"], b, h // G, N),
+                                    O.gather_logical(oa["v_pool"], oa["page_table"], b, h // G, N))
+        k_log, v_log = logical[(b, h // G)]
+        rows = slice(qb * Bq, (qb + 1) * Bq)
+        gs = skip[idx][:n]
+        assert np.all(skip[idx][n:] == 7), "skip log written past count"
+        force = {}
+        for _ in range(n + 1):
+            ref = O.osk_block_rules(oa["q"][b, h, rows], k_log, v_log, qb, Bq, P, lst, eps, scale,
+                                    force=force, max_run=r)
+            dis = np.nonzero(gs != ref["skip"])[0]
+            if len(dis) == 0:
+                break
+            j = int(dis[0])
+            assert abs(ref["margin"][j]) <= SKIP_MARGIN, f"decision differs outside the margin at {idx}"
+            force[j] = bool(gs[j])
+        assert np.array_equal(gs, ref["skip"])
+        assert computed[idx] == ref["computed"]
+        want_out[b, h, rows] = ref["out"]
+        want_lse[b, h, rows] = ref["lse"]
+        n_breaks += int(ref["visited"] < n)
+        n_forced += len(force)
+    n_tiles = int(np.prod(sel["count"].shape))
+    assert n_forced <= max(2, n_tiles // 100), f"{n_forced} decisions within the skip margin"
+    assert_out_close(out, want_out, f"osk break {case} r={r}")
+    assert_lse_close(lse, want_lse, f"osk break {case} r={r}")
+    assert n_breaks > 0, "no tile broke early: the case does not exercise the break"
