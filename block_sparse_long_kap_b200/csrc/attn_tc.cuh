@@ -57,6 +57,12 @@
 // timeout the CTA records COSA_ERR_TIMEOUT in the status word, drains what it
 // issued, frees TMEM and exits; a timed-out CTA makes every later CTA of the
 // launch exit at once.
+// Optional early break (max_run = r > 0, not part of the pages' method): a page with
+// r skipped pages right before it, and every page after it, is skipped unvisited.  The
+// exact path applies this page by page from the list position of the last kept page;
+// a stop group index, lowered once the break is proven from settled groups, ends the
+// K loads, the QK^T issue and the softmax loop early, and every wait that could be for
+// a group past it gives up.
 #pragma once
 
 #include "common.cuh"
