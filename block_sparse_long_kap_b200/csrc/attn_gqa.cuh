@@ -254,9 +254,9 @@ __global__ void __launch_bounds__(384, 1)
       }
       // loads never consumed (abort only) land before the CTA leaves
       const uint64_t t0 = globaltimer_ns();
-      while (!mbar_try_wait(b_q, 0) && globaltimer_ns() - t0 < tmo) {}
+      drain_wait(b_q, 0, t0, tmo);
       for (int x = max(0, g - C::KS); x < g; ++x)
-        while (!mbar_try_wait(b_kfull(x % C::KS), (x / C::KS) & 1) && globaltimer_ns() - t0 < tmo) {}
+        drain_wait(b_kfull(x % C::KS), (x / C::KS) & 1, t0, tmo);
     }
   } else if (warp == 2) {
     if (lane == 0) {
@@ -281,7 +281,7 @@ __global__ void __launch_bounds__(384, 1)
       }
       const uint64_t t0 = globaltimer_ns();
       for (int x = max(0, vc - C::VS); x < vc; ++x)
-        while (!mbar_try_wait(b_vfull(x % C::VS), (x / C::VS) & 1) && globaltimer_ns() - t0 < tmo) {}
+        drain_wait(b_vfull(x % C::VS), (x / C::VS) & 1, t0, tmo);
     }
   } else if (warp == 1) {
     if (lane == 0) {
@@ -358,7 +358,7 @@ __global__ void __launch_bounds__(384, 1)
       // every issued MMA completes before teardown frees TMEM
       mma_commit(b_done);
       const uint64_t t0 = globaltimer_ns();
-      while (!mbar_try_wait(b_done, 0) && globaltimer_ns() - t0 < tmo) {}
+      drain_wait(b_done, 0, t0, tmo);
     }
   } else if (warp >= 4 && active((warp - 4) >> 2)) {
     // ================= softmax of head i, one query row per thread ==================

@@ -82,6 +82,7 @@ struct TcParams {
   float scale_log2, log2_eps;
   int max_run;  // OSK early break after this many consecutive skipped pages; 0: none
   unsigned long long timeout_ns;
+  int fault_k_group;  // test hook: the K copies of this listed group are never issued (-1: none)
 };
 
 template <int D, int P>
@@ -392,11 +393,13 @@ __global__ void __launch_bounds__(TcCfg<D, P>::NT, 1)
         int cz[GP];
 #pragma unroll
         for (int t = 0; t < GP; ++t) cz[t] = __shfl_sync(0xffffffffu, cz_l, mm * GP + t);
+        // test hook: a withheld group's copies never arrive, so its waits run out
+        const bool withhold = g == prm.fault_k_group;
         // lane 0 posts the group's bytes, then lane t copies page t: copies issued from
         // separate threads stream side by side
-        if (lane == 0) mbar_arrive_expect_tx(b_kfull(s), (uint32_t)nb * C::KV_BYTES);
+        if (lane == 0 && !withhold) mbar_arrive_expect_tx(b_kfull(s), (uint32_t)nb * C::KV_BYTES);
         __syncwarp();
-        if (lane < nb) {
+        if (lane < nb && !withhold) {
           const int czt = (GP == 2 && lane == 1) ? cz[GP - 1] : cz[0];
 #pragma unroll
           for (int kb = 0; kb < D / 64; ++kb)
@@ -411,10 +414,9 @@ __global__ void __launch_bounds__(TcCfg<D, P>::NT, 1)
     if (lane == 0 && *abort_flag) {  // drain what was issued and never consumed
       const uint64_t t0 = globaltimer_ns();
       if (kp == 0)
-        while (!mbar_try_wait(b_q, 0) && globaltimer_ns() - t0 < tmo) {}
+        drain_wait(b_q, 0, t0, tmo);
       for (int g = last; g >= 0 && g > last - C::NPROD * C::KG; g -= C::NPROD)
-        while (!mbar_try_wait(b_kfull(g % C::KG), (g / C::KG) & 1) &&
-               globaltimer_ns() - t0 < tmo) {}
+        if (g != prm.fault_k_group) drain_wait(b_kfull(g % C::KG), (g / C::KG) & 1, t0, tmo);
     }
   } else if (warp == 2) {
     if (lane == 0) {
@@ -481,9 +483,9 @@ __global__ void __launch_bounds__(TcCfg<D, P>::NT, 1)
       // (abort only) land before the CTA leaves
       mma_commit(b_done_pv);
       const uint64_t t0 = globaltimer_ns();
-      while (!mbar_try_wait(b_done_pv, 0) && globaltimer_ns() - t0 < tmo) {}
+      drain_wait(b_done_pv, 0, t0, tmo);
       for (int x = c; x < nv; ++x)
-        while (!mbar_try_wait(b_vfull(x % C::VS), (x / C::VS) & 1) && globaltimer_ns() - t0 < tmo) {}
+        drain_wait(b_vfull(x % C::VS), (x / C::VS) & 1, t0, tmo);
     }
   } else if (warp == 3 || (C::TWO_QK && warp == 1)) {
     if (lane == 0) {
@@ -532,7 +534,7 @@ __global__ void __launch_bounds__(TcCfg<D, P>::NT, 1)
       const uint32_t bd = par == 0 ? b_done : b_done_odd;
       mma_commit(bd);
       const uint64_t t0 = globaltimer_ns();
-      while (!mbar_try_wait(bd, 0) && globaltimer_ns() - t0 < tmo) {}
+      drain_wait(bd, 0, t0, tmo);
     }
   } else if (warp >= 4) {
     // ================= softmax: two warpgroups taking the groups in turn ========
@@ -959,7 +961,7 @@ __global__ void __launch_bounds__(TcCfg<D, P>::NT, 1)
             break;
           }
       if (best >= 0)
-        while (!mbar_try_wait(b_kfull(s), (best / C::KG) & 1) && globaltimer_ns() - t0 < tmo) {}
+        drain_wait(b_kfull(s), (best / C::KG) & 1, t0, tmo);
     }
   }
   if (warp == 3) {

@@ -154,10 +154,9 @@ __global__ void __launch_bounds__(192, 1)
       }
       if (*abort_flag) {  // drain what was issued and never consumed
         const uint64_t t0 = globaltimer_ns();
-        while (!mbar_try_wait(b_afull, 0) && globaltimer_ns() - t0 < tmo) {}
+        drain_wait(b_afull, 0, t0, tmo);
         for (int it = max(0, issued - C::STAGES); it < issued; ++it)
-          while (!mbar_try_wait(b_bfull(it % C::STAGES), (it / C::STAGES) & 1) &&
-                 globaltimer_ns() - t0 < tmo) {}
+          drain_wait(b_bfull(it % C::STAGES), (it / C::STAGES) & 1, t0, tmo);
       }
     }
   } else if (warp == 1) {
@@ -190,7 +189,7 @@ __global__ void __launch_bounds__(192, 1)
       }
       mma_commit(b_done);
       const uint64_t t0 = globaltimer_ns();
-      while (!mbar_try_wait(b_done, 0) && globaltimer_ns() - t0 < tmo) {}
+      drain_wait(b_done, 0, t0, tmo);
     }
   } else {
     // ================= epilogue: thread = row = TMEM lane =================

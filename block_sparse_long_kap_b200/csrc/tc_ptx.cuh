@@ -5,6 +5,8 @@
 #include <cuda.h>
 #include <stdint.h>
 
+#include "common.cuh"
+
 namespace cosa {
 namespace tc {
 
@@ -38,6 +40,21 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
       : "r"(bar), "r"(parity)
       : "memory");
   return ok != 0;
+}
+
+// Teardown wait, bounded by t0 + tmo: copies or MMAs that may still be in flight are
+// waited for before shared memory and TMEM are released.  Running out of time here
+// is recorded as a timeout (the CTA then leaves with work possibly still in flight,
+// which the status word reports).
+__device__ __forceinline__ bool drain_wait(uint32_t bar, uint32_t parity, uint64_t t0,
+                                           uint64_t tmo) {
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer_ns() - t0 >= tmo) {
+      set_status(COSA_ERR_TIMEOUT);
+      return false;
+    }
+  }
+  return true;
 }
 
 // As mbar_try_wait, but the thread may sleep up to suspend_ns waiting for the

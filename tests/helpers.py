@@ -151,3 +151,40 @@ def check_order_valid(order_g, count_g, S_ref, hrm_g, qb, Bq, P, sink, budget, d
             va, vb = val(a), val(b)
             assert va[0] > vb[0] or (va[0] == vb[0] and va[1] >= vb[1] - delta), \
                 f"qb {qb}: {a} {va} listed before {b} {vb}"
+
+
+def check_osk_tiles(skip, computed, out, lse, ref, count, tiles, q_block, page_size, eps, vmax,
+                    what):
+    """Compare one OSK launch with the oracle on the given (b, h, qb) tiles.
+
+    skip / computed / out / lse are the kernel's (numpy; the skip log was
+    pre-filled with 7 so that writes past count show), ref the oracle's
+    osk_attention on the same lists.  Skip decisions are bit-exact outside the
+    float64 margin SKIP_MARGIN; a tile with a decision inside it is held to the
+    skip error bound instead of the element-wise bar.  Returns the number of
+    steps checked and of steps inside the margin."""
+    rows_ok = np.zeros(out.shape[:3], dtype=bool)
+    n_amb = n_steps = 0
+    for (b, h, qb) in tiles:
+        idx = (b, h, qb)
+        n = int(count[idx])
+        n_steps += n
+        gs, rs, mg = skip[idx][:n], ref["skip"][idx][:n], ref["margin"][idx][:n]
+        assert np.all(skip[idx][n:] == 7), f"{what}: skip log written past count at {idx}"
+        assert computed[idx] == n - int(gs.sum()), f"{what}: computed != unskipped at {idx}"
+        amb = np.abs(mg) <= SKIP_MARGIN
+        n_amb += int(amb.sum())
+        dis = gs != rs
+        assert not np.any(dis & ~amb), f"{what}: skip decision differs outside the margin at {idx}"
+        rows = slice(qb * q_block, (qb + 1) * q_block)
+        if dis.any():
+            bound = 2 * int(dis.sum()) * page_size * eps * vmax
+            assert np.abs(out[b, h, rows] - ref["out"][b, h, rows]).max() <= bound + OUT_MAX_ABS
+        else:
+            assert computed[idx] == ref["computed"][idx], f"{what}: computed differs at {idx}"
+            rows_ok[b, h, rows] = True
+    assert n_amb <= max(2, n_steps // 1000), f"{what}: {n_amb} of {n_steps} steps in the margin"
+    assert rows_ok.any(), f"{what}: no tile compared element-wise"
+    assert_out_close(out, ref["out"], what, rows_mask=rows_ok)
+    assert_lse_close(lse, ref["lse"], what, rows_mask=rows_ok)
+    return n_steps, n_amb

@@ -190,3 +190,14 @@ def test_early_break_argument_checks():
     assert lib.cosa_osk_attention_group(ctypes.byref(s), ctypes.byref(brk), 16, 16, 16, 16, 16,
                                         16, 4, 16, None, None, None, None) == 2
     assert C.OskParams(1e-3, 8).c().max_run == 8 and C.OskParams().c().max_run == 0
+
+
+def test_wait_fault_hook_argument_checks_on_host():
+    """The test hook (cosa_debug_osk_wait_fault) only records a one-shot setting:
+    no CUDA call, so it is checked here; a group below -1 is rejected."""
+    lib = C.lib()
+    assert lib.cosa_debug_osk_wait_fault(-2, 0) == 1
+    assert lib.cosa_debug_osk_wait_fault(-1, 0) == 0
+    # consumed by the next OSK call even when that call fails its own checks
+    assert lib.cosa_osk_attention(None, None, None, None, None, None, None, None, 0, None, None,
+                                  None, None, None) == 1

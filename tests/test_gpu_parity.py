@@ -14,7 +14,8 @@ import block_sparse_long_kap_b200 as C
 import oracle as O
 import workloads as W
 from helpers import (SKIP_MARGIN, assert_lse_close, assert_out_close, check_order_valid,
-                     gpu_dense, gpu_kap, gpu_osk, np64, score_tolerance, shape_of, to_dev)
+                     check_osk_tiles, gpu_dense, gpu_kap, gpu_osk, np64, score_tolerance,
+                     shape_of, to_dev)
 
 pytestmark = pytest.mark.gpu
 
@@ -115,6 +116,12 @@ def test_kap_select_parity(case):
                                   h_g[b, h, qb], qb, wl.q_block, wl.page_size, 1, budget, 2 * tol,
                                   False)
     assert n_hrm_diff <= max(1, wl.batch * wl.num_q_heads * nQB // 100)
+    # bit-exact: the oracle's selection and order run on the GPU's own fp32 scores and
+    # flags give the GPU's list (the fused order kernel ranks by exactly those values)
+    want_o, want_c = O.kap_order(S_g, h_g, page_size=wl.page_size, q_block=wl.q_block,
+                                 budget=budget, sink_pages=1)
+    np.testing.assert_array_equal(c, want_c)
+    np.testing.assert_array_equal(o, want_o)
 
 
 def test_kap_planted_pages_first_on_gpu():
@@ -288,9 +295,21 @@ def test_osk_never_reads_unlisted_pages():
     ref = O.osk_attention(oa["q"], oa["k_pool"], oa["v_pool"], oa["page_table"], o, c,
                           num_kv_heads=1, page_size=64, q_block=128, eps=1e-4,
                           scale=1 / math.sqrt(128))
-    amb = np.abs(np.nan_to_num(ref["margin"], nan=1.0)) <= SKIP_MARGIN
-    if not amb.any():
-        assert_out_close(np64(out_a), ref["out"], "osk on host-built lists")
+    # every tile whose decisions are clear of the threshold's rounding is compared
+    # element-wise (check_osk_tiles), the others against the skip error bound
+    tiles = [(0, h, qb) for h in range(Hq) for qb in range(nQB)]
+    skip_a = torch.full((B, Hq, nQB, kc), 7, dtype=torch.uint8, device="cuda")
+    comp_a = torch.full((B, Hq, nQB), -7, dtype=torch.int32, device="cuda")
+    out_c = torch.empty_like(out_a)
+    lse_c = torch.empty_like(lse_a)
+    C.cosa_osk_attention(shape, C.OskParams(1e-4), xd2["q"], kp, vp, pt, order, count, out_c,
+                         lse=lse_c, computed=comp_a, skip_log=skip_a)
+    torch.cuda.synchronize()
+    assert C.cosa_get_status() == 0
+    assert torch.equal(out_c, out_a)
+    check_osk_tiles(skip_a.cpu().numpy(), comp_a.cpu().numpy(), np64(out_a), lse_a.cpu().numpy(),
+                    ref, c, tiles, 128, 64, 1e-4, float(np.abs(oa["v_pool"]).max()),
+                    "osk on host-built lists")
 
 
 def test_osk_infinite_eps_with_page0_first():
@@ -415,3 +434,22 @@ def test_osk_early_break_parity(case, r):
     assert_out_close(out, want_out, f"osk break {case} r={r}")
     assert_lse_close(lse, want_lse, f"osk break {case} r={r}")
     assert n_breaks > 0, "no tile broke early: the case does not exercise the break"
+
+
+def test_kap_pool_then_rank_equals_kap_select():
+    """The two stage entry points on one workspace are cosa_kap_select, bit for bit."""
+    wl = W.small_workload("narrow-kv-64k", 4096, 14, 2, batch=2)
+    x = W.make_inputs(wl, seed=12)
+    xd = to_dev(x)
+    shape = shape_of(wl, x)
+    kap = C.KapParams(budget=0.2, q_sub=32, k_sub=16, sink_pages=1)
+    o1, c1, s1, h1 = gpu_kap(shape, kap, xd)
+    o2, c2, s2, h2 = (torch.full_like(o1, -7), torch.full_like(c1, -7), torch.full_like(s1, -1),
+                      torch.full_like(h1, 9))
+    ws = torch.empty(C.cosa_kap_workspace_size(shape, kap), dtype=torch.uint8, device="cuda")
+    C.cosa_kap_pool(shape, kap, xd["q"], xd["k_pool"], xd["page_table"], ws)
+    C.cosa_kap_rank(shape, kap, o2, c2, ws, scores=s2, hrm=h2)
+    torch.cuda.synchronize()
+    assert C.cosa_get_status() == 0
+    assert torch.equal(o1, o2) and torch.equal(c1, c2)
+    assert torch.equal(s1, s2) and torch.equal(h1, h2)

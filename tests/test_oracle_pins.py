@@ -293,6 +293,40 @@ def test_osk_full_budget_no_skip_equals_dense():
         assert comp == n_b and sk.sum() == 0
 
 
+def test_osk_attention_whole_problem_gqa_equals_sdpa():
+    """osk_attention over a whole GQA problem (4 query heads on 2 KV heads, batch 2,
+    shuffled page table, 32-token pages, 64-row q-blocks) with every causal page
+    listed in a random order and eps = 0 is exact causal attention in which query
+    head h reads KV head h // 2 (torch SDPA on repeat-interleaved K and V).  A wrong
+    head map (h % H_kv), a wrong page-table gather or a q-block row offset fails it."""
+    wl = W.small_workload("gqa-32k", 512, num_q_heads=4, num_kv_heads=2, batch=2, head_dim=32,
+                          page_size=32, q_block=64, shuffle_pages=True)
+    x = W.make_inputs(wl, seed=15, keep_logical=True)
+    scale = 1 / math.sqrt(32)
+    nQB, kc = 512 // 64, 512 // 32
+    g = np.random.default_rng(15)
+    order = np.full((2, 4, nQB, kc), -1, dtype=np.int32)
+    count = np.zeros((2, 4, nQB), dtype=np.int32)
+    for b in range(2):
+        for h in range(4):
+            for qb in range(nQB):
+                n = O.causal_pages(qb, 64, 32)
+                order[b, h, qb, :n] = g.permutation(n)
+                count[b, h, qb] = n
+    r = O.osk_attention(x["q"].double().numpy(), x["k_pool"].double().numpy(),
+                        x["v_pool"].double().numpy(), x["page_table"].numpy(), order, count,
+                        num_kv_heads=2, page_size=32, q_block=64, eps=0.0, scale=scale)
+    q = x["q"].double()
+    k = x["k_log"].double().repeat_interleave(2, dim=1)
+    v = x["v_log"].double().repeat_interleave(2, dim=1)
+    want = torch.nn.functional.scaled_dot_product_attention(q, k, v, is_causal=True, scale=scale)
+    np.testing.assert_allclose(r["out"], want.numpy(), rtol=0, atol=1e-12)
+    np.testing.assert_array_equal(r["computed"], count)
+    s = torch.einsum("bhid,bhjd->bhij", q, k) * scale
+    s = s.masked_fill(torch.ones(512, 512, dtype=torch.bool).triu(1), -math.inf)
+    np.testing.assert_allclose(r["lse"], torch.logsumexp(s, -1).numpy(), rtol=0, atol=1e-11)
+
+
 def test_osk_order_invariance_every_permutation():
     q, k, v = _tiny_problem(seed=7)
     P, Bq, scale = 16, 16, 1 / math.sqrt(8)
