@@ -34,23 +34,42 @@ METRIC = "128K causal prefill attention ms & effective TFLOP/s; % of bf16 tensor
 WORKLOAD = "gqa-128k"
 
 
-# DRAM traffic (read + write) of one OSK launch at gqa-128k, from one ncu capture
-# (profiles/osk_attention_gqa-128k_traffic.md).  It describes the kernel source the
-# capture ran, identified by the hash below; any other source reports null.
-OSK_TRAFFIC = {"workload": "gqa-128k", "bytes": 2695605504, "source_sha256_16": "37ec78a68845158c"}
+# DRAM traffic (read + write) of one launch at gqa-128k, from the ncu traffic captures
+# of these kernels.  Each figure describes the kernel source the capture ran,
+# identified by a hash of the files below; any other source reports null.
+TRAFFIC = {
+    "osk": {"workload": "gqa-128k", "bytes": None, "source_sha256_16": None,
+            "files": ("attn_tc.cuh", "tc_ptx.cuh", "common.cuh")},
+    "kap_pool": {"workload": "gqa-128k", "bytes": None, "source_sha256_16": None,
+                 "files": ("kap.cuh", "common.cuh")},
+}
 
 
-def _osk_traffic(workload: str):
+def source_hash(files) -> str:
     import hashlib
     h = hashlib.sha256()
     csrc = os.path.join(os.path.dirname(os.path.abspath(__file__)), "block_sparse_long_kap_b200",
                         "csrc")
-    for f in ("attn_tc.cuh", "tc_ptx.cuh", "common.cuh"):
+    for f in files:
         with open(os.path.join(csrc, f), "rb") as fh:
             h.update(fh.read())
-    if workload != OSK_TRAFFIC["workload"] or h.hexdigest()[:16] != OSK_TRAFFIC["source_sha256_16"]:
+    return h.hexdigest()[:16]
+
+
+def _traffic(kernel: str, workload: str):
+    t = TRAFFIC[kernel]
+    if t["bytes"] is None or workload != t["workload"] or \
+            source_hash(t["files"]) != t["source_sha256_16"]:
         return None
-    return OSK_TRAFFIC["bytes"]
+    return t["bytes"]
+
+
+def _osk_traffic(workload: str):
+    return _traffic("osk", workload)
+
+
+def _pool_traffic(workload: str):
+    return _traffic("kap_pool", workload)
 
 
 def _peaks():
@@ -115,8 +134,11 @@ class ClockSampler:
         except Exception:
             pass
         try:
+            import torch
+            # by UUID: under CUDA_VISIBLE_DEVICES the torch ordinal can name another GPU
+            gid = "GPU-" + str(torch.cuda.get_device_properties(self.dev).uuid)
             self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.dev}", f"--query-gpu={self.FIELDS}",
+                ["nvidia-smi", f"--id={gid}", f"--query-gpu={self.FIELDS}",
                  "--format=csv,noheader,nounits", "-lms", "100"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self._t = threading.Thread(target=self._read, daemon=True)
@@ -262,9 +284,10 @@ def run_reference(args):
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": full_ms, "higher_is_better": True, "scaling": "weak",
+        "ms_per_step": full_ms, "higher_is_better": True,
+        "scaling": "strong" if args.shard == "kv-heads" else "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": _config(wl, budget, eps),
+        "config": _config(wl, budget, eps, args.shard, args.gpus),
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads or cores,
                          "kind": "oracle", "sample": desc + " (ms_per_step extrapolated to the full layer)"},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -273,13 +296,138 @@ def run_reference(args):
     return 0
 
 
-def _config(wl, budget, eps):
+def kv_head_shard(rank: int, world: int, num_kv_heads: int):
+    """KV heads [h0, h1) of this rank when one layer's KV heads are split evenly over
+    the ranks.  Heads are independent in both stages (per-head pooling, scoring,
+    lists and attention), so each rank runs its heads' Q and KV pages alone and the
+    outputs stay head-sharded, as in tensor-parallel attention: no data exchange."""
+    if world < 1 or num_kv_heads % world:
+        raise ValueError(f"{num_kv_heads} KV heads do not split evenly over {world} ranks")
+    n = num_kv_heads // world
+    return rank * n, (rank + 1) * n
+
+
+def shard_inputs(x: dict, num_q_heads: int, num_kv_heads: int, h0: int, h1: int) -> dict:
+    """The inputs of KV heads [h0, h1): their G query heads of Q and their column of
+    the K and V page pools (contiguous copies); the page table is shared."""
+    G = num_q_heads // num_kv_heads
+    return {"q": x["q"][:, h0 * G:h1 * G].contiguous(),
+            "k_pool": x["k_pool"][:, h0:h1].contiguous(),
+            "v_pool": x["v_pool"][:, h0:h1].contiguous(),
+            "page_table": x["page_table"]}
+
+
+def strong_value(flop_job: float, ms: float) -> float:
+    """Whole-job TFLOP/s when the ranks split one job: its FLOP over the slowest
+    rank's time."""
+    return flop_job / (ms * 1e-3) / 1e12
+
+
+def kap_pool_bytes(batch, num_q_heads, num_kv_heads, seq_len, head_dim, q_sub, k_sub) -> float:
+    """Algorithmic DRAM bytes of one KAP pooling launch: Q and K read once (bf16), the
+    pooled vectors written once as two fp32 TF32 terms."""
+    read = 2.0 * batch * seq_len * head_dim * (num_q_heads + num_kv_heads)
+    write = 2 * 4.0 * head_dim * batch * (num_q_heads * seq_len / q_sub + num_kv_heads * seq_len / k_sub)
+    return read + write
+
+
+def _config(wl, budget, eps, shard, world):
+    par = ("kv-head shards: one layer's KV heads split evenly over the GPUs, outputs "
+           "head-sharded, no data exchange" if shard == "kv-heads"
+           else "independent layer per GPU")
     return {"workload": wl.name, "batch": wl.batch, "num_q_heads": wl.num_q_heads,
             "num_kv_heads": wl.num_kv_heads, "seq_len": wl.seq_len, "head_dim": wl.head_dim,
-            "page_size": wl.page_size, "q_block": wl.q_block, "page_table": "shuffled",
+            "page_size": wl.page_size, "q_block": wl.q_block,
+            "page_table": "shuffled" if wl.shuffle_pages else "identity",
             "budget": budget, "eps": eps, "q_sub": wl.q_block // 4, "k_sub": 16, "sink_pages": 1,
             "l2": "inputs larger than L2 (Q 1 GiB + K/V 0.5 GiB read per step)",
-            "parallelism": "independent layer per GPU"}
+            "parallelism": f"{par} ({world} GPU{'s' if world > 1 else ''})"}
+
+
+def _timed(fn, reps, stream, warm=1):
+    """Mean CUDA-event time (ms) of fn() over reps calls on stream, after warm calls."""
+    import torch
+    for _ in range(warm):
+        fn()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(reps):
+        fn()
+    e1.record(stream)
+    e1.synchronize()
+    return e0.elapsed_time(e1) / reps
+
+
+# Per-budget sweep (the speedup over the own dense kernel at each budget, and the ordered
+# against the page-order visit): workload -> (budgets, eps values, visit orders)
+SWEEP = (
+    ("wide-head-128k", (0.05, 0.10, 0.15, 0.20, 0.25, 0.30, 0.40, 0.50), (1e-4, 0.0), (False,)),
+    ("narrow-kv-64k", (0.05, 0.10, 0.20), (1e-4,), (False, True)),
+    ("gqa-32k", (0.10, 0.25, 0.50), (1e-4, 0.0), (False,)),
+)
+
+
+def budget_sweep(C, W, dev, stream, burst, reps=3):
+    """KAP + OSK at every budget / eps / visit order of SWEEP on each workload's seeded
+    inputs, against the own dense kernel on the same inputs: ms, speedup, the pages kept
+    and computed as fractions of the causal pages, visited TFLOP/s and the output's
+    relative L2 distance from the dense output."""
+    import torch
+    res = {}
+    for name, budgets, eps_list, modes in SWEEP:
+        wl = W.WORKLOADS[name]
+        x = W.make_inputs(wl, seed=0, device=str(dev))
+        B, Hq, N, D = wl.batch, wl.num_q_heads, wl.seq_len, wl.head_dim
+        shape = C.Shape(B, Hq, wl.num_kv_heads, N, D, wl.page_size, wl.q_block)
+        dense_out = torch.empty(B, Hq, N, D, dtype=torch.bfloat16, device=dev)
+        dense_ms = _timed(lambda: C.cosa_dense_attention(shape, x["q"], x["k_pool"], x["v_pool"],
+                                                         x["page_table"], dense_out,
+                                                         stream=stream), reps, stream)
+        dref = dense_out.float()
+        dnorm = float(dref.norm())
+        out = torch.empty_like(dense_out)
+        comp = torch.empty(B, Hq, shape.num_q_blocks, dtype=torch.int32, device=dev)
+        n_b_total = sum(((qb + 1) * wl.q_block + wl.page_size - 1) // wl.page_size
+                        for qb in range(shape.num_q_blocks)) * B * Hq
+        tile = 2.0 * wl.q_block * wl.page_size * D
+        pts = []
+        for asc in modes:
+            for budget in budgets:
+                kap = C.KapParams(budget=budget, q_sub=wl.q_block // 4, k_sub=16, sink_pages=1,
+                                  ascending=asc)
+                kc = C.cosa_kap_kcap(shape, kap)
+                order = torch.empty(B, Hq, shape.num_q_blocks, kc, dtype=torch.int32, device=dev)
+                count = torch.empty(B, Hq, shape.num_q_blocks, dtype=torch.int32, device=dev)
+                ws = torch.empty(C.cosa_kap_workspace_size(shape, kap), dtype=torch.uint8,
+                                 device=dev)
+                kap_ms = _timed(lambda: C.cosa_kap_select(shape, kap, x["q"], x["k_pool"],
+                                                          x["page_table"], order, count, ws,
+                                                          stream=stream), reps, stream)
+                listed = int(count.to(torch.int64).sum().item())
+                for eps in eps_list:
+                    osk = C.OskParams(eps=eps)
+                    osk_ms = _timed(lambda: C.cosa_osk_attention(
+                        shape, osk, x["q"], x["k_pool"], x["v_pool"], x["page_table"], order,
+                        count, out, computed=comp, stream=stream), reps, stream)
+                    if C.cosa_get_status(stream) != 0:
+                        raise RuntimeError(f"in-kernel error status in the sweep ({name})")
+                    cmp_ = int(comp.to(torch.int64).sum().item())
+                    vis_tf = tile * (listed + cmp_) / (osk_ms * 1e-3) / 1e12
+                    pts.append({
+                        "budget": budget, "eps": eps, "visit": "page order" if asc else "ordered",
+                        "kap_ms": kap_ms, "osk_ms": osk_ms, "ms": kap_ms + osk_ms,
+                        "speedup_vs_dense": dense_ms / (kap_ms + osk_ms),
+                        "kept_frac": listed / n_b_total, "computed_frac": cmp_ / n_b_total,
+                        "visited_tflops": vis_tf, "visited_frac_vs_burst": vis_tf / burst,
+                        "effective_tflops": wl.dense_flops() / ((kap_ms + osk_ms) * 1e-3) / 1e12,
+                        "rel_l2_vs_dense": float((out.float() - dref).norm()) / dnorm})
+                del order, count, ws
+        res[name] = {"dense_ms": dense_ms,
+                     "dense_tflops": wl.dense_flops() / (dense_ms * 1e-3) / 1e12,
+                     "points": pts}
+        del x, dense_out, out, dref
+        torch.cuda.empty_cache()
+    return res
 
 
 def main():
@@ -291,7 +439,12 @@ def main():
     ap.add_argument("--workload", default=WORKLOAD)
     ap.add_argument("--budget", type=float, default=0.2)
     ap.add_argument("--eps", type=float, default=1e-4)
+    ap.add_argument("--shard", default="kv-heads", choices=["kv-heads", "replica"],
+                    help="N > 1: split one layer's KV heads over the GPUs (strong scaling), "
+                         "or run an independent layer on each (weak scaling)")
     ap.add_argument("--no-extras", action="store_true", help="skip dense/sweep/e2e/cpu legs")
+    ap.add_argument("--sweep-only", action="store_true",
+                    help="run only the per-budget sweep and print it")
     ap.add_argument("--dense-only", action="store_true",
                     help="time only the dense kernel on the workload (for profiling it)")
     args = ap.parse_args()
@@ -300,7 +453,6 @@ def main():
     if args.impl == "reference":
         return run_reference(args)
 
-    import numpy as np
     import torch
     import torch.distributed as dist
 
@@ -316,58 +468,79 @@ def main():
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=dev)
+    stream = torch.cuda.current_stream(dev)
+    peaks, peak_src = _peaks()
+    burst = float(peaks.get("bf16_tflops", 1590.0))
+    sustained = float(peaks.get("bf16_tflops_sustained", burst))
+    hbm = float(peaks.get("hbm_gbs", 6650.0))
+
+    if args.sweep_only:
+        sw = budget_sweep(C, W, dev, stream, burst)
+        if rank == 0:
+            print(json.dumps({"budget_sweep": sw}), flush=True)
+        if world > 1:
+            dist.destroy_process_group()
+        return 0
 
     wl = W.WORKLOADS[args.workload]
-    x = W.make_inputs(wl, seed=rank, device=str(dev))
-    shape = C.Shape(wl.batch, wl.num_q_heads, wl.num_kv_heads, wl.seq_len, wl.head_dim,
-                    wl.page_size, wl.q_block)
+    B, N, D = wl.batch, wl.seq_len, wl.head_dim
+    G = wl.num_q_heads // wl.num_kv_heads
+    if args.shard == "kv-heads":
+        # every rank draws the same layer and keeps its KV heads' share
+        h0, h1 = kv_head_shard(rank, world, wl.num_kv_heads)
+        x = shard_inputs(W.make_inputs(wl, seed=0, device=str(dev)), wl.num_q_heads,
+                         wl.num_kv_heads, h0, h1)
+        torch.cuda.empty_cache()
+    else:
+        h0, h1 = 0, wl.num_kv_heads
+        x = W.make_inputs(wl, seed=rank, device=str(dev))
+    Hk = h1 - h0
+    Hq = Hk * G
+    shape = C.Shape(B, Hq, Hk, N, D, wl.page_size, wl.q_block,
+                    pages_per_seq=x["page_table"].shape[1], num_phys_pages=x["k_pool"].shape[0])
     kap = C.KapParams(budget=args.budget, q_sub=wl.q_block // 4, k_sub=16, sink_pages=1)
     osk = C.OskParams(eps=args.eps)
-    B, Hq, N, D = wl.batch, wl.num_q_heads, wl.seq_len, wl.head_dim
     kc = C.cosa_kap_kcap(shape, kap)
     order = torch.empty(B, Hq, shape.num_q_blocks, kc, dtype=torch.int32, device=dev)
     count = torch.empty(B, Hq, shape.num_q_blocks, dtype=torch.int32, device=dev)
     ws = torch.empty(C.cosa_kap_workspace_size(shape, kap), dtype=torch.uint8, device=dev)
     out = torch.empty(B, Hq, N, D, dtype=torch.bfloat16, device=dev)
     computed = torch.empty(B, Hq, shape.num_q_blocks, dtype=torch.int32, device=dev)
-    stream = torch.cuda.current_stream(dev)
+    dense_flop = wl.dense_flops()  # of one whole layer
+
+    def job_value(ms):
+        if args.shard == "kv-heads":
+            return strong_value(dense_flop, ms)
+        return weak_value(world, dense_flop, ms)
 
     def step(ev=None):
+        # cosa_kap_pool + cosa_kap_rank is cosa_kap_select, with an event between the two
         if ev is not None:
             ev[0].record(stream)
-        C.cosa_kap_select(shape, kap, x["q"], x["k_pool"], x["page_table"], order, count, ws,
-                          stream=stream)
+        C.cosa_kap_pool(shape, kap, x["q"], x["k_pool"], x["page_table"], ws, stream=stream)
         if ev is not None:
             ev[1].record(stream)
+        C.cosa_kap_rank(shape, kap, order, count, ws, stream=stream)
+        if ev is not None:
+            ev[2].record(stream)
         C.cosa_osk_attention(shape, osk, x["q"], x["k_pool"], x["v_pool"], x["page_table"], order,
                              count, out, computed=computed, stream=stream)
         if ev is not None:
-            ev[2].record(stream)
+            ev[3].record(stream)
 
     def barrier():
         if world > 1:
             dist.barrier()
 
-
     if args.dense_only:
-        dense_flop = 4.0 * B * Hq * D * N * (N + 1) / 2
-        for _ in range(args.warmup):
-            C.cosa_dense_attention(shape, x["q"], x["k_pool"], x["v_pool"], x["page_table"], out,
-                                   stream=stream)
-        torch.cuda.synchronize(dev)
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(args.steps):
-            C.cosa_dense_attention(shape, x["q"], x["k_pool"], x["v_pool"], x["page_table"], out,
-                                   stream=stream)
-        e1.record(stream)
-        torch.cuda.synchronize(dev)
+        ms = _timed(lambda: C.cosa_dense_attention(shape, x["q"], x["k_pool"], x["v_pool"],
+                                                   x["page_table"], out, stream=stream),
+                    args.steps, stream, warm=args.warmup)
         assert C.cosa_get_status(stream) == 0
-        ms = e0.elapsed_time(e1) / max(args.steps, 1)
         if rank == 0:
             print(json.dumps({"kernel": "dense_attention", "workload": args.workload, "ms": ms,
-                              "tflops": dense_flop / (ms * 1e-3) / 1e12, "steps": args.steps,
-                              "warmup": args.warmup}), flush=True)
+                              "tflops": dense_flop * Hq / wl.num_q_heads / (ms * 1e-3) / 1e12,
+                              "steps": args.steps, "warmup": args.warmup}), flush=True)
         if world > 1:
             dist.destroy_process_group()
         return 0
@@ -377,7 +550,7 @@ def main():
     torch.cuda.synchronize(dev)
     assert C.cosa_get_status(stream) == 0
 
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
     clocks = ClockSampler(torch.cuda.current_device())
     barrier()
     torch.cuda.synchronize(dev)
@@ -392,24 +565,20 @@ def main():
     barrier()
     clk = clocks.stop()
     total_ms = max_over_ranks(t_start.elapsed_time(t_end), world, dev)
-    kap_ms = [e[0].elapsed_time(e[1]) for e in evs]
-    osk_ms = [e[1].elapsed_time(e[2]) for e in evs]
+    pool_ms = [e[0].elapsed_time(e[1]) for e in evs]
+    kap_ms = [e[0].elapsed_time(e[2]) for e in evs]
+    osk_ms = [e[2].elapsed_time(e[3]) for e in evs]
     assert C.cosa_get_status(stream) == 0
 
     ms_per_step = total_ms / args.steps
-    dense_flop = wl.dense_flops()
-    value = weak_value(world, dense_flop, ms_per_step)
+    value = job_value(ms_per_step)
 
     # algorithmic work of the dominant kernel (OSK) for the roofline
-    cnt = count.to(torch.int64)
-    steps_visited = int(cnt.sum().item())
+    steps_visited = int(count.to(torch.int64).sum().item())
     steps_computed = int(computed.to(torch.int64).sum().item())
     tile = 2.0 * wl.q_block * wl.page_size * wl.head_dim
     osk_flop = tile * (steps_visited + steps_computed)
     osk_avg_ms = statistics.mean(osk_ms)
-    peaks, peak_src = _peaks()
-    burst = float(peaks.get("bf16_tflops", 1590.0))
-    sustained = float(peaks.get("bf16_tflops_sustained", burst))
     # the burst figure unless the clocks seen in the timed region sat well below max
     # (the sustained figure is a seconds-long GEMM under the power cap, at ~1.35 GHz)
     throttled = (clk.get("sm_mhz") is not None and clk.get("sm_max_mhz")
@@ -420,25 +589,43 @@ def main():
     achieved = osk_flop / (osk_avg_ms * 1e-3) / 1e12
     n_b_total = sum(((qb + 1) * wl.q_block + wl.page_size - 1) // wl.page_size
                     for qb in range(shape.num_q_blocks)) * B * Hq
+    pool_bytes = kap_pool_bytes(B, Hq, Hk, N, D, wl.q_block // 4, 16)
+    pool_avg_ms = statistics.mean(pool_ms)
+    pool_gbs = pool_bytes / (pool_avg_ms * 1e-3) / 1e9
 
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-        "data": "synthetic", "config": _config(wl, args.budget, args.eps),
+        "higher_is_better": True, "scaling": "strong" if args.shard == "kv-heads" else "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": _config(wl, args.budget, args.eps, args.shard, world),
         "gpu_launches": 4 * args.steps,
         "clocks": clk,
         "roofline": {"kernel": "osk_attention", "bound": "tensor", "achieved": achieved,
                      "peak": peak_tflops, "unit": "TFLOP/s", "frac": achieved / peak_tflops,
                      "peak_source": f"{peak_src} bf16 {peak_kind}",
                      "frac_vs_burst": achieved / burst, "frac_vs_sustained": achieved / sustained,
-                     "traffic": _osk_traffic(args.workload),
+                     "traffic": _osk_traffic(args.workload) if Hq == wl.num_q_heads else None,
                      "traffic_unit": "bytes per launch (DRAM read + write, ncu)",
-                     "work": "visited FLOP = 2*Bq*P*D*(visited pages + computed pages) per launch"},
-        "breakdown_ms": {"kap_select": statistics.mean(kap_ms), "osk_attention": osk_avg_ms},
+                     "work": "visited FLOP = 2*Bq*P*D*(visited pages + computed pages) per launch",
+                     "others": [{
+                         "kernel": "kap_pool_kernel", "bound": "hbm", "achieved": pool_gbs,
+                         "peak": hbm, "unit": "GB/s", "frac": pool_gbs / hbm,
+                         "peak_source": f"{peak_src} HBM copy bandwidth",
+                         "traffic": _pool_traffic(args.workload) if Hq == wl.num_q_heads else None,
+                         "traffic_unit": "bytes per launch (DRAM read + write, ncu)",
+                         "work": "Q and K read once (bf16) + pooled vectors written once "
+                                 f"(2 fp32 terms): {pool_bytes:.4g} B per launch",
+                         "ms": pool_avg_ms}]},
+        "breakdown_ms": {"kap_select": statistics.mean(kap_ms), "kap_pool": pool_avg_ms,
+                         "kap_rank": statistics.mean(kap_ms) - pool_avg_ms,
+                         "osk_attention": osk_avg_ms},
         "budgets": {"kap_kept_frac": steps_visited / n_b_total,
                     "osk_computed_frac": steps_computed / n_b_total},
     }
+    if world > 1:
+        line["shard"] = {"rank0_kv_heads": [h0, h1], "kv_heads_per_rank": Hk}
+
     # ---- end to end through the C-ABI with host buffers (every rank, every N) ---
     def e2e_leg():
         # through the library's host-buffer entry point: every step copies its inputs in
@@ -469,8 +656,9 @@ def main():
         e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, world, dev)
         h2d = sum(t.numel() * t.element_size() for t in (qh, kh, vh, pth))
         d2h = outh.numel() * outh.element_size()
-        return {"value": weak_value(world, dense_flop, e2e_ms), "unit": "TFLOP/s",
-                "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+        return {"value": job_value(e2e_ms), "unit": "TFLOP/s",
+                "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "entry_point": "cosa_attention_host"}
 
     if world > 1:
         line["e2e"] = e2e_leg()
@@ -483,47 +671,32 @@ def main():
 
     # ---- own dense kernel on the same inputs -------------------------------
     dense_out = torch.empty_like(out)
-    for _ in range(2):
-        C.cosa_dense_attention(shape, x["q"], x["k_pool"], x["v_pool"], x["page_table"], dense_out,
-                               stream=stream)
-    torch.cuda.synchronize(dev)
-    d_ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
-    d_ev[0].record(stream)
-    for _ in range(3):
-        C.cosa_dense_attention(shape, x["q"], x["k_pool"], x["v_pool"], x["page_table"], dense_out,
-                               stream=stream)
-    d_ev[1].record(stream)
-    torch.cuda.synchronize(dev)
-    dense_ms = d_ev[0].elapsed_time(d_ev[1]) / 3
+    dense_ms = _timed(lambda: C.cosa_dense_attention(shape, x["q"], x["k_pool"], x["v_pool"],
+                                                     x["page_table"], dense_out, stream=stream),
+                      3, stream, warm=2)
     dense_tf = dense_flop / (dense_ms * 1e-3) / 1e12
     line["dense"] = {"ms": dense_ms, "tflops": dense_tf, "frac_vs_burst": dense_tf / burst,
                      "frac_vs_sustained": dense_tf / sustained,
                      "speedup_sparse_vs_dense": dense_ms / ms_per_step}
+    k_mean = statistics.mean(kap_ms)
 
     # ---- eps sweep at this budget (OSK only, KAP list reused) --------------
     sweep = []
     for eps in wl.eps_list:
         o2 = C.OskParams(eps=eps)
-        C.cosa_osk_attention(shape, o2, x["q"], x["k_pool"], x["v_pool"], x["page_table"], order,
-                             count, out, computed=computed, stream=stream)
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(3):
-            C.cosa_osk_attention(shape, o2, x["q"], x["k_pool"], x["v_pool"], x["page_table"],
-                                 order, count, out, computed=computed, stream=stream)
-        e1.record(stream)
-        torch.cuda.synchronize(dev)
-        ms = e0.elapsed_time(e1) / 3
+        ms = _timed(lambda: C.cosa_osk_attention(shape, o2, x["q"], x["k_pool"], x["v_pool"],
+                                                 x["page_table"], order, count, out,
+                                                 computed=computed, stream=stream), 3, stream)
         comp = int(computed.to(torch.int64).sum().item())
         fl = tile * (steps_visited + comp)
-        sweep.append({"eps": eps, "osk_ms": ms, "kap_plus_osk_ms": ms + statistics.mean(kap_ms),
+        sweep.append({"eps": eps, "osk_ms": ms, "kap_plus_osk_ms": ms + k_mean,
                       "computed_frac": comp / n_b_total, "visited_tflops": fl / (ms * 1e-3) / 1e12,
-                      "speedup_vs_dense": dense_ms / (ms + statistics.mean(kap_ms))})
+                      "visited_frac_vs_burst": fl / (ms * 1e-3) / 1e12 / burst,
+                      "speedup_vs_dense": dense_ms / (ms + k_mean)})
     line["eps_sweep"] = sweep
 
     # ---- group-shared selection: one list per KV head and q-block (KAP group +
     # OSK over head pairs), same budget and eps; quality against the dense output
-    Hk = wl.num_kv_heads
     og = torch.empty(B, Hk, shape.num_q_blocks, kc, dtype=torch.int32, device=dev)
     cg = torch.empty(B, Hk, shape.num_q_blocks, dtype=torch.int32, device=dev)
     outg = torch.empty_like(out)
@@ -561,8 +734,7 @@ def main():
     def rel_l2(a):
         return float((a.float() - dref).norm() / dref.norm())
 
-    G_ = Hq // Hk
-    vis_g = G_ * int(cg.to(torch.int64).sum().item())
+    vis_g = G * int(cg.to(torch.int64).sum().item())
     comp_g = int(compg.to(torch.int64).sum().item())
     vis_tf = tile * (vis_g + comp_g) / (g_osk * 1e-3) / 1e12
     line["group_shared"] = {
@@ -578,29 +750,18 @@ def main():
         bout = torch.empty_like(out)
         bcomp = torch.empty_like(computed)
         pref = out.float()
-        k_ms = statistics.mean(kap_ms)
         res = []
         for r in (16, 8):
             o3 = C.OskParams(eps=args.eps, max_run=r)
-
-            def run():
-                C.cosa_osk_attention(shape, o3, x["q"], x["k_pool"], x["v_pool"], x["page_table"],
-                                     order, count, bout, computed=bcomp, stream=stream)
-
-            run()
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
-            for _ in range(3):
-                run()
-            e1.record(stream)
-            torch.cuda.synchronize(dev)
+            ms = _timed(lambda: C.cosa_osk_attention(shape, o3, x["q"], x["k_pool"], x["v_pool"],
+                                                     x["page_table"], order, count, bout,
+                                                     computed=bcomp, stream=stream), 3, stream)
             if C.cosa_get_status(stream) != 0:
                 raise RuntimeError("in-kernel error status")
-            ms = e0.elapsed_time(e1) / 3
             comp = int(bcomp.to(torch.int64).sum().item())
-            res.append({"max_run": r, "eps": args.eps, "osk_ms": ms, "kap_plus_osk_ms": ms + k_ms,
-                        "tflops": dense_flop / ((ms + k_ms) * 1e-3) / 1e12,
-                        "speedup_vs_dense": dense_ms / (ms + k_ms),
+            res.append({"max_run": r, "eps": args.eps, "osk_ms": ms, "kap_plus_osk_ms": ms + k_mean,
+                        "tflops": dense_flop / ((ms + k_mean) * 1e-3) / 1e12,
+                        "speedup_vs_dense": dense_ms / (ms + k_mean),
                         "computed_frac": comp / n_b_total,
                         "rel_l2_vs_pages_rule": float((bout.float() - pref).norm() / pref.norm()),
                         "rel_l2_vs_dense": rel_l2(bout)})
@@ -612,6 +773,14 @@ def main():
         line["early_break"] = {"error": repr(exc)}
 
     line["e2e"] = e2e_leg()
+    del dense_out, dref, outg
+    torch.cuda.empty_cache()
+
+    # ---- speedup per budget on the other long-context layers ----------------
+    try:
+        line["budget_sweep"] = budget_sweep(C, W, dev, stream, burst)
+    except Exception as exc:  # an extra leg: report the failure, keep the line
+        line["budget_sweep"] = {"error": repr(exc)}
 
     # ---- CPU oracle on a bounded sample of the same workload ----------------
     xh = {"q": x["q"][:, :1].cpu(), "k_pool": x["k_pool"][:, :1].cpu(),

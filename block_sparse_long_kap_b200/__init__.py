@@ -20,7 +20,7 @@ __all__ = [
     "cosa_kap_select", "cosa_kap_select_noalloc", "cosa_kap_order", "cosa_osk_attention",
     "cosa_dense_attention", "cosa_get_status", "EXPORTED_SYMBOLS", "NOALLOC_SCRATCH_BYTES",
     "cosa_kap_select_group", "cosa_osk_attention_group", "cosa_attention_host_workspace_size",
-    "cosa_attention_host",
+    "cosa_attention_host", "cosa_debug_osk_wait_fault", "cosa_kap_pool", "cosa_kap_rank",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -30,7 +30,8 @@ EXPORTED_SYMBOLS = (
     "cosa_status_string", "cosa_version", "cosa_kap_kcap", "cosa_kap_workspace_size",
     "cosa_kap_select", "cosa_kap_select_noalloc", "cosa_kap_order", "cosa_osk_attention",
     "cosa_dense_attention", "cosa_get_status", "cosa_kap_select_group", "cosa_osk_attention_group",
-    "cosa_attention_host_workspace_size", "cosa_attention_host",
+    "cosa_attention_host_workspace_size", "cosa_attention_host", "cosa_debug_osk_wait_fault",
+    "cosa_kap_pool", "cosa_kap_rank",
 )
 
 # Largest workspace the allocation-free Stage-1 entry point accepts (cosa.h).
@@ -151,6 +152,9 @@ def lib():
     L.cosa_get_status.argtypes = [vp]
     L.cosa_attention_host_workspace_size.argtypes = [P(_Shape), P(_Kap), P(sz)]
     L.cosa_attention_host.argtypes = [P(_Shape), P(_Kap), P(_Osk), vp, vp, vp, vp, vp, vp, sz, vp]
+    L.cosa_debug_osk_wait_fault.argtypes = [i32, ctypes.c_uint64]
+    L.cosa_kap_pool.argtypes = [P(_Shape), P(_Kap), vp, vp, vp, vp, sz, vp]
+    L.cosa_kap_rank.argtypes = [P(_Shape), P(_Kap), vp, vp, vp, vp, vp, sz, vp]
     for name in EXPORTED_SYMBOLS:
         if name not in ("cosa_status_string", "cosa_version"):
             getattr(L, name).restype = ctypes.c_int
@@ -239,6 +243,45 @@ def cosa_kap_select(shape: Shape, kap: KapParams, q, k_pool, page_table, order, 
                                  _ptr(page_table), _ptr(order), _ptr(count), _ptr(scores),
                                  _ptr(hrm), _ptr(workspace), nbytes, _stream(stream)),
            "cosa_kap_select")
+
+
+def cosa_kap_pool(shape: Shape, kap: KapParams, q, k_pool, page_table, workspace,
+                  stream=None) -> None:
+    """Stage 1, downsampling alone: pooled queries and keys into the workspace."""
+    import torch
+    s, k = shape.c(), kap.c(shape)
+    B, Hq, N, D = shape.batch, shape.num_q_heads, shape.seq_len, shape.head_dim
+    _expect(q, "q", torch.bfloat16, (B, Hq, N, D))
+    _expect(k_pool, "k_pool", torch.bfloat16, _kv_shape(shape))
+    _expect(page_table, "page_table", torch.int32, (B, s.pages_per_seq))
+    if workspace is None or not workspace.is_cuda:
+        raise ValueError("workspace must be a CUDA tensor")
+    nbytes = workspace.numel() * workspace.element_size()
+    _check(lib().cosa_kap_pool(ctypes.byref(s), ctypes.byref(k), _ptr(q), _ptr(k_pool),
+                               _ptr(page_table), _ptr(workspace), nbytes, _stream(stream)),
+           "cosa_kap_pool")
+
+
+def cosa_kap_rank(shape: Shape, kap: KapParams, order, count, workspace, scores=None, hrm=None,
+                  stream=None) -> None:
+    """Stage 1 after cosa_kap_pool on the same workspace: scores, MaxPool, MaxNorm,
+    HRM, selection and ordering (order, count, optional scores / hrm)."""
+    import torch
+    s, k = shape.c(), kap.c(shape)
+    B, Hq = shape.batch, shape.num_q_heads
+    kc = cosa_kap_kcap(shape, kap)
+    _expect(order, "order", torch.int32, (B, Hq, shape.num_q_blocks, kc))
+    _expect(count, "count", torch.int32, (B, Hq, shape.num_q_blocks))
+    if scores is not None:
+        _expect(scores, "scores", torch.float32, (B, Hq, shape.num_q_blocks, shape.num_pages))
+    if hrm is not None:
+        _expect(hrm, "hrm", torch.uint8, (B, Hq, shape.num_q_blocks, shape.num_pages))
+    if workspace is None or not workspace.is_cuda:
+        raise ValueError("workspace must be a CUDA tensor")
+    nbytes = workspace.numel() * workspace.element_size()
+    _check(lib().cosa_kap_rank(ctypes.byref(s), ctypes.byref(k), _ptr(order), _ptr(count),
+                               _ptr(scores), _ptr(hrm), _ptr(workspace), nbytes, _stream(stream)),
+           "cosa_kap_rank")
 
 
 def cosa_kap_select_group(shape: Shape, kap: KapParams, q, k_pool, page_table, order, count,
@@ -421,6 +464,14 @@ def cosa_attention_host(shape: Shape, kap: KapParams, osk: OskParams, q, k_pool,
                                      _ptr(k_pool), _ptr(v_pool), _ptr(page_table), _ptr(out),
                                      _ptr(workspace), workspace.numel(), _stream(stream)),
            "cosa_attention_host")
+
+
+def cosa_debug_osk_wait_fault(withhold_k_group: int, wait_limit_ns: int = 0) -> None:
+    """Test hook: the next cosa_osk_attention call from this thread runs with its waits
+    limited to wait_limit_ns and the K copies of listed group withhold_k_group never
+    issued (-1: none), so that a wait runs out on purpose (see cosa.h)."""
+    _check(lib().cosa_debug_osk_wait_fault(int(withhold_k_group), int(wait_limit_ns)),
+           "cosa_debug_osk_wait_fault")
 
 
 def cosa_get_status(stream=None) -> int:

@@ -187,11 +187,31 @@ cosa_status_t launch_order(const cosa_shape_t* s, const cosa_kap_params_t* k, bo
   return last_launch();
 }
 
+// K1: pooling of Q and of the paged K into the workspace
 template <int D>
-cosa_status_t launch_kap(const cosa_shape_t* s, const cosa_kap_params_t* k, const void* q,
-                         const void* k_pool, const int32_t* page_table, int32_t* order,
-                         int32_t* count, float* scores, uint8_t* hrm, const KapLayout& L,
-                         uint8_t* ws, int k_cap, cudaStream_t st, bool group = false) {
+cosa_status_t launch_pool(const cosa_shape_t* s, const cosa_kap_params_t* k, const void* q,
+                          const void* k_pool, const int32_t* page_table, const KapLayout& L,
+                          uint8_t* ws, cudaStream_t st) {
+  const int B = s->batch, Hq = s->num_q_heads, Hk = s->num_kv_heads, N = s->seq_len;
+  const int P = s->page_size, Bq = s->q_block, nP = N / P, nQB = N / Bq;
+  const int R = Bq / k->q_sub, T = P / k->k_sub, G = Hq / Hk;
+  const long long n_qvec = (long long)B * Hq * nQB * R;
+  const long long n_kvec = (long long)B * Hk * nP * T;
+  const long long blocks = (n_qvec + n_kvec + 7) / 8;
+  if (blocks > 0x7fffffffll) return COSA_ERR_UNSUPPORTED;
+  kap_pool_kernel<D><<<(unsigned)blocks, 256, 0, st>>>(
+      reinterpret_cast<const __nv_bfloat16*>(q), reinterpret_cast<const __nv_bfloat16*>(k_pool),
+      page_table, reinterpret_cast<float*>(ws + L.q_hi), reinterpret_cast<float*>(ws + L.q_lo),
+      reinterpret_cast<float*>(ws + L.k_hi), reinterpret_cast<float*>(ws + L.k_lo), n_qvec,
+      k->q_sub, n_kvec, k->k_sub, Hq, Hk, G, R, nQB, P, nP, s->pages_per_seq, T);
+  return last_launch();
+}
+
+// K2 + K3 from the pooled vectors in the workspace
+template <int D>
+cosa_status_t launch_rank(const cosa_shape_t* s, const cosa_kap_params_t* k, int32_t* order,
+                          int32_t* count, float* scores, uint8_t* hrm, const KapLayout& L,
+                          uint8_t* ws, int k_cap, cudaStream_t st, bool group = false) {
   const int B = s->batch, Hq = s->num_q_heads, Hk = s->num_kv_heads, N = s->seq_len;
   const int P = s->page_size, Bq = s->q_block, nP = N / P, nQB = N / Bq;
   const int R = Bq / k->q_sub, T = P / k->k_sub, G = Hq / Hk;
@@ -199,17 +219,8 @@ cosa_status_t launch_kap(const cosa_shape_t* s, const cosa_kap_params_t* k, cons
   float* q_lo = reinterpret_cast<float*>(ws + L.q_lo);
   float* k_hi = reinterpret_cast<float*>(ws + L.k_hi);
   float* k_lo = reinterpret_cast<float*>(ws + L.k_lo);
-
-  // K1: pooling
   const long long n_qvec = (long long)B * Hq * nQB * R;
   const long long n_kvec = (long long)B * Hk * nP * T;
-  const long long blocks = (n_qvec + n_kvec + 7) / 8;
-  if (blocks > 0x7fffffffll) return COSA_ERR_UNSUPPORTED;
-  kap_pool_kernel<D><<<(unsigned)blocks, 256, 0, st>>>(
-      reinterpret_cast<const __nv_bfloat16*>(q), reinterpret_cast<const __nv_bfloat16*>(k_pool),
-      page_table, q_hi, q_lo, k_hi, k_lo, n_qvec, k->q_sub, n_kvec, k->k_sub, Hq, Hk, G, R, nQB,
-      P, nP, s->pages_per_seq, T);
-  if (last_launch() != COSA_OK) return COSA_ERR_CUDA;
 
   // K2: scores + MaxPool on the tensor cores
   ScoreParams sp;
@@ -255,6 +266,15 @@ cosa_status_t launch_kap(const cosa_shape_t* s, const cosa_kap_params_t* k, cons
   pm.R = R;
   return launch_order(s, k, true, nullptr, nullptr, pm, scores, hrm, order, count, k_cap, st,
                       group);
+}
+
+template <int D>
+cosa_status_t launch_kap(const cosa_shape_t* s, const cosa_kap_params_t* k, const void* q,
+                         const void* k_pool, const int32_t* page_table, int32_t* order,
+                         int32_t* count, float* scores, uint8_t* hrm, const KapLayout& L,
+                         uint8_t* ws, int k_cap, cudaStream_t st, bool group = false) {
+  if (launch_pool<D>(s, k, q, k_pool, page_table, L, ws, st) != COSA_OK) return COSA_ERR_CUDA;
+  return launch_rank<D>(s, k, order, count, scores, hrm, L, ws, k_cap, st, group);
 }
 
 template <int D, int P>
@@ -340,8 +360,17 @@ TcParams make_params(const cosa_shape_t* s, void* out, float* lse, const int32_t
   p.log2_eps = -INFINITY;
   p.max_run = 0;
   p.timeout_ns = kWaitTimeoutNs;
+  p.fault_k_group = -1;
   return p;
 }
+
+// Test hook of cosa_debug_osk_wait_fault: one-shot, per host thread.
+struct OskFault {
+  bool armed = false;
+  int32_t k_group = -1;
+  uint64_t wait_limit_ns = 0;
+};
+thread_local OskFault t_osk_fault;
 
 // ---------------------------------------------------------------------------
 // Scratch for cosa_kap_select_noalloc.  Some callers cannot allocate device
@@ -357,19 +386,48 @@ static __device__ __align__(256) uint8_t g_kap_noalloc_scratch[COSA_KAP_NOALLOC_
 constexpr int kMaxDevices = 64;
 std::mutex g_noalloc_mutex;
 void* g_noalloc_addr[kMaxDevices] = {};
+unsigned long long g_noalloc_ctx[kMaxDevices] = {};  // context the address belongs to
 
-// Device address of the scratch array on the current device (looked up on the
-// first call for that device, with that device current).
+// Unique id of the current CUDA context (0 if it cannot be had): after a device
+// reset the library's module loads again in a new context, possibly elsewhere.
+unsigned long long current_context_id() {
+  using CtxGetCurrent = CUresult (*)(CUcontext*);
+  using CtxGetId = CUresult (*)(CUcontext, unsigned long long*);
+  static CtxGetCurrent get_cur = nullptr;
+  static CtxGetId get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_cur = reinterpret_cast<CtxGetCurrent>(p);
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<CtxGetId>(p);
+  });
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (!get_cur || !get_id || get_cur(&ctx) != CUDA_SUCCESS || !ctx || get_id(ctx, &id) != CUDA_SUCCESS)
+    return 0;
+  return id;
+}
+
+// Device address of the scratch array on the current device, looked up with that
+// device current on the first call in each context (a device reset starts a new one;
+// while no context is current yet, the address is looked up on every call).
 cosa_status_t noalloc_scratch_address(void** out) {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess) return COSA_ERR_CUDA;
   if (dev < 0 || dev >= kMaxDevices) return COSA_ERR_UNSUPPORTED;
+  const unsigned long long ctx = current_context_id();
   std::lock_guard<std::mutex> lock(g_noalloc_mutex);
-  if (g_noalloc_addr[dev] == nullptr) {
+  if (g_noalloc_addr[dev] == nullptr || ctx == 0 || g_noalloc_ctx[dev] != ctx) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_kap_noalloc_scratch) != cudaSuccess || p == nullptr)
       return COSA_ERR_CUDA;
     g_noalloc_addr[dev] = p;
+    g_noalloc_ctx[dev] = ctx;
   }
   *out = g_noalloc_addr[dev];
   return COSA_OK;
@@ -510,6 +568,42 @@ cosa_status_t cosa_kap_select(const cosa_shape_t* shape, const cosa_kap_params_t
                         st);
 }
 
+cosa_status_t cosa_kap_pool(const cosa_shape_t* shape, const cosa_kap_params_t* kap,
+                            const void* q, const void* k_pool, const int32_t* page_table,
+                            void* workspace, size_t workspace_bytes, cosa_stream_t stream) {
+  cosa_status_t e = check_shape(shape);
+  if (e != COSA_OK) return e;
+  if ((e = check_kap(shape, kap)) != COSA_OK) return e;
+  if (!q || !k_pool || !page_table) return COSA_ERR_INVALID_ARG;
+  KapLayout L = kap_layout(shape, kap);
+  if (!workspace || workspace_bytes < L.total) return COSA_ERR_WORKSPACE;
+  if (reinterpret_cast<uintptr_t>(workspace) % 256) return COSA_ERR_WORKSPACE;
+  if (reinterpret_cast<uintptr_t>(q) % 16 || reinterpret_cast<uintptr_t>(k_pool) % 16)
+    return COSA_ERR_INVALID_ARG;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* ws = reinterpret_cast<uint8_t*>(workspace);
+  if (shape->head_dim == 128) return launch_pool<128>(shape, kap, q, k_pool, page_table, L, ws, st);
+  return launch_pool<64>(shape, kap, q, k_pool, page_table, L, ws, st);
+}
+
+cosa_status_t cosa_kap_rank(const cosa_shape_t* shape, const cosa_kap_params_t* kap,
+                            int32_t* order, int32_t* count, float* scores, uint8_t* hrm,
+                            void* workspace, size_t workspace_bytes, cosa_stream_t stream) {
+  cosa_status_t e = check_shape(shape);
+  if (e != COSA_OK) return e;
+  if ((e = check_kap(shape, kap)) != COSA_OK) return e;
+  if (!order || !count) return COSA_ERR_INVALID_ARG;
+  KapLayout L = kap_layout(shape, kap);
+  if (!workspace || workspace_bytes < L.total) return COSA_ERR_WORKSPACE;
+  if (reinterpret_cast<uintptr_t>(workspace) % 256) return COSA_ERR_WORKSPACE;
+  const int k_cap = kcap_of(shape, kap);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* ws = reinterpret_cast<uint8_t*>(workspace);
+  if (shape->head_dim == 128)
+    return launch_rank<128>(shape, kap, order, count, scores, hrm, L, ws, k_cap, st);
+  return launch_rank<64>(shape, kap, order, count, scores, hrm, L, ws, k_cap, st);
+}
+
 cosa_status_t cosa_kap_select_group(const cosa_shape_t* shape, const cosa_kap_params_t* kap,
                                     const void* q, const void* k_pool, const int32_t* page_table,
                                     int32_t* order, int32_t* count, float* scores, uint8_t* hrm,
@@ -576,6 +670,8 @@ cosa_status_t cosa_osk_attention(const cosa_shape_t* shape, const cosa_osk_param
                                  const int32_t* page_table, const int32_t* order,
                                  const int32_t* count, int32_t k_cap, void* out, float* lse,
                                  int32_t* computed, uint8_t* skip_log, cosa_stream_t stream) {
+  const OskFault fault = t_osk_fault;  // the test hook is consumed by this call, whatever it returns
+  t_osk_fault = OskFault();
   cosa_status_t e = check_shape(shape);
   if (e != COSA_OK) return e;
   if (!osk || !(osk->eps >= 0.f) || osk->max_run < 0) return COSA_ERR_INVALID_ARG;
@@ -595,6 +691,11 @@ cosa_status_t cosa_osk_attention(const cosa_shape_t* shape, const cosa_osk_param
   p.max_run = osk->max_run;
   const long long grid = (long long)shape->batch * shape->num_q_heads * (shape->seq_len / shape->q_block);
   if (grid > 0x7fffffffll) return COSA_ERR_UNSUPPORTED;
+  if (fault.armed) {
+    if (osk->max_run != 0) return COSA_ERR_INVALID_ARG;
+    p.fault_k_group = fault.k_group;
+    if (fault.wait_limit_ns) p.timeout_ns = fault.wait_limit_ns;
+  }
   return launch_osk(shape, p, q, k_pool, v_pool, (int)grid, reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -654,6 +755,14 @@ cosa_status_t cosa_dense_attention(const cosa_shape_t* shape, const void* q, con
   if (D == 64 && P == 64) return launch_dense_t<64, 64>(shape, p, q, k_pool, v_pool, (int)grid, st);
   if (D == 64 && P == 128) return launch_dense_t<64, 128>(shape, p, q, k_pool, v_pool, (int)grid, st);
   return COSA_ERR_UNSUPPORTED;
+}
+
+cosa_status_t cosa_debug_osk_wait_fault(int32_t withhold_k_group, uint64_t wait_limit_ns) {
+  if (withhold_k_group < -1) return COSA_ERR_INVALID_ARG;
+  t_osk_fault.armed = true;
+  t_osk_fault.k_group = withhold_k_group;
+  t_osk_fault.wait_limit_ns = wait_limit_ns;
+  return COSA_OK;
 }
 
 cosa_status_t cosa_get_status(cosa_stream_t stream) {

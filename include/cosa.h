@@ -146,6 +146,28 @@ cosa_status_t cosa_kap_select(const cosa_shape_t* shape, const cosa_kap_params_t
                               int32_t* order, int32_t* count, float* scores, uint8_t* hrm,
                               void* workspace, size_t workspace_bytes, cosa_stream_t stream);
 
+/* Stage 1 in two launches, for callers that time or schedule the steps apart;
+ * cosa_kap_pool followed by cosa_kap_rank on the same workspace is
+ * cosa_kap_select (same kernels, same results).
+ *
+ * cosa_kap_pool: the downsampling step alone (gist.science/pt §2.2 "Ranking de
+ * Blocos": downsampling of queries and keys): q^ and k^ as above, written to the
+ * workspace (at least cosa_kap_workspace_size bytes, 256-byte aligned) as two
+ * TF32 terms each.  Reads Q and the K pages once: the step is bound by HBM
+ * bandwidth. */
+cosa_status_t cosa_kap_pool(const cosa_shape_t* shape, const cosa_kap_params_t* kap,
+                            const void* q, const void* k_pool, const int32_t* page_table,
+                            void* workspace, size_t workspace_bytes, cosa_stream_t stream);
+
+/* cosa_kap_rank: the remaining Stage-1 steps (approximate scores, MaxPool over
+ * keys, MaxNorm, HRM flags, budgeted selection and flag-group ordering;
+ * gist.science/pt §2.2) from the pooled vectors that cosa_kap_pool left in the
+ * workspace for the same shape and parameters (stream order: queue it after
+ * that call).  order, count, scores and hrm as for cosa_kap_select. */
+cosa_status_t cosa_kap_rank(const cosa_shape_t* shape, const cosa_kap_params_t* kap,
+                            int32_t* order, int32_t* count, float* scores, uint8_t* hrm,
+                            void* workspace, size_t workspace_bytes, cosa_stream_t stream);
+
 /* Stage 1 with one list per KV head: the G query heads that read KV head h_kv
  * share one ordered list per q-block (the group-shared selection; the pages
  * describe per-head selection only, this is the next step after it).  Every
@@ -178,7 +200,9 @@ cosa_status_t cosa_kap_select_group(const cosa_shape_t* shape, const cosa_kap_pa
  *   - Shapes whose cosa_kap_workspace_size exceeds COSA_KAP_NOALLOC_SCRATCH_BYTES
  *     return COSA_ERR_UNSUPPORTED before anything is launched.
  *   - The first call on a device looks up the array's device address (with that
- *     device current); make that first call before any stream capture.
+ *     device current); make that first call before any stream capture.  The
+ *     address is cached per CUDA context: after a device reset (a new context) the
+ *     next call looks it up again, and that call too belongs before any capture.
  *   - Allocates nothing: no cudaMalloc, no cudaFree, no allocating library call.
  *   - All calls on a device share the one array, and it keeps the last call's
  *     contents (every kernel writes what it later reads, so nothing needs
@@ -261,6 +285,24 @@ cosa_status_t cosa_attention_host(const cosa_shape_t* shape, const cosa_kap_para
                                   const void* k_pool_host, const void* v_pool_host,
                                   const int32_t* page_table_host, void* out_host, void* workspace,
                                   size_t workspace_bytes, cosa_stream_t stream);
+
+/* Test hook, not part of the method (the pages describe no failure handling): it
+ * lets a test make one of the attention kernel's bounded waits run out on purpose
+ * and check that the failure is reported and leaves the device usable.  The next
+ * cosa_osk_attention call made from this host thread (and only that call: the
+ * setting is consumed by it, whatever it returns) runs with
+ *   - every bounded wait limited to wait_limit_ns of no progress (0 keeps the
+ *     default of one second), and
+ *   - when withhold_k_group >= 0, the K tile copies of that listed group (list
+ *     entries 2g and 2g+1 for 64-token pages, entry g for 128-token pages) never
+ *     issued in any q-block whose list reaches it, so the waits for it run out.
+ * The kernel then records COSA_ERR_TIMEOUT in the status word, waits (bounded)
+ * for the copies and MMAs it did issue, frees its tensor memory and returns; the
+ * other CTAs of the launch stop early.  That call's outputs are undefined; the
+ * following calls run normally.  That call must have max_run = 0
+ * (COSA_ERR_INVALID_ARG otherwise).  withhold_k_group < -1: COSA_ERR_INVALID_ARG.
+ * Host-only; no CUDA call. */
+cosa_status_t cosa_debug_osk_wait_fault(int32_t withhold_k_group, uint64_t wait_limit_ns);
 
 /* Read (and clear) the current device's status word: COSA_OK, or the first
  * in-kernel error recorded since the last call (e.g. COSA_ERR_TIMEOUT).
