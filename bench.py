@@ -442,6 +442,9 @@ def main():
     ap.add_argument("--shard", default="kv-heads", choices=["kv-heads", "replica"],
                     help="N > 1: split one layer's KV heads over the GPUs (strong scaling), "
                          "or run an independent layer on each (weak scaling)")
+    ap.add_argument("--kv-heads", type=int, default=0,
+                    help="run only the first K KV heads of the layer (a smaller case of the "
+                         "same layer, for profiling; one GPU)")
     ap.add_argument("--no-extras", action="store_true", help="skip dense/sweep/e2e/cpu legs")
     ap.add_argument("--sweep-only", action="store_true",
                     help="run only the per-budget sweep and print it")
@@ -485,7 +488,14 @@ def main():
     wl = W.WORKLOADS[args.workload]
     B, N, D = wl.batch, wl.seq_len, wl.head_dim
     G = wl.num_q_heads // wl.num_kv_heads
-    if args.shard == "kv-heads":
+    if args.kv_heads > 0:
+        if world > 1 or args.kv_heads > wl.num_kv_heads:
+            raise SystemExit("--kv-heads: one GPU, at most the layer's KV heads")
+        h0, h1 = 0, args.kv_heads
+        x = shard_inputs(W.make_inputs(wl, seed=0, device=str(dev)), wl.num_q_heads,
+                         wl.num_kv_heads, h0, h1)
+        torch.cuda.empty_cache()
+    elif args.shard == "kv-heads":
         # every rank draws the same layer and keeps its KV heads' share
         h0, h1 = kv_head_shard(rank, world, wl.num_kv_heads)
         x = shard_inputs(W.make_inputs(wl, seed=0, device=str(dev)), wl.num_q_heads,
@@ -507,6 +517,8 @@ def main():
     out = torch.empty(B, Hq, N, D, dtype=torch.bfloat16, device=dev)
     computed = torch.empty(B, Hq, shape.num_q_blocks, dtype=torch.int32, device=dev)
     dense_flop = wl.dense_flops()  # of one whole layer
+    if args.kv_heads > 0:
+        dense_flop *= Hk / wl.num_kv_heads
 
     def job_value(ms):
         if args.shard == "kv-heads":
@@ -625,6 +637,8 @@ def main():
     }
     if world > 1:
         line["shard"] = {"rank0_kv_heads": [h0, h1], "kv_heads_per_rank": Hk}
+    if args.kv_heads > 0:
+        line["config"]["kv_heads_run"] = [h0, h1]
 
     # ---- end to end through the C-ABI with host buffers (every rank, every N) ---
     def e2e_leg():

@@ -43,6 +43,7 @@ __all__ = [
     "kap_maxnorm_hrm", "rank_key", "kap_order_from_scores", "kap_select_block",
     "kap_select", "kap_order", "osk_block", "osk_block_rules", "osk_attention", "dense_rows",
     "dense_attention", "kap_group_scores", "kap_select_group", "expand_group_order",
+    "kap_preskip", "kap_preskip_lists",
 ]
 
 NEG_INF = -math.inf
@@ -358,6 +359,85 @@ def expand_group_order(order_g: np.ndarray, count_g: np.ndarray, num_q_heads: in
     G = num_q_heads // Hkv
     hk = np.arange(num_q_heads) // G
     return order_g[:, hk], count_g[:, hk]
+
+
+# ----------------------------------------------------------------------------
+# Proxy-bound pre-skip: a variant the pages do not give (off unless asked).
+# The pages' in-kernel rule ([TS §2.3] "Saltado no Kernel") compares a page's
+# exact local max with the exact running max, so every listed page still costs
+# its K load and QK^T.  This variant applies the same kind of test one stage
+# earlier, on the proxy's page maxima a[r][p] (kap_block_scores) and the proxy's
+# own running max along the ordered list, and removes the pages it rejects from
+# the list, so the kernel never visits them.  Reading (the plainest one the
+# spec example allows): along the list L = (p_0, p_1, ...),
+#   ahat_r(j) = max over positions j' < j of a[r][p_j'];
+#   representative r keeps position j iff a[r][p_j] > -inf and (ahat_r(j) = -inf
+#     or a[r][p_j] + margin - ahat_r(j) >= ln(eps));
+#   position j >= 1 is pre-skipped iff no representative keeps it; position 0
+#   is always kept; eps = 0 pre-skips nothing.
+# The surviving pages keep their order and go to the kernel's own rule.  The
+# margin (>= 0, in nats) is slack for the proxy's error: pooled scores are
+# estimates of a page's logits, not bounds on them, so the quality of the
+# pages this removes is measured against the full rule, not guaranteed.
+# ----------------------------------------------------------------------------
+def kap_preskip(order: Sequence[int], a: np.ndarray, eps: float, margin: float):
+    """Pre-skip along one q-block's ordered list.  order: logical page ids;
+    a [R][n_b]: the block's proxy page maxima.  Returns (kept int32 list,
+    skipped uint8 [len(order)], margin float64 [len(order)] = max over the
+    representatives that see the page of (a + margin - ahat) minus ln(eps),
+    +inf where a representative that sees the page has ahat = -inf, NaN at
+    position 0)."""
+    a = np.asarray(a, dtype=np.float64)
+    R = a.shape[0]
+    n = len(order)
+    log_eps = math.log(eps) if eps > 0 else NEG_INF
+    ahat = np.full(R, NEG_INF)
+    skipped = np.zeros(n, dtype=np.uint8)
+    tested = np.full(n, np.nan)
+    kept = []
+    for j, p in enumerate(order):
+        col = a[:, int(p)]
+        if j > 0:
+            best = NEG_INF
+            for r in range(R):
+                if col[r] == NEG_INF:
+                    continue                    # this representative sees no key of p
+                if ahat[r] == NEG_INF:
+                    best = math.inf             # its first visible page: kept
+                else:
+                    best = max(best, col[r] + margin - ahat[r])
+            tested[j] = best - log_eps if log_eps > NEG_INF else math.inf
+            if log_eps > NEG_INF and best < log_eps:
+                skipped[j] = 1
+        if not skipped[j]:
+            kept.append(int(p))
+        ahat = np.maximum(ahat, col)
+    return np.asarray(kept, dtype=np.int32), skipped, tested
+
+
+def kap_preskip_lists(order: np.ndarray, count: np.ndarray, a_of, eps: float, margin: float,
+                      tiles: Optional[Sequence] = None):
+    """kap_preskip over whole lists [B][H][nQB][k_cap] / counts [B][H][nQB].
+    a_of(b, h, qb) gives that block's a [R][n_b].  Returns dict with order
+    (survivors first, -1 padded), count, skipped uint8 [B][H][nQB][k_cap] (at the
+    original list positions) and margin float64 (same layout, NaN past count).
+    Tiles not requested keep their list (skipped 0, margin NaN)."""
+    B, H, nQB, kc = order.shape
+    out_o = order.copy()
+    out_c = count.copy()
+    skipped = np.zeros(order.shape, dtype=np.uint8)
+    tested = np.full(order.shape, np.nan)
+    if tiles is None:
+        tiles = [(b, h, qb) for b in range(B) for h in range(H) for qb in range(nQB)]
+    for (b, h, qb) in tiles:
+        n = int(count[b, h, qb])
+        kept, sk, mg = kap_preskip(order[b, h, qb, :n], a_of(b, h, qb), eps, margin)
+        out_o[b, h, qb, :] = -1
+        out_o[b, h, qb, :len(kept)] = kept
+        out_c[b, h, qb] = len(kept)
+        skipped[b, h, qb, :n] = sk
+        tested[b, h, qb, :n] = mg
+    return {"order": out_o, "count": out_c, "skipped": skipped, "margin": tested}
 
 
 # ----------------------------------------------------------------------------
