@@ -611,7 +611,7 @@ def main():
         "higher_is_better": True, "scaling": "strong" if args.shard == "kv-heads" else "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": _config(wl, args.budget, args.eps, args.shard, world),
-        "gpu_launches": 4 * args.steps,
+        "gpu_launches": 4 * args.steps,  # pool, score, order, OSK per step
         "clocks": clk,
         "roofline": {"kernel": "osk_attention", "bound": "tensor", "achieved": achieved,
                      "peak": peak_tflops, "unit": "TFLOP/s", "frac": achieved / peak_tflops,
@@ -785,6 +785,60 @@ def main():
         line["early_break"] = early_break_leg()
     except Exception as exc:  # an extra leg: report the failure, keep the line
         line["early_break"] = {"error": repr(exc)}
+
+    # ---- proxy-bound pre-skip (not part of the pages' method): KAP, the pre-skip
+    # filter, then the pages' rule on the survivors; output against the pages' rule on
+    # the full lists (in `out`) and against dense
+    def preskip_leg():
+        po, pc = torch.empty_like(order), torch.empty_like(count)
+        pout, pcomp = torch.empty_like(out), torch.empty_like(computed)
+        pref = out.float()
+        res = []
+        for eps_pre, margin in ((1e-4, 0.0), (1e-4, 2.0), (1e-4, 4.0), (1e-3, 4.0), (1e-2, 0.0)):
+            ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+
+            def run(rec):
+                if rec:
+                    ev[0].record(stream)
+                C.cosa_kap_select(shape, kap, x["q"], x["k_pool"], x["page_table"], po, pc, ws,
+                                  stream=stream)
+                if rec:
+                    ev[1].record(stream)
+                C.cosa_kap_preskip(shape, kap, eps_pre, margin, po, pc, ws, stream=stream)
+                if rec:
+                    ev[2].record(stream)
+                C.cosa_osk_attention(shape, osk, x["q"], x["k_pool"], x["v_pool"], x["page_table"],
+                                     po, pc, pout, computed=pcomp, stream=stream)
+                if rec:
+                    ev[3].record(stream)
+
+            run(False)
+            tms = [0.0, 0.0, 0.0]
+            for _ in range(3):
+                run(True)
+                ev[3].synchronize()
+                for i in range(3):
+                    tms[i] += ev[i].elapsed_time(ev[i + 1]) / 3
+            if C.cosa_get_status(stream) != 0:
+                raise RuntimeError("in-kernel error status")
+            vis = int(pc.to(torch.int64).sum().item())
+            comp = int(pcomp.to(torch.int64).sum().item())
+            fl = tile * (vis + comp)
+            tot = sum(tms)
+            res.append({"eps_pre": eps_pre, "margin": margin, "eps": args.eps,
+                        "kap_ms": tms[0], "preskip_ms": tms[1], "osk_ms": tms[2], "ms": tot,
+                        "tflops": dense_flop / (tot * 1e-3) / 1e12,
+                        "speedup_vs_dense": dense_ms / tot,
+                        "visited_frac": vis / n_b_total, "computed_frac": comp / n_b_total,
+                        "visited_tflops": fl / (tms[2] * 1e-3) / 1e12,
+                        "rel_l2_vs_pages_rule": float((pout.float() - pref).norm() / pref.norm()),
+                        "rel_l2_vs_dense": rel_l2(pout)})
+        return res
+
+    try:
+        line["preskip"] = preskip_leg()
+    except Exception as exc:  # an extra leg: report the failure, keep the line
+        line["preskip"] = {"error": repr(exc)}
 
     line["e2e"] = e2e_leg()
     del dense_out, dref, outg

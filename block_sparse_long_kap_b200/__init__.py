@@ -21,6 +21,7 @@ __all__ = [
     "cosa_dense_attention", "cosa_get_status", "EXPORTED_SYMBOLS", "NOALLOC_SCRATCH_BYTES",
     "cosa_kap_select_group", "cosa_osk_attention_group", "cosa_attention_host_workspace_size",
     "cosa_attention_host", "cosa_debug_osk_wait_fault", "cosa_kap_pool", "cosa_kap_rank",
+    "cosa_kap_preskip",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -31,7 +32,7 @@ EXPORTED_SYMBOLS = (
     "cosa_kap_select", "cosa_kap_select_noalloc", "cosa_kap_order", "cosa_osk_attention",
     "cosa_dense_attention", "cosa_get_status", "cosa_kap_select_group", "cosa_osk_attention_group",
     "cosa_attention_host_workspace_size", "cosa_attention_host", "cosa_debug_osk_wait_fault",
-    "cosa_kap_pool", "cosa_kap_rank",
+    "cosa_kap_pool", "cosa_kap_rank", "cosa_kap_preskip",
 )
 
 # Largest workspace the allocation-free Stage-1 entry point accepts (cosa.h).
@@ -155,6 +156,8 @@ def lib():
     L.cosa_debug_osk_wait_fault.argtypes = [i32, ctypes.c_uint64]
     L.cosa_kap_pool.argtypes = [P(_Shape), P(_Kap), vp, vp, vp, vp, sz, vp]
     L.cosa_kap_rank.argtypes = [P(_Shape), P(_Kap), vp, vp, vp, vp, vp, sz, vp]
+    L.cosa_kap_preskip.argtypes = [P(_Shape), P(_Kap), ctypes.c_float, ctypes.c_float, vp, vp, vp,
+                                   vp, sz, vp]
     for name in EXPORTED_SYMBOLS:
         if name not in ("cosa_status_string", "cosa_version"):
             getattr(L, name).restype = ctypes.c_int
@@ -282,6 +285,26 @@ def cosa_kap_rank(shape: Shape, kap: KapParams, order, count, workspace, scores=
     _check(lib().cosa_kap_rank(ctypes.byref(s), ctypes.byref(k), _ptr(order), _ptr(count),
                                _ptr(scores), _ptr(hrm), _ptr(workspace), nbytes, _stream(stream)),
            "cosa_kap_rank")
+
+
+def cosa_kap_preskip(shape: Shape, kap: KapParams, eps: float, margin: float, order, count,
+                     workspace, skip_log=None, stream=None) -> None:
+    """Proxy-bound pre-skip (not the pages' rule): filter the lists cosa_kap_select just
+    wrote with this workspace, in place; skip_log gets 1 at the removed positions."""
+    import torch
+    s, k = shape.c(), kap.c(shape)
+    B, Hq = shape.batch, shape.num_q_heads
+    kc = cosa_kap_kcap(shape, kap)
+    _expect(order, "order", torch.int32, (B, Hq, shape.num_q_blocks, kc))
+    _expect(count, "count", torch.int32, (B, Hq, shape.num_q_blocks))
+    if skip_log is not None:
+        _expect(skip_log, "skip_log", torch.uint8, (B, Hq, shape.num_q_blocks, kc))
+    if workspace is None or not workspace.is_cuda:
+        raise ValueError("workspace must be a CUDA tensor")
+    nbytes = workspace.numel() * workspace.element_size()
+    _check(lib().cosa_kap_preskip(ctypes.byref(s), ctypes.byref(k), float(eps), float(margin),
+                                  _ptr(order), _ptr(count), _ptr(skip_log), _ptr(workspace),
+                                  nbytes, _stream(stream)), "cosa_kap_preskip")
 
 
 def cosa_kap_select_group(shape: Shape, kap: KapParams, q, k_pool, page_table, order, count,

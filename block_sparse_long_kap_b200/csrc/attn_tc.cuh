@@ -550,15 +550,36 @@ __global__ void __launch_bounds__(TcCfg<D, P>::NT, 1)
     float m_run = -INFINITY, m_ref = -INFINITY, l = 0.f;  // l: this warpgroup's share, base m_ref
     bool ok = true;     // OSK: collective within the warpgroup
     bool fail = false;  // this warp missed a wait after the vote; reported at the next vote
-    int fb = -1, pid_l = 0, cz_l = 0;
+    // Page ids of list entries [fb, fb + 32) (lane l: entry fb + l) in pid_l and, in the
+    // leading warp, their TMA coordinates in cz_l.  The next block's ids and coordinates
+    // (pid_1, cz_1) and the ids of the block after it (pid_2) are loaded ahead, so that
+    // moving on to a new block waits on no global load.
+    int fb = -1, pid_l = 0, cz_l = 0, pid_1 = 0, cz_1 = 0, pid_2 = 0;
+    auto ids_of = [&](int base) {
+      const int jl = base + lane;
+      return jl < n_list ? page_at(jl) : 0;
+    };
+    auto coords_of = [&](int base, int pid) {
+      const int jl = base + lane;
+      return (lead_warp && jl < n_list) ? coord_of(pid) : 0;
+    };
     // page id (and, in the leading warp, TMA coordinate) of list entry j; j only grows
     auto fetch = [&](int j, int& cz) -> int {
       const int base = j & ~31;
       if (base != fb) {
+        if (base == fb + 32) {  // the block loaded ahead
+          pid_l = pid_1;
+          cz_l = cz_1;
+          pid_1 = pid_2;
+          cz_1 = coords_of(base + 32, pid_1);
+        } else {  // first block: loaded here
+          pid_l = ids_of(base);
+          cz_l = coords_of(base, pid_l);
+          pid_1 = ids_of(base + 32);
+          cz_1 = coords_of(base + 32, pid_1);
+        }
+        pid_2 = ids_of(base + 64);
         fb = base;
-        const int jl = base + lane;
-        pid_l = jl < n_list ? page_at(jl) : 0;
-        if (lead_warp) cz_l = jl < n_list ? coord_of(pid_l) : 0;
       }
       cz = __shfl_sync(0xffffffffu, cz_l, j & 31);
       return __shfl_sync(0xffffffffu, pid_l, j & 31);
@@ -577,22 +598,27 @@ __global__ void __launch_bounds__(TcCfg<D, P>::NT, 1)
           for (int e = 0; e < 64; ++e)
             if (k0 + e > grow) v[e] = __float_as_uint(-INFINITY);
         }
+        // 64 values to one with three-input maxima: eight running maxima take two
+        // values at a time, then one more each, then three steps combine them
         float a[8];
 #pragma unroll
-        for (int e = 0; e < 64; ++e)
-          a[e & 7] = e < 8 ? __uint_as_float(v[e]) : fmaxf(a[e & 7], __uint_as_float(v[e]));
+        for (int e = 0; e < 8; ++e) a[e] = __uint_as_float(v[e]);
 #pragma unroll
-        for (int w = 4; w > 0; w >>= 1)
+        for (int r = 8; r + 16 <= 64; r += 16)
 #pragma unroll
-          for (int e = 0; e < w; ++e) a[e] = fmaxf(a[e], a[e + w]);
-        mx = fmaxf(mx, a[0]);
+          for (int e = 0; e < 8; ++e)
+            a[e] = fmax3f(a[e], __uint_as_float(v[r + e]), __uint_as_float(v[r + 8 + e]));
+#pragma unroll
+        for (int e = 0; e < 8; ++e) a[e] = fmaxf(a[e], __uint_as_float(v[56 + e]));
+        mx = fmax3f(mx, fmax3f(a[0], a[1], a[2]), fmax3f(a[3], a[4], a[5]));
+        mx = fmax3f(mx, a[6], a[7]);
       }
       return mx;
     };
     // leader: publish kept page c to the queue: its TMA coordinate (for the V
     // load), then its P column and last-of-group flag (for the PV issue)
     auto bounded_until = [&](volatile int* pos, int c) {
-      if (c < C::KQ) return;
+      if (c < C::KQ || *pos > c - C::KQ) return;
       const uint64_t t0 = globaltimer_ns();
       while (*pos <= c - C::KQ) {  // the entry's previous use has been read
         if (*abort_flag || timed_out(t0)) { give_up(); break; }
@@ -604,12 +630,6 @@ __global__ void __launch_bounds__(TcCfg<D, P>::NT, 1)
       kq[c % C::KQ].x = cz;
       __threadfence_block();
       *vq_count = c + 1;
-    };
-    auto publish_info = [&](int c, int info) {
-      bounded_until(pv_pos, c);
-      kq[c % C::KQ].y = info;
-      __threadfence_block();
-      *kq_count = c + 1;
     };
     uint8_t* slog = prm.skip_log ? prm.skip_log + (bh * prm.num_q_blocks + qb) * prm.k_cap
                                              : nullptr;
@@ -753,15 +773,14 @@ __global__ void __launch_bounds__(TcCfg<D, P>::NT, 1)
       // page 1 kept (4), page 2 after page 1 skipped (8)
       auto vote_bits = [&](float m) -> uint32_t {
         const bool n0 = lv[0] && (m == -INFINITY || mloc[0] - m >= le);
-        uint32_t bits = __any_sync(0xffffffffu, n0) ? 2u : 0u;
+        uint32_t bits = n0 ? 2u : 0u;
         if (GP == 2 && nb == 2) {
           const float mk = fmaxf(m, mloc[0]);
           const bool nk = lv[GP - 1] && (mk == -INFINITY || mloc[GP - 1] - mk >= le);
           const bool ns = lv[GP - 1] && (m == -INFINITY || mloc[GP - 1] - m >= le);
-          bits |= __any_sync(0xffffffffu, nk) ? 4u : 0u;
-          bits |= __any_sync(0xffffffffu, ns) ? 8u : 0u;
+          bits |= (nk ? 4u : 0u) | (ns ? 8u : 0u);
         }
-        return bits;
+        return __reduce_or_sync(0xffffffffu, bits);  // the warp's votes
       };
       {
         const bool exact = j == 0;  // the first listed page is always kept
@@ -789,7 +808,10 @@ __global__ void __launch_bounds__(TcCfg<D, P>::NT, 1)
               }
             }
           }
-          mark_settled(g);
+          // a skipped group writes no state rows or queue entries: nothing to order
+          // before its settled mark (the last exact group's writes were fenced)
+          __syncwarp();
+          if (lane == 0) settled[wg * 4 + q4] = g;
           continue;
         }
       }
@@ -839,8 +861,10 @@ __global__ void __launch_bounds__(TcCfg<D, P>::NT, 1)
           const float m_new = fmaxf(m_run, mloc[t]);
           m_run = m_new;
           const bool resc = (m_ref != -INFINITY) && (m_new > m_ref + kRescaleLog2);
-          alpha[t] = resc ? ex2_approx(m_ref - m_new) : 1.f;
           rany[t] = __any_sync(0xffffffffu, resc);
+          // (the exponential only in the rare warp that rescales: the special-function
+          // unit is busy with the other warpgroup's P)
+          if (rany[t] && resc) alpha[t] = ex2_approx(m_ref - m_new);
           if (m_new != -INFINITY && (m_ref == -INFINITY || resc)) m_ref = m_new;
           mb[t] = m_ref;
           ++nk;
@@ -853,16 +877,29 @@ __global__ void __launch_bounds__(TcCfg<D, P>::NT, 1)
       }
       if (leader) {
         int c = c0;
+        bool new_v = false;
 #pragma unroll
         for (int t = 0; t < GP; ++t)
           if (t < nb) {
             if (slog) slog[j + t] = keep[t] ? 0 : 1;
             if (keep[t]) {
-              if (j + t > 0) publish_v(c, czp[t]);
-              publish_info(c, (sb * 128 + t * P) | ((t == lastk ? 1 : 0) << 15) | (wg << 16));
+              // the entry's coordinate (for the V load; page 0's went out before any
+              // vote) and P location (for the PV issue), once its previous use is read
+              if (j + t > 0) {
+                bounded_until(v_pos, c);
+                kq[c % C::KQ].x = czp[t];
+                new_v = true;
+              }
+              bounded_until(pv_pos, c);
+              kq[c % C::KQ].y = (sb * 128 + t * P) | ((t == lastk ? 1 : 0) << 15) | (wg << 16);
               ++c;
             }
           }
+        if (c > c0) {  // entries before counts
+          __threadfence_block();
+          if (new_v) *vq_count = c;
+          *kq_count = c;
+        }
         if (nk == 0) mbar_arrive(b_sfree(sb, wg ^ 1));  // nothing kept: the S buffer goes back now
         if (R > 0 && oks) {  // early break: the last kept page, and whether the rest is past it
           const int kl2 = nk > 0 ? j + lastk : kl;

@@ -604,6 +604,39 @@ cosa_status_t cosa_kap_rank(const cosa_shape_t* shape, const cosa_kap_params_t* 
   return launch_rank<64>(shape, kap, order, count, scores, hrm, L, ws, k_cap, st);
 }
 
+cosa_status_t cosa_kap_preskip(const cosa_shape_t* shape, const cosa_kap_params_t* kap,
+                               float eps, float margin, int32_t* order, int32_t* count,
+                               uint8_t* skip_log, const void* workspace, size_t workspace_bytes,
+                               cosa_stream_t stream) {
+  cosa_status_t e = check_shape(shape);
+  if (e != COSA_OK) return e;
+  if ((e = check_kap(shape, kap)) != COSA_OK) return e;
+  if (!(eps >= 0.f) || !(margin >= 0.f) || !std::isfinite(margin)) return COSA_ERR_INVALID_ARG;
+  if (!order || !count) return COSA_ERR_INVALID_ARG;
+  KapLayout L = kap_layout(shape, kap);
+  if (!workspace || workspace_bytes < L.total) return COSA_ERR_WORKSPACE;
+  if (reinterpret_cast<uintptr_t>(workspace) % 256) return COSA_ERR_WORKSPACE;
+  const int k_cap = kcap_of(shape, kap);
+  if (k_cap > PRESKIP_THREADS * 32) return COSA_ERR_UNSUPPORTED;  // 32 positions per thread
+  const int nQB = shape->seq_len / shape->q_block;
+  const long long rows = (long long)shape->batch * shape->num_q_heads;
+  if (rows > 65535) return COSA_ERR_UNSUPPORTED;
+  const uint8_t* ws = reinterpret_cast<const uint8_t*>(workspace);
+  KapPageMax pm;
+  std::memset(&pm, 0, sizeof(pm));
+  pm.a = reinterpret_cast<const float*>(ws + L.a);
+  pm.num_kv_heads = shape->num_kv_heads;
+  pm.group = shape->num_q_heads / shape->num_kv_heads;
+  pm.R = shape->q_block / kap->q_sub;
+  const float log_eps = eps > 0.f ? logf(eps) : -INFINITY;
+  dim3 grid(nQB, (unsigned)rows);
+  kap_preskip_kernel<<<grid, PRESKIP_THREADS, (size_t)k_cap * sizeof(int),
+                       reinterpret_cast<cudaStream_t>(stream)>>>(
+      pm, order, count, skip_log, shape->num_q_heads, nQB, shape->q_block, shape->page_size,
+      k_cap, log_eps, margin);
+  return last_launch();
+}
+
 cosa_status_t cosa_kap_select_group(const cosa_shape_t* shape, const cosa_kap_params_t* kap,
                                     const void* q, const void* k_pool, const int32_t* page_table,
                                     int32_t* order, int32_t* count, float* scores, uint8_t* hrm,

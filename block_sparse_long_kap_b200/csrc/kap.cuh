@@ -401,4 +401,121 @@ __global__ void __launch_bounds__(ORDER_THREADS) kap_order_kernel(
   }
 }
 
+// ---------------------------------------------------------------------------
+// Proxy-bound pre-skip (a variant the pages do not give; off unless asked).  The
+// pages' in-kernel skip (gist.science/pt §2.3 "Saltado no Kernel") still costs every
+// listed page its K load and QK^T.  This filter applies the same kind of test one
+// stage earlier, on the proxy's page maxima a[r][p] and the proxy's own running max
+// along the ordered list, and removes the pages it rejects before the kernel runs:
+//   ahat_r(j) = max over list positions j' < j of a[r][p_j'];
+//   representative r keeps position j iff a[r][p_j] > -inf and (ahat_r(j) = -inf
+//     or (a[r][p_j] + margin) - ahat_r(j) >= ln eps);
+//   position j >= 1 is removed iff no representative keeps it.
+// One CTA per (b, h_q, q-block): the list is read into shared memory, each thread
+// takes a contiguous run of positions, the runs' maxima are scanned per
+// representative (one warp per representative), each thread then walks its run,
+// and the survivors are written back in list order (-1 after them).
+// ---------------------------------------------------------------------------
+constexpr int PRESKIP_THREADS = 256;
+constexpr int PRESKIP_MAX_R = 8;
+
+__global__ void __launch_bounds__(PRESKIP_THREADS) kap_preskip_kernel(
+    KapPageMax pm, int32_t* __restrict__ order, int32_t* __restrict__ count,
+    uint8_t* __restrict__ skip_log, int num_q_heads, int num_q_blocks, int q_block,
+    int page_size, int k_cap, float log_eps, float margin) {
+  extern __shared__ int lst[];  // [k_cap] the list, as read
+  __shared__ float run_max[PRESKIP_THREADS][PRESKIP_MAX_R];  // per run, then exclusive scan
+  __shared__ int warp_sums[32];
+  const int qb = blockIdx.x, bhq = blockIdx.y;
+  const long long row = (long long)bhq * num_q_blocks + qb;
+  const int n_b = causal_pages(qb, q_block, page_size);
+  const int R = pm.R;
+  const int b = bhq / num_q_heads, h = bhq % num_q_heads;
+  const int hk = h / pm.group, g = h % pm.group;
+  const int GR = pm.group * R;
+  const long long slab = (long long)b * pm.num_kv_heads + hk;
+  const float* arow = pm.a + slab * GR * cum_pages(num_q_blocks, q_block, page_size) +
+                      (long long)GR * cum_pages(qb, q_block, page_size) + (long long)g * R * n_b;
+  int32_t* orow = order + row * k_cap;
+  const int n = min(max(count[row], 0), k_cap);
+  for (int j = threadIdx.x; j < n; j += blockDim.x) {
+    const int p = orow[j];
+    lst[j] = (p >= 0 && p < n_b) ? p : -1;  // out-of-range ids are flagged below
+  }
+  __syncthreads();
+  const int per = (n + blockDim.x - 1) / blockDim.x;
+  const int j0 = min(n, (int)threadIdx.x * per), j1 = min(n, j0 + per);
+  int bad = 0;
+  float rm[PRESKIP_MAX_R];
+#pragma unroll
+  for (int r = 0; r < PRESKIP_MAX_R; ++r) rm[r] = -INFINITY;
+  for (int j = j0; j < j1; ++j) {
+    const int p = lst[j];
+    if (p < 0) { bad = 1; continue; }
+#pragma unroll
+    for (int r = 0; r < PRESKIP_MAX_R; ++r)
+      if (r < R) rm[r] = fmaxf(rm[r], __ldg(arow + (long long)r * n_b + p));
+  }
+#pragma unroll
+  for (int r = 0; r < PRESKIP_MAX_R; ++r) run_max[threadIdx.x][r] = rm[r];
+  if (__syncthreads_or(bad)) {  // not a list of this block's causal pages: left as is
+    if (threadIdx.x == 0) set_status(COSA_ERR_INVALID_ARG);
+    return;
+  }
+  // exclusive max-scan of the runs' maxima, warp r for representative r
+  {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    constexpr int PL = PRESKIP_THREADS / 32;  // runs per lane
+    if (warp < R) {
+      float loc = -INFINITY;
+#pragma unroll
+      for (int i = 0; i < PL; ++i) loc = fmaxf(loc, run_max[lane * PL + i][warp]);
+      float inc = loc;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const float y = __shfl_up_sync(0xffffffffu, inc, o);
+        if (lane >= o) inc = fmaxf(inc, y);
+      }
+      float run = __shfl_up_sync(0xffffffffu, inc, 1);  // max over the lanes before
+      if (lane == 0) run = -INFINITY;
+      __syncwarp();
+#pragma unroll
+      for (int i = 0; i < PL; ++i) {
+        const float v = run_max[lane * PL + i][warp];
+        run_max[lane * PL + i][warp] = run;
+        run = fmaxf(run, v);
+      }
+    }
+  }
+  __syncthreads();
+  // walk this thread's run: decisions, then the survivors' positions
+  float ahat[PRESKIP_MAX_R];
+#pragma unroll
+  for (int r = 0; r < PRESKIP_MAX_R; ++r) ahat[r] = run_max[threadIdx.x][r];
+  uint32_t keep_bits = 0;  // per = ceil(n / 256) <= 32 positions per thread (n <= 8192)
+  int kept = 0;
+  for (int j = j0; j < j1; ++j) {
+    const int p = lst[j];
+    bool keep = j == 0;
+#pragma unroll
+    for (int r = 0; r < PRESKIP_MAX_R; ++r) {
+      if (r >= R) break;
+      const float v = __ldg(arow + (long long)r * n_b + p);
+      if (v != -INFINITY && (ahat[r] == -INFINITY || (v + margin) - ahat[r] >= log_eps)) keep = true;
+      ahat[r] = fmaxf(ahat[r], v);
+    }
+    if (keep) {
+      keep_bits |= 1u << (j - j0);
+      ++kept;
+    }
+    if (skip_log) skip_log[row * k_cap + j] = keep ? 0 : 1;
+  }
+  int total = 0;
+  int pos = block_excl_scan(kept, warp_sums, &total);
+  for (int j = j0; j < j1; ++j)
+    if (keep_bits >> (j - j0) & 1u) orow[pos++] = lst[j];
+  for (int j = total + threadIdx.x; j < k_cap; j += blockDim.x) orow[j] = -1;
+  if (threadIdx.x == 0) count[row] = total;
+}
+
 }  // namespace cosa

@@ -168,6 +168,31 @@ cosa_status_t cosa_kap_rank(const cosa_shape_t* shape, const cosa_kap_params_t* 
                             int32_t* order, int32_t* count, float* scores, uint8_t* hrm,
                             void* workspace, size_t workspace_bytes, cosa_stream_t stream);
 
+/* Proxy-bound pre-skip: a variant the pages do not give (their in-kernel skip,
+ * gist.science/pt §2.3 "Saltado no Kernel", still pays every listed page its K
+ * load and QK^T).  It applies the same kind of test one stage earlier, on the
+ * proxy's page maxima a[r][p] and the proxy's own running maximum along each
+ * q-block's ordered list, and removes the pages it rejects before the kernel
+ * runs: with ahat_r(j) the maximum of a[r][.] over the pages listed before
+ * position j, representative r keeps position j iff a[r][p_j] > -inf and
+ * (ahat_r(j) = -inf or a[r][p_j] + margin - ahat_r(j) >= ln(eps)); position
+ * j >= 1 is removed iff no representative keeps it.  The survivors keep their
+ * order.  Filters order / count in place: the per-head lists that
+ * cosa_kap_select (or cosa_kap_rank) just wrote with this workspace, shape and
+ * kap, whose page maxima the workspace still holds.  skip_log (uint8
+ * [B][H_q][nQB][k_cap], may be NULL) gets 1 at the original list positions
+ * removed, 0 at the others (entries past the old count untouched).  eps >= 0
+ * (0 removes nothing), margin >= 0 and finite (nats).  Lists of up to 8192
+ * entries (COSA_ERR_UNSUPPORTED beyond); a list entry outside the q-block's
+ * causal pages leaves that list as it is and records COSA_ERR_INVALID_ARG in the
+ * status word.  The pre-skip decides on proxy estimates, not bounds: the output
+ * can differ from the pages' rule on the full list, and the pages' rule is
+ * what cosa_osk_attention then applies to the survivors. */
+cosa_status_t cosa_kap_preskip(const cosa_shape_t* shape, const cosa_kap_params_t* kap,
+                               float eps, float margin, int32_t* order, int32_t* count,
+                               uint8_t* skip_log, const void* workspace, size_t workspace_bytes,
+                               cosa_stream_t stream);
+
 /* Stage 1 with one list per KV head: the G query heads that read KV head h_kv
  * share one ordered list per q-block (the group-shared selection; the pages
  * describe per-head selection only, this is the next step after it).  Every
