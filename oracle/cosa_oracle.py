@@ -43,7 +43,7 @@ __all__ = [
     "kap_maxnorm_hrm", "rank_key", "kap_order_from_scores", "kap_select_block",
     "kap_select", "kap_order", "osk_block", "osk_block_rules", "osk_attention", "dense_rows",
     "dense_attention", "kap_group_scores", "kap_select_group", "expand_group_order",
-    "kap_preskip", "kap_preskip_lists",
+    "kap_preskip", "kap_preskip_lists", "osk_decode",
 ]
 
 NEG_INF = -math.inf
@@ -604,6 +604,53 @@ def osk_attention(q: np.ndarray, k_pool: np.ndarray, v_pool: np.ndarray,
             margin[b, h, qb, :c] = r["margin"]
     return {"out": out, "lse": lse, "computed": computed, "visited": visited, "skip": skip,
             "margin": margin}
+
+
+# ----------------------------------------------------------------------------
+# Decode: one new query per sequence and head, after the prefill.  The pages
+# leave decoding as future work ([TS] closing section); the reading here is the
+# plainest continuation of the prefill method: the query at position t sees keys
+# 0..t of the paged cache and visits an ordered page list (for instance the list
+# KAP produced for the q-block holding t) under the same in-kernel rule, as a
+# q-block of one row (osk_block_rules with q_block = 1 and qb = t).
+# ----------------------------------------------------------------------------
+def osk_decode(q: np.ndarray, k_pool: np.ndarray, v_pool: np.ndarray, page_table: np.ndarray,
+               positions: Sequence[int], order: np.ndarray, count: np.ndarray, *,
+               num_kv_heads: int, page_size: int, eps: float, scale: float,
+               heads: Optional[Sequence] = None):
+    """Single-query ordered-skipping attention.  q [B][H_q][D] (the new query of
+    each sequence and head), positions [B] (its position t: it sees keys 0..t),
+    order [B][H_q][k_cap] (logical pages, each <= t // P), count [B][H_q].
+    Returns dict with out float64 [B][H_q][D], lse [B][H_q], computed int32
+    [B][H_q], skip uint8 [B][H_q][k_cap], margin float64 [B][H_q][k_cap]."""
+    B, Hq, D = q.shape
+    G = Hq // num_kv_heads
+    kc = order.shape[-1]
+    out = np.zeros((B, Hq, D))
+    lse = np.full((B, Hq), NEG_INF)
+    computed = np.zeros((B, Hq), dtype=np.int32)
+    skip = np.zeros((B, Hq, kc), dtype=np.uint8)
+    margin = np.full((B, Hq, kc), np.nan)
+    if heads is None:
+        heads = [(b, h) for b in range(B) for h in range(Hq)]
+    cache = {}
+    for (b, h) in heads:
+        t = int(positions[b])
+        hk = h // G
+        if (b, hk) not in cache:
+            n_tok = (t // page_size + 1) * page_size
+            cache[(b, hk)] = (gather_logical(k_pool, page_table, b, hk, n_tok),
+                              gather_logical(v_pool, page_table, b, hk, n_tok))
+        k_log, v_log = cache[(b, hk)]
+        c = int(count[b, h])
+        r = osk_block_rules(np.asarray(q[b, h], dtype=np.float64)[None, :], k_log, v_log, t, 1,
+                            page_size, order[b, h, :c], eps, scale)
+        out[b, h] = r["out"][0]
+        lse[b, h] = r["lse"][0]
+        computed[b, h] = r["computed"]
+        skip[b, h, :c] = r["skip"]
+        margin[b, h, :c] = r["margin"]
+    return {"out": out, "lse": lse, "computed": computed, "skip": skip, "margin": margin}
 
 
 # ----------------------------------------------------------------------------
