@@ -840,6 +840,49 @@ def main():
     except Exception as exc:  # an extra leg: report the failure, keep the line
         line["preskip"] = {"error": repr(exc)}
 
+    # ---- decode (the pages' future work): the last token of every head with the list
+    # KAP wrote for its q-block, against the same kernel visiting every page
+    def decode_leg():
+        t = N - 1
+        P_ = wl.page_size
+        qdec = x["q"][:, :, t].contiguous()
+        pos = torch.full((B,), t, dtype=torch.int32, device=dev)
+        o_dec, c_dec = order[:, :, -1].contiguous(), count[:, :, -1].contiguous()
+        n_all = t // P_ + 1
+        o_full = torch.full((B, Hq, wl.num_pages), -1, dtype=torch.int32, device=dev)
+        o_full[:, :, :n_all] = torch.arange(n_all, dtype=torch.int32, device=dev)
+        c_full = torch.full((B, Hq), n_all, dtype=torch.int32, device=dev)
+        outd = torch.empty(B, Hq, D, dtype=torch.bfloat16, device=dev)
+        compd = torch.empty(B, Hq, dtype=torch.int32, device=dev)
+        wsd = torch.empty(C.cosa_osk_decode_workspace_size(shape, wl.num_pages), dtype=torch.uint8,
+                          device=dev)
+        page_bytes = P_ * D * 2
+        res = []
+        for label, o, c, eps in (("KAP list", o_dec, c_dec, args.eps), ("KAP list", o_dec, c_dec, 0.0),
+                                 ("every page", o_full, c_full, 0.0)):
+            od = C.OskParams(eps=eps)
+            ms = _timed(lambda: C.cosa_osk_decode(shape, od, qdec, x["k_pool"], x["v_pool"],
+                                                  x["page_table"], pos, o, c, outd, wsd,
+                                                  computed=compd, stream=stream), 20, stream, warm=3)
+            if C.cosa_get_status(stream) != 0:
+                raise RuntimeError("in-kernel error status in decode")
+            listed = int(c.to(torch.int64).sum().item())
+            kept = int(compd.to(torch.int64).sum().item())
+            byts = (listed + kept) * page_bytes  # K of every listed page, V of every kept one
+            res.append({"list": label, "eps": eps, "us": ms * 1e3, "listed_pages": listed,
+                        "computed_pages": kept, "bytes": byts,
+                        "gbs": byts / (ms * 1e-3) / 1e9, "frac_vs_hbm": byts / (ms * 1e-3) / 1e9 / hbm})
+        for r in res:
+            r["speedup_vs_every_page"] = res[-1]["us"] / r["us"]
+        return {"position": t, "heads": B * Hq, "points": res,
+                "note": "bytes: K of the listed pages + V of the kept pages, read by each head "
+                        "(the G heads of a KV head share pages through L2)"}
+
+    try:
+        line["decode"] = decode_leg()
+    except Exception as exc:  # an extra leg: report the failure, keep the line
+        line["decode"] = {"error": repr(exc)}
+
     line["e2e"] = e2e_leg()
     del dense_out, dref, outg
     torch.cuda.empty_cache()

@@ -21,7 +21,7 @@ __all__ = [
     "cosa_dense_attention", "cosa_get_status", "EXPORTED_SYMBOLS", "NOALLOC_SCRATCH_BYTES",
     "cosa_kap_select_group", "cosa_osk_attention_group", "cosa_attention_host_workspace_size",
     "cosa_attention_host", "cosa_debug_osk_wait_fault", "cosa_kap_pool", "cosa_kap_rank",
-    "cosa_kap_preskip",
+    "cosa_kap_preskip", "cosa_osk_decode", "cosa_osk_decode_workspace_size",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -32,7 +32,8 @@ EXPORTED_SYMBOLS = (
     "cosa_kap_select", "cosa_kap_select_noalloc", "cosa_kap_order", "cosa_osk_attention",
     "cosa_dense_attention", "cosa_get_status", "cosa_kap_select_group", "cosa_osk_attention_group",
     "cosa_attention_host_workspace_size", "cosa_attention_host", "cosa_debug_osk_wait_fault",
-    "cosa_kap_pool", "cosa_kap_rank", "cosa_kap_preskip",
+    "cosa_kap_pool", "cosa_kap_rank", "cosa_kap_preskip", "cosa_osk_decode",
+    "cosa_osk_decode_workspace_size",
 )
 
 # Largest workspace the allocation-free Stage-1 entry point accepts (cosa.h).
@@ -156,6 +157,9 @@ def lib():
     L.cosa_debug_osk_wait_fault.argtypes = [i32, ctypes.c_uint64]
     L.cosa_kap_pool.argtypes = [P(_Shape), P(_Kap), vp, vp, vp, vp, sz, vp]
     L.cosa_kap_rank.argtypes = [P(_Shape), P(_Kap), vp, vp, vp, vp, vp, sz, vp]
+    L.cosa_osk_decode_workspace_size.argtypes = [P(_Shape), i32, P(sz)]
+    L.cosa_osk_decode.argtypes = [P(_Shape), P(_Osk), vp, vp, vp, vp, vp, vp, vp, i32, vp, vp, vp,
+                                  vp, vp, sz, vp]
     L.cosa_kap_preskip.argtypes = [P(_Shape), P(_Kap), ctypes.c_float, ctypes.c_float, vp, vp, vp,
                                    vp, sz, vp]
     for name in EXPORTED_SYMBOLS:
@@ -428,6 +432,48 @@ def cosa_osk_attention_group(shape: Shape, osk: OskParams, q, k_pool, v_pool, pa
                                           _ptr(v_pool), _ptr(page_table), _ptr(order), _ptr(count),
                                           kc, _ptr(out), _ptr(lse), _ptr(computed), _ptr(skip_log),
                                           _stream(stream)), "cosa_osk_attention_group")
+
+
+def cosa_osk_decode_workspace_size(shape: Shape, k_cap: int) -> int:
+    s = shape.c()
+    n = ctypes.c_size_t(0)
+    _check(lib().cosa_osk_decode_workspace_size(ctypes.byref(s), int(k_cap), ctypes.byref(n)),
+           "cosa_osk_decode_workspace_size")
+    return n.value
+
+
+def cosa_osk_decode(shape: Shape, osk: OskParams, q, k_pool, v_pool, page_table, positions, order,
+                    count, out, workspace, lse=None, computed=None, skip_log=None,
+                    stream=None) -> None:
+    """Decode: the query of each sequence and head (q [B][H_q][D], at positions [B])
+    visits its ordered page list (order [B][H_q][k_cap], count [B][H_q]) under the
+    in-kernel skip rule; out [B][H_q][D]."""
+    import torch
+    s, o = shape.c(), osk.c()
+    B, Hq, D = shape.batch, shape.num_q_heads, shape.head_dim
+    kc = order.shape[-1]
+    _expect(q, "q", torch.bfloat16, (B, Hq, D))
+    _expect(k_pool, "k_pool", torch.bfloat16, _kv_shape(shape))
+    _expect(v_pool, "v_pool", torch.bfloat16, _kv_shape(shape))
+    _expect(page_table, "page_table", torch.int32, (B, s.pages_per_seq))
+    _expect(positions, "positions", torch.int32, (B,))
+    _expect(order, "order", torch.int32, (B, Hq, kc))
+    _expect(count, "count", torch.int32, (B, Hq))
+    _expect(out, "out", torch.bfloat16, (B, Hq, D))
+    if lse is not None:
+        _expect(lse, "lse", torch.float32, (B, Hq))
+    if computed is not None:
+        _expect(computed, "computed", torch.int32, (B, Hq))
+    if skip_log is not None:
+        _expect(skip_log, "skip_log", torch.uint8, (B, Hq, kc))
+    if workspace is None or not workspace.is_cuda:
+        raise ValueError("workspace must be a CUDA tensor")
+    nbytes = workspace.numel() * workspace.element_size()
+    _check(lib().cosa_osk_decode(ctypes.byref(s), ctypes.byref(o), _ptr(q), _ptr(k_pool),
+                                 _ptr(v_pool), _ptr(page_table), _ptr(positions), _ptr(order),
+                                 _ptr(count), kc, _ptr(out), _ptr(lse), _ptr(computed),
+                                 _ptr(skip_log), _ptr(workspace), nbytes, _stream(stream)),
+           "cosa_osk_decode")
 
 
 def cosa_dense_attention(shape: Shape, q, k_pool, v_pool, page_table, out, lse=None,

@@ -14,6 +14,7 @@
 #include "attn_tc.cuh"
 #include "attn_dense.cuh"
 #include "attn_gqa.cuh"
+#include "decode.cuh"
 
 using namespace cosa;
 
@@ -362,6 +363,43 @@ TcParams make_params(const cosa_shape_t* s, void* out, float* lse, const int32_t
   p.timeout_ns = kWaitTimeoutNs;
   p.fault_k_group = -1;
   return p;
+}
+
+// Workspace of cosa_osk_decode: the listed pages' logits and local maxima, and the
+// per-chunk partial sums.
+struct DecodeLayout {
+  size_t logits, mloc, po, pl, pn, total;
+  int n_chunks;
+};
+
+DecodeLayout decode_layout(const cosa_shape_t* s, int k_cap) {
+  DecodeLayout L;
+  const size_t bh = (size_t)s->batch * s->num_q_heads;
+  L.n_chunks = (k_cap + DEC_CHUNK - 1) / DEC_CHUNK;
+  size_t off = 0;
+  L.logits = off;
+  off = align256(off + bh * k_cap * s->page_size * sizeof(float));
+  L.mloc = off;
+  off = align256(off + bh * k_cap * sizeof(float));
+  L.po = off;
+  off = align256(off + bh * L.n_chunks * s->head_dim * sizeof(float));
+  L.pl = off;
+  off = align256(off + bh * L.n_chunks * sizeof(float));
+  L.pn = off;
+  off = align256(off + bh * L.n_chunks * sizeof(int));
+  L.total = off;
+  return L;
+}
+
+template <int D, int P>
+cosa_status_t launch_decode_t(const DecodeParams& prm, int bh, cudaStream_t st) {
+  dim3 grid(prm.n_chunks, bh);
+  decode_qk_kernel<D, P><<<grid, DEC_THREADS, 0, st>>>(prm);
+  if (last_launch() != COSA_OK) return COSA_ERR_CUDA;
+  decode_pv_kernel<D, P><<<grid, DEC_THREADS, 0, st>>>(prm);
+  if (last_launch() != COSA_OK) return COSA_ERR_CUDA;
+  decode_combine_kernel<D><<<bh, 128, 0, st>>>(prm);
+  return last_launch();
 }
 
 // Test hook of cosa_debug_osk_wait_fault: one-shot, per host thread.
@@ -787,6 +825,73 @@ cosa_status_t cosa_dense_attention(const cosa_shape_t* shape, const void* q, con
   if (D == 128 && P == 128) return launch_dense_t<128, 128>(shape, p, q, k_pool, v_pool, (int)grid, st);
   if (D == 64 && P == 64) return launch_dense_t<64, 64>(shape, p, q, k_pool, v_pool, (int)grid, st);
   if (D == 64 && P == 128) return launch_dense_t<64, 128>(shape, p, q, k_pool, v_pool, (int)grid, st);
+  return COSA_ERR_UNSUPPORTED;
+}
+
+cosa_status_t cosa_osk_decode_workspace_size(const cosa_shape_t* shape, int32_t k_cap,
+                                             size_t* bytes) {
+  cosa_status_t e = check_shape(shape);
+  if (e != COSA_OK) return e;
+  if (!bytes || k_cap <= 0 || k_cap > shape->seq_len / shape->page_size) return COSA_ERR_INVALID_ARG;
+  *bytes = decode_layout(shape, k_cap).total;
+  return COSA_OK;
+}
+
+cosa_status_t cosa_osk_decode(const cosa_shape_t* shape, const cosa_osk_params_t* osk,
+                              const void* q, const void* k_pool, const void* v_pool,
+                              const int32_t* page_table, const int32_t* positions,
+                              const int32_t* order, const int32_t* count, int32_t k_cap, void* out,
+                              float* lse, int32_t* computed, uint8_t* skip_log, void* workspace,
+                              size_t workspace_bytes, cosa_stream_t stream) {
+  cosa_status_t e = check_shape(shape);
+  if (e != COSA_OK) return e;
+  if (!osk || !(osk->eps >= 0.f && osk->eps <= 1.f) || osk->max_run < 0) return COSA_ERR_INVALID_ARG;
+  if (osk->max_run != 0) return COSA_ERR_UNSUPPORTED;
+  if (!q || !k_pool || !v_pool || !page_table || !positions || !order || !count || !out)
+    return COSA_ERR_INVALID_ARG;
+  if (k_cap <= 0 || k_cap > shape->seq_len / shape->page_size) return COSA_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(q) % 16 || reinterpret_cast<uintptr_t>(k_pool) % 16 ||
+      reinterpret_cast<uintptr_t>(v_pool) % 16)
+    return COSA_ERR_INVALID_ARG;
+  const DecodeLayout L = decode_layout(shape, k_cap);
+  if (!workspace || workspace_bytes < L.total || reinterpret_cast<uintptr_t>(workspace) % 256)
+    return COSA_ERR_WORKSPACE;
+  const long long bh = (long long)shape->batch * shape->num_q_heads;
+  if (bh > 65535) return COSA_ERR_UNSUPPORTED;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  DecodeParams prm;
+  std::memset(&prm, 0, sizeof(prm));
+  prm.q = reinterpret_cast<const __nv_bfloat16*>(q);
+  prm.k_pool = reinterpret_cast<const __nv_bfloat16*>(k_pool);
+  prm.v_pool = reinterpret_cast<const __nv_bfloat16*>(v_pool);
+  prm.page_table = page_table;
+  prm.positions = positions;
+  prm.order = order;
+  prm.count = count;
+  prm.out = reinterpret_cast<__nv_bfloat16*>(out);
+  prm.lse = lse;
+  prm.computed = computed;
+  prm.skip_log = skip_log;
+  prm.logits = reinterpret_cast<float*>(ws + L.logits);
+  prm.mloc = reinterpret_cast<float*>(ws + L.mloc);
+  prm.part_o = reinterpret_cast<float*>(ws + L.po);
+  prm.part_l = reinterpret_cast<float*>(ws + L.pl);
+  prm.part_n = reinterpret_cast<int*>(ws + L.pn);
+  prm.num_q_heads = shape->num_q_heads;
+  prm.num_kv_heads = shape->num_kv_heads;
+  prm.group = shape->num_q_heads / shape->num_kv_heads;
+  prm.seq_len = shape->seq_len;
+  prm.pages_per_seq = shape->pages_per_seq;
+  prm.k_cap = k_cap;
+  prm.n_chunks = L.n_chunks;
+  prm.scale_log2 = shape->softmax_scale * 1.4426950408889634f;
+  prm.log2_eps = osk->eps > 0.f ? log2f(osk->eps) : -INFINITY;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int D = shape->head_dim, P = shape->page_size;
+  if (D == 128 && P == 64) return launch_decode_t<128, 64>(prm, (int)bh, st);
+  if (D == 128 && P == 128) return launch_decode_t<128, 128>(prm, (int)bh, st);
+  if (D == 64 && P == 64) return launch_decode_t<64, 64>(prm, (int)bh, st);
+  if (D == 64 && P == 128) return launch_decode_t<64, 128>(prm, (int)bh, st);
   return COSA_ERR_UNSUPPORTED;
 }
 

@@ -274,6 +274,33 @@ cosa_status_t cosa_osk_attention_group(const cosa_shape_t* shape, const cosa_osk
                                        const int32_t* count, int32_t k_cap, void* out, float* lse,
                                        int32_t* computed, uint8_t* skip_log, cosa_stream_t stream);
 
+/* Bytes of device workspace cosa_osk_decode needs for lists of k_cap entries: the
+ * listed pages' logits and local maxima, and per-chunk partial sums.  Host-only. */
+cosa_status_t cosa_osk_decode_workspace_size(const cosa_shape_t* shape, int32_t k_cap,
+                                             size_t* bytes);
+
+/* Decode: one new query per sequence and head visits an ordered page list under
+ * the in-kernel rule of Stage 2 (gist.science/pt §2.3), as a q-block of one row.
+ * The pages leave decoding as future work (closing section); this is the plainest
+ * continuation of the prefill method (for instance with the list KAP wrote for the
+ * q-block that holds the query).  q bf16 [B][H_q][D]: the query of each sequence
+ * and head; positions int32 [B] (device): its position t, 0 <= t < seq_len; it
+ * sees keys 0..t of the paged cache (k_pool / v_pool / page_table as above,
+ * holding at least t + 1 tokens).  order int32 [B][H_q][k_cap] (logical pages,
+ * each <= t / P, distinct), count int32 [B][H_q].  eps in [0, 1] (the rule above;
+ * eps > 1 is rejected with COSA_ERR_INVALID_ARG), max_run 0 (COSA_ERR_UNSUPPORTED
+ * otherwise).  out bf16 [B][H_q][D]; lse fp32 [B][H_q], computed int32 [B][H_q]
+ * and skip_log uint8 [B][H_q][k_cap] may be NULL.  workspace: at least
+ * cosa_osk_decode_workspace_size(shape, k_cap) bytes, 256-byte aligned.  A list
+ * entry past the query's page, or a position out of range, is never read: it is
+ * recorded as COSA_ERR_INVALID_ARG in the status word. */
+cosa_status_t cosa_osk_decode(const cosa_shape_t* shape, const cosa_osk_params_t* osk,
+                              const void* q, const void* k_pool, const void* v_pool,
+                              const int32_t* page_table, const int32_t* positions,
+                              const int32_t* order, const int32_t* count, int32_t k_cap, void* out,
+                              float* lse, int32_t* computed, uint8_t* skip_log, void* workspace,
+                              size_t workspace_bytes, cosa_stream_t stream);
+
 /* Dense causal attention over the same paged cache (every causal page in page
  * order, no skipping): the comparison point for the sparse path's speedup.
  * lse may be NULL. */
