@@ -883,6 +883,59 @@ def main():
     except Exception as exc:  # an extra leg: report the failure, keep the line
         line["decode"] = {"error": repr(exc)}
 
+    # ---- KAP pooling fused into the prefill's write of Q / K / V: the plain write then
+    # cosa_kap_select, against the fused write then cosa_kap_rank (same lists)
+    def fused_write_leg():
+        P_ = wl.page_size
+        pt = x["page_table"].long()
+        tok = lambda pool: torch.stack([pool[pt[b_]].permute(0, 2, 1, 3).reshape(N, Hk, D)
+                                        for b_ in range(B)]).contiguous()
+        q_tok, k_tok, v_tok = x["q"].permute(0, 2, 1, 3).contiguous(), tok(x["k_pool"]), tok(x["v_pool"])
+        q2, kp2, vp2 = torch.empty_like(x["q"]), torch.empty_like(x["k_pool"]), torch.empty_like(x["v_pool"])
+        ws2 = torch.empty_like(ws)
+        o2, c2 = torch.empty_like(order), torch.empty_like(count)
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+
+        def run(fused):
+            ev[0].record(stream)
+            C.cosa_prefill_write(shape, kap, q_tok, k_tok, v_tok, x["page_table"], q2, kp2, vp2,
+                                 workspace=ws2 if fused else None, stream=stream)
+            ev[1].record(stream)
+            if fused:
+                C.cosa_kap_rank(shape, kap, o2, c2, ws2, stream=stream)
+            else:
+                C.cosa_kap_select(shape, kap, q2, kp2, x["page_table"], o2, c2, ws2, stream=stream)
+            ev[2].record(stream)
+            C.cosa_osk_attention(shape, osk, q2, kp2, vp2, x["page_table"], o2, c2, out,
+                                 stream=stream)
+            ev[3].record(stream)
+            ev[3].synchronize()
+            return [ev[i].elapsed_time(ev[i + 1]) for i in range(3)]
+
+        res = {}
+        for fused in (False, True):
+            run(fused)
+            t = [0.0, 0.0, 0.0]
+            for _ in range(3):
+                t = [a + b_ / 3 for a, b_ in zip(t, run(fused))]
+            res["fused" if fused else "plain"] = {"write_ms": t[0], "stage1_ms": t[1],
+                                                  "osk_ms": t[2], "ms": sum(t)}
+        if C.cosa_get_status(stream) != 0:
+            raise RuntimeError("in-kernel error status")
+        rw = 2.0 * 2 * B * N * D * (Hq + 2 * Hk)  # Q, K, V read once and written once (bf16)
+        pooled = 2 * 4.0 * D * B * (Hq * N / (wl.q_block // 4) + Hk * N / 16)
+        fw = res["fused"]["write_ms"]
+        res["fused_write_roofline"] = {"bound": "hbm", "bytes": rw + pooled,
+                                       "achieved": (rw + pooled) / (fw * 1e-3) / 1e9, "peak": hbm,
+                                       "unit": "GB/s", "frac": (rw + pooled) / (fw * 1e-3) / 1e9 / hbm}
+        res["saved_ms"] = res["plain"]["ms"] - res["fused"]["ms"]
+        return res
+
+    try:
+        line["fused_write"] = fused_write_leg()
+    except Exception as exc:  # an extra leg: report the failure, keep the line
+        line["fused_write"] = {"error": repr(exc)}
+
     line["e2e"] = e2e_leg()
     del dense_out, dref, outg
     torch.cuda.empty_cache()

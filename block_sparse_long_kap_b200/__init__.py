@@ -22,6 +22,7 @@ __all__ = [
     "cosa_kap_select_group", "cosa_osk_attention_group", "cosa_attention_host_workspace_size",
     "cosa_attention_host", "cosa_debug_osk_wait_fault", "cosa_kap_pool", "cosa_kap_rank",
     "cosa_kap_preskip", "cosa_osk_decode", "cosa_osk_decode_workspace_size",
+    "cosa_prefill_write",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -33,7 +34,7 @@ EXPORTED_SYMBOLS = (
     "cosa_dense_attention", "cosa_get_status", "cosa_kap_select_group", "cosa_osk_attention_group",
     "cosa_attention_host_workspace_size", "cosa_attention_host", "cosa_debug_osk_wait_fault",
     "cosa_kap_pool", "cosa_kap_rank", "cosa_kap_preskip", "cosa_osk_decode",
-    "cosa_osk_decode_workspace_size",
+    "cosa_osk_decode_workspace_size", "cosa_prefill_write",
 )
 
 # Largest workspace the allocation-free Stage-1 entry point accepts (cosa.h).
@@ -160,6 +161,7 @@ def lib():
     L.cosa_osk_decode_workspace_size.argtypes = [P(_Shape), i32, P(sz)]
     L.cosa_osk_decode.argtypes = [P(_Shape), P(_Osk), vp, vp, vp, vp, vp, vp, vp, i32, vp, vp, vp,
                                   vp, vp, sz, vp]
+    L.cosa_prefill_write.argtypes = [P(_Shape), P(_Kap), vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
     L.cosa_kap_preskip.argtypes = [P(_Shape), P(_Kap), ctypes.c_float, ctypes.c_float, vp, vp, vp,
                                    vp, sz, vp]
     for name in EXPORTED_SYMBOLS:
@@ -289,6 +291,32 @@ def cosa_kap_rank(shape: Shape, kap: KapParams, order, count, workspace, scores=
     _check(lib().cosa_kap_rank(ctypes.byref(s), ctypes.byref(k), _ptr(order), _ptr(count),
                                _ptr(scores), _ptr(hrm), _ptr(workspace), nbytes, _stream(stream)),
            "cosa_kap_rank")
+
+
+def cosa_prefill_write(shape: Shape, kap: KapParams, q_tok, k_tok, v_tok, page_table, q, k_pool,
+                       v_pool, workspace=None, stream=None) -> None:
+    """Write token-major Q / K / V ([B][N][H][D]) as head-major q and the paged k_pool /
+    v_pool, pooling Q and K into the KAP workspace in the same pass (workspace None: the
+    plain write).  cosa_kap_rank on that workspace then finishes Stage 1."""
+    import torch
+    s, k = shape.c(), kap.c(shape)
+    B, Hq, Hk, N, D = shape.batch, shape.num_q_heads, shape.num_kv_heads, shape.seq_len, shape.head_dim
+    _expect(q_tok, "q_tok", torch.bfloat16, (B, N, Hq, D))
+    _expect(k_tok, "k_tok", torch.bfloat16, (B, N, Hk, D))
+    _expect(v_tok, "v_tok", torch.bfloat16, (B, N, Hk, D))
+    _expect(page_table, "page_table", torch.int32, (B, s.pages_per_seq))
+    _expect(q, "q", torch.bfloat16, (B, Hq, N, D))
+    _expect(k_pool, "k_pool", torch.bfloat16, _kv_shape(shape))
+    _expect(v_pool, "v_pool", torch.bfloat16, _kv_shape(shape))
+    nbytes = 0
+    if workspace is not None:
+        if not workspace.is_cuda:
+            raise ValueError("workspace must be a CUDA tensor")
+        nbytes = workspace.numel() * workspace.element_size()
+    _check(lib().cosa_prefill_write(ctypes.byref(s), ctypes.byref(k), _ptr(q_tok), _ptr(k_tok),
+                                    _ptr(v_tok), _ptr(page_table), _ptr(q), _ptr(k_pool),
+                                    _ptr(v_pool), _ptr(workspace), nbytes, _stream(stream)),
+           "cosa_prefill_write")
 
 
 def cosa_kap_preskip(shape: Shape, kap: KapParams, eps: float, margin: float, order, count,

@@ -142,7 +142,9 @@ struct TcCfg {
 // so it is kept rare; P = exp2(s - m_ref) <= 2^32, l <= 2^32 * keys, all in range
 constexpr float kRescaleLog2 = 32.0f;
 
-template <int D, int P>
+// BRK: the early break is compiled in (max_run > 0); without it the kernel carries none
+// of its code, which keeps the hot loop's instruction footprint small
+template <int D, int P, bool BRK>
 __global__ void __launch_bounds__(TcCfg<D, P>::NT, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const TcParams prm) {
@@ -276,7 +278,7 @@ __global__ void __launch_bounds__(TcCfg<D, P>::NT, 1)
   const uint32_t tmem = *tmem_slot;
 
   const unsigned long long tmo = prm.timeout_ns;
-  const int R = prm.max_run;  // early break after R consecutive skipped pages (0: none)
+  const int R = BRK ? prm.max_run : 0;  // early break after R consecutive skipped pages (0: none)
   auto give_up = [&]() {
     *abort_flag = 1;
     set_status(COSA_ERR_TIMEOUT);
@@ -949,7 +951,7 @@ __global__ void __launch_bounds__(TcCfg<D, P>::NT, 1)
     const float inv = (have && lt > 0.f) ? 1.f / lt : 0.f;
     constexpr int HD = D / 2;  // each warpgroup writes half of the columns
     __nv_bfloat16* orow = prm.out + (bh * prm.seq_len + grow) * D + wg * HD;
-#pragma unroll
+#pragma unroll 1
     for (int k = 0; k < HD / 32; ++k) {
       uint32_t r[32];
       if (have) {

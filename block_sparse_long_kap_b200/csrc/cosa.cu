@@ -288,7 +288,7 @@ cosa_status_t launch_tc_t(const cosa_shape_t* s, const TcParams& prm, const void
   if (!make_map(&mq, q, D, s->seq_len, BH, s->q_block) ||
       !make_map(&mk, k_pool, D, P, PZ, P) || !make_map(&mv, v_pool, D, P, PZ, P))
     return COSA_ERR_CUDA;
-  auto kern = attn_tc_kernel<D, P>;
+  auto kern = prm.max_run > 0 ? attn_tc_kernel<D, P, true> : attn_tc_kernel<D, P, false>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)Cfg::SMEM_ALLOC) != cudaSuccess)
     return COSA_ERR_CUDA;
@@ -640,6 +640,50 @@ cosa_status_t cosa_kap_rank(const cosa_shape_t* shape, const cosa_kap_params_t* 
   if (shape->head_dim == 128)
     return launch_rank<128>(shape, kap, order, count, scores, hrm, L, ws, k_cap, st);
   return launch_rank<64>(shape, kap, order, count, scores, hrm, L, ws, k_cap, st);
+}
+
+cosa_status_t cosa_prefill_write(const cosa_shape_t* shape, const cosa_kap_params_t* kap,
+                                 const void* q_tok, const void* k_tok, const void* v_tok,
+                                 const int32_t* page_table, void* q, void* k_pool, void* v_pool,
+                                 void* workspace, size_t workspace_bytes, cosa_stream_t stream) {
+  cosa_status_t e = check_shape(shape);
+  if (e != COSA_OK) return e;
+  if ((e = check_kap(shape, kap)) != COSA_OK) return e;
+  if (!q_tok || !k_tok || !v_tok || !page_table || !q || !k_pool || !v_pool)
+    return COSA_ERR_INVALID_ARG;
+  const void* bufs[] = {q_tok, k_tok, v_tok, q, k_pool, v_pool};
+  for (const void* b : bufs)
+    if (reinterpret_cast<uintptr_t>(b) % 16) return COSA_ERR_INVALID_ARG;
+  KapLayout L = kap_layout(shape, kap);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  if (ws && (workspace_bytes < L.total || reinterpret_cast<uintptr_t>(ws) % 256))
+    return COSA_ERR_WORKSPACE;
+  const int B = shape->batch, Hq = shape->num_q_heads, Hk = shape->num_kv_heads, N = shape->seq_len;
+  const int P = shape->page_size, Bq = shape->q_block, nP = N / P, nQB = N / Bq;
+  const int R = Bq / kap->q_sub, T = P / kap->k_sub, G = Hq / Hk;
+  const long long n_qvec = (long long)B * Hq * nQB * R;
+  const long long n_kvec = (long long)B * Hk * nP * T;
+  const long long blocks = (n_qvec + n_kvec + 7) / 8;
+  if (blocks > 0x7fffffffll) return COSA_ERR_UNSUPPORTED;
+  float* f[4] = {nullptr, nullptr, nullptr, nullptr};
+  if (ws) {
+    f[0] = reinterpret_cast<float*>(ws + L.q_hi);
+    f[1] = reinterpret_cast<float*>(ws + L.q_lo);
+    f[2] = reinterpret_cast<float*>(ws + L.k_hi);
+    f[3] = reinterpret_cast<float*>(ws + L.k_lo);
+  }
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  using bf = __nv_bfloat16;
+  auto args = [&](auto kern) {
+    kern<<<(unsigned)blocks, 256, 0, st>>>(
+        static_cast<const bf*>(q_tok), static_cast<const bf*>(k_tok), static_cast<const bf*>(v_tok),
+        page_table, static_cast<bf*>(q), static_cast<bf*>(k_pool), static_cast<bf*>(v_pool), f[0],
+        f[1], f[2], f[3], n_qvec, kap->q_sub, n_kvec, kap->k_sub, Hq, Hk, G, R, nQB, P, nP,
+        shape->pages_per_seq, T, N);
+  };
+  if (shape->head_dim == 128) args(prefill_write_kernel<128>);
+  else args(prefill_write_kernel<64>);
+  return last_launch();
 }
 
 cosa_status_t cosa_kap_preskip(const cosa_shape_t* shape, const cosa_kap_params_t* kap,

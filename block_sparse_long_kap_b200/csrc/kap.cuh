@@ -133,6 +133,122 @@ __global__ void __launch_bounds__(256) kap_pool_kernel(
 }
 
 // ---------------------------------------------------------------------------
+// KAP pooling fused into the prefill's write of its attention inputs.  The Q, K and
+// V a prefill layer produces arrive token-major ([B][N][H][D], the projection's
+// layout); attention reads Q head-major and K / V from the paged cache.  This kernel
+// does that write (Q relaid head-major, K and V scattered into their pages through
+// the page table) and, in the same pass over the rows, the downsampling of
+// kap_pool_kernel, so Stage 1 needs no second read of Q and K (cosa_kap_rank then
+// finishes it from the workspace).  Work items are those of kap_pool_kernel; a key
+// item also copies the V rows of its token range.  Each lane accumulates the same
+// rows in the same order as kap_pool_kernel, so the pooled vectors are identical.
+// With pooling off (q_hi null) it is the plain write.
+// ---------------------------------------------------------------------------
+template <int D>
+__global__ void __launch_bounds__(256) prefill_write_kernel(
+    const __nv_bfloat16* __restrict__ q_tok, const __nv_bfloat16* __restrict__ k_tok,
+    const __nv_bfloat16* __restrict__ v_tok, const int32_t* __restrict__ page_table,
+    __nv_bfloat16* __restrict__ q_out, __nv_bfloat16* __restrict__ k_pool,
+    __nv_bfloat16* __restrict__ v_pool, float* __restrict__ q_hi, float* __restrict__ q_lo,
+    float* __restrict__ k_hi, float* __restrict__ k_lo, long long n_qvec, int q_sub,
+    long long n_kvec, int k_sub, int num_q_heads, int num_kv_heads, int group, int R,
+    int num_q_blocks, int page_size, int num_pages, int pages_per_seq, int T, int seq_len) {
+  constexpr int LPR = D / 8;     // lanes per row: each lane moves 8 bf16 (16 B)
+  constexpr int RPI = 32 / LPR;  // rows covered per warp-wide load
+  const int lane = threadIdx.x & 31;
+  const long long w = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const bool pool = q_hi != nullptr;
+  const __nv_bfloat16* src;
+  const __nv_bfloat16* vsrc = nullptr;
+  __nv_bfloat16* dst;
+  __nv_bfloat16* vdst = nullptr;
+  long long src_stride, drow;
+  float *dhi, *dlo;
+  int rows;
+  if (w < n_qvec) {
+    const int r = (int)(w % R);
+    long long t1 = w / R;
+    const int qb = (int)(t1 % num_q_blocks);
+    const long long bhq = t1 / num_q_blocks;
+    const int h = (int)(bhq % num_q_heads);
+    const int b = (int)(bhq / num_q_heads);
+    const int hk = h / group, g = h % group;
+    const long long tok0 = (long long)qb * (R * q_sub) + (long long)r * q_sub;
+    src = q_tok + (((long long)b * seq_len + tok0) * num_q_heads + h) * D;
+    src_stride = (long long)num_q_heads * D;
+    dst = q_out + (bhq * seq_len + tok0) * D;
+    drow = ((long long)(b * num_kv_heads + hk) * num_q_blocks + qb) * (group * R) + g * R + r;
+    dhi = q_hi;
+    dlo = q_lo;
+    rows = q_sub;
+  } else {
+    const long long kv = w - n_qvec;
+    if (kv >= n_kvec) return;
+    const int t = (int)(kv % T);
+    long long r = kv / T;
+    const int p = (int)(r % num_pages);
+    r /= num_pages;
+    const int hk = (int)(r % num_kv_heads);
+    const int b = (int)(r / num_kv_heads);
+    const int phys = page_table[(long long)b * pages_per_seq + p];
+    const long long tok0 = (long long)p * page_size + (long long)t * k_sub;
+    const long long off_src = (((long long)b * seq_len + tok0) * num_kv_heads + hk) * D;
+    src = k_tok + off_src;
+    vsrc = v_tok + off_src;
+    src_stride = (long long)num_kv_heads * D;
+    const long long off_dst = (((long long)phys * num_kv_heads + hk) * page_size + (long long)t * k_sub) * D;
+    dst = k_pool + off_dst;
+    vdst = v_pool + off_dst;
+    drow = kv;
+    dhi = k_hi;
+    dlo = k_lo;
+    rows = k_sub;
+  }
+  const int c = lane % LPR;
+  float acc[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+#pragma unroll 4
+  for (int r = lane / LPR; r < rows; r += RPI) {
+    const uint4 v = __ldg(reinterpret_cast<const uint4*>(src + (long long)r * src_stride) + c);
+    reinterpret_cast<uint4*>(dst + (long long)r * D)[c] = v;
+    if (vsrc) {
+      const uint4 vv = __ldg(reinterpret_cast<const uint4*>(vsrc + (long long)r * src_stride) + c);
+      reinterpret_cast<uint4*>(vdst + (long long)r * D)[c] = vv;
+    }
+    const __nv_bfloat162* hh = reinterpret_cast<const __nv_bfloat162*>(&v);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      float2 f = __bfloat1622float2(hh[i]);
+      acc[2 * i] += f.x;
+      acc[2 * i + 1] += f.y;
+    }
+  }
+  if (!pool) return;
+#pragma unroll
+  for (int off = LPR; off < 32; off <<= 1) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], off);
+  }
+  if (lane < LPR) {
+    const float inv = 1.0f / (float)rows;  // rows is a power of two: exact
+    float hi[8], lo[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const float x = acc[i] * inv;
+      hi[i] = to_tf32(x);
+      lo[i] = to_tf32(x - hi[i]);
+    }
+    float4* ph = reinterpret_cast<float4*>(dhi + drow * D) + 2 * c;
+    float4* pl = reinterpret_cast<float4*>(dlo + drow * D) + 2 * c;
+    ph[0] = make_float4(hi[0], hi[1], hi[2], hi[3]);
+    ph[1] = make_float4(hi[4], hi[5], hi[6], hi[7]);
+    pl[0] = make_float4(lo[0], lo[1], lo[2], lo[3]);
+    pl[1] = make_float4(lo[4], lo[5], lo[6], lo[7]);
+  }
+}
+
+// ---------------------------------------------------------------------------
 // K3: MaxNorm + HRM (from the page maxima) or caller-given scores, then
 // selection + ordering.  grid.x = nQB (heaviest first), grid.y = B * H_q, or
 // B * H_kv in group mode: one list for the G query heads of a KV head, from

@@ -168,6 +168,26 @@ cosa_status_t cosa_kap_rank(const cosa_shape_t* shape, const cosa_kap_params_t* 
                             int32_t* order, int32_t* count, float* scores, uint8_t* hrm,
                             void* workspace, size_t workspace_bytes, cosa_stream_t stream);
 
+/* The prefill's write of its attention inputs with Stage 1's downsampling fused in
+ * (gist.science/pt §2.2 "Ranking de Blocos": downsampling of queries and keys).  A
+ * prefill layer produces Q, K and V token-major; attention reads Q head-major and K
+ * and V from the paged cache.  This call does that write and, in the same pass over
+ * the rows, the pooling of cosa_kap_pool into the workspace, so Stage 1 needs no
+ * second read of Q and K: cosa_kap_rank on the same workspace then finishes it, and
+ * the result is bit-identical to cosa_kap_select on the written q and k_pool.
+ *   q_tok bf16 [B][N][H_q][D], k_tok / v_tok bf16 [B][N][H_kv][D] (inputs);
+ *   q bf16 [B][H_q][N][D], k_pool / v_pool bf16 [num_phys_pages][H_kv][P][D]
+ *   (outputs: the layouts above; every page the page table names for the
+ *   sequences' N tokens is written, others untouched; page-table entries of one
+ *   call must be distinct).
+ * workspace: a cosa_kap_select workspace (cosa_kap_workspace_size bytes, 256-byte
+ * aligned) for the pooled vectors, or NULL for the plain write without pooling.
+ * All buffers 16-byte aligned. */
+cosa_status_t cosa_prefill_write(const cosa_shape_t* shape, const cosa_kap_params_t* kap,
+                                 const void* q_tok, const void* k_tok, const void* v_tok,
+                                 const int32_t* page_table, void* q, void* k_pool, void* v_pool,
+                                 void* workspace, size_t workspace_bytes, cosa_stream_t stream);
+
 /* Proxy-bound pre-skip: a variant the pages do not give (their in-kernel skip,
  * gist.science/pt §2.3 "Saltado no Kernel", still pays every listed page its K
  * load and QK^T).  It applies the same kind of test one stage earlier, on the

@@ -201,3 +201,17 @@ def test_wait_fault_hook_argument_checks_on_host():
     # consumed by the next OSK call even when that call fails its own checks
     assert lib.cosa_osk_attention(None, None, None, None, None, None, None, None, 0, None, None,
                                   None, None, None) == 1
+
+
+def test_prefill_write_argument_checks_on_host():
+    lib = C.lib()
+    s = C.Shape(1, 4, 2, 256, 128, 64, 128).c()
+    k = C.KapParams(budget=0.2, q_sub=32, k_sub=16).c(C.Shape(1, 4, 2, 256, 128, 64, 128))
+    # a missing buffer, then a misaligned one, both before anything is launched
+    assert lib.cosa_prefill_write(ctypes.byref(s), ctypes.byref(k), None, 16, 16, 16, 16, 16, 16,
+                                  None, 0, None) == 1
+    assert lib.cosa_prefill_write(ctypes.byref(s), ctypes.byref(k), 8, 16, 16, 16, 16, 16, 16,
+                                  None, 0, None) == 1
+    # a workspace smaller than cosa_kap_workspace_size
+    assert lib.cosa_prefill_write(ctypes.byref(s), ctypes.byref(k), 16, 16, 16, 16, 16, 16, 16,
+                                  256, 16, None) == 5
