@@ -38,9 +38,11 @@ WORKLOAD = "gqa-128k"
 # of these kernels.  Each figure describes the kernel source the capture ran,
 # identified by a hash of the files below; any other source reports null.
 TRAFFIC = {
-    "osk": {"workload": "gqa-128k", "bytes": None, "source_sha256_16": None,
+    "osk": {"workload": "gqa-128k", "bytes": 1652187648 + 1034937088,
+            "source_sha256_16": "ff641ed0d6779605",
             "files": ("attn_tc.cuh", "tc_ptx.cuh", "common.cuh")},
-    "kap_pool": {"workload": "gqa-128k", "bytes": None, "source_sha256_16": None,
+    "kap_pool": {"workload": "gqa-128k", "bytes": 1342214656 + 183686656,
+                 "source_sha256_16": "7e8a9719a4f6b857",
                  "files": ("kap.cuh", "common.cuh")},
 }
 
@@ -430,6 +432,46 @@ def budget_sweep(C, W, dev, stream, burst, reps=3):
     return res
 
 
+def decode_leg(C, torch, x, shape, wl, order, count, dev, stream, eps_run, hbm, reps=20):
+    """Decode (the pages' future work): the last token of every head with the list KAP
+    wrote for its q-block, against the same kernel visiting every page."""
+    B, Hq, N, D = shape.batch, shape.num_q_heads, shape.seq_len, shape.head_dim
+    t = N - 1
+    P_ = wl.page_size
+    qdec = x["q"][:, :, t].contiguous()
+    pos = torch.full((B,), t, dtype=torch.int32, device=dev)
+    o_dec, c_dec = order[:, :, -1].contiguous(), count[:, :, -1].contiguous()
+    n_all = t // P_ + 1
+    o_full = torch.full((B, Hq, wl.num_pages), -1, dtype=torch.int32, device=dev)
+    o_full[:, :, :n_all] = torch.arange(n_all, dtype=torch.int32, device=dev)
+    c_full = torch.full((B, Hq), n_all, dtype=torch.int32, device=dev)
+    outd = torch.empty(B, Hq, D, dtype=torch.bfloat16, device=dev)
+    compd = torch.empty(B, Hq, dtype=torch.int32, device=dev)
+    wsd = torch.empty(C.cosa_osk_decode_workspace_size(shape, wl.num_pages), dtype=torch.uint8,
+                      device=dev)
+    page_bytes = P_ * D * 2
+    res = []
+    for label, o, c, eps in (("KAP list", o_dec, c_dec, eps_run), ("KAP list", o_dec, c_dec, 0.0),
+                             ("every page", o_full, c_full, 0.0)):
+        od = C.OskParams(eps=eps)
+        ms = _timed(lambda: C.cosa_osk_decode(shape, od, qdec, x["k_pool"], x["v_pool"],
+                                              x["page_table"], pos, o, c, outd, wsd,
+                                              computed=compd, stream=stream), reps, stream, warm=3)
+        if C.cosa_get_status(stream) != 0:
+            raise RuntimeError("in-kernel error status in decode")
+        listed = int(c.to(torch.int64).sum().item())
+        kept = int(compd.to(torch.int64).sum().item())
+        byts = (listed + kept) * page_bytes  # K of every listed page, V of every kept one
+        res.append({"list": label, "eps": eps, "us": ms * 1e3, "listed_pages": listed,
+                    "computed_pages": kept, "bytes": byts,
+                    "gbs": byts / (ms * 1e-3) / 1e9, "frac_vs_hbm": byts / (ms * 1e-3) / 1e9 / hbm})
+    for r in res:
+        r["speedup_vs_every_page"] = res[-1]["us"] / r["us"]
+    return {"position": t, "heads": B * Hq, "points": res,
+            "note": "bytes: K of the listed pages + V of the kept pages, read by each head "
+                    "(the G heads of a KV head share pages through L2)"}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -448,6 +490,8 @@ def main():
     ap.add_argument("--no-extras", action="store_true", help="skip dense/sweep/e2e/cpu legs")
     ap.add_argument("--sweep-only", action="store_true",
                     help="run only the per-budget sweep and print it")
+    ap.add_argument("--decode-only", action="store_true",
+                    help="time only the decode leg on the workload (for profiling it)")
     ap.add_argument("--dense-only", action="store_true",
                     help="time only the dense kernel on the workload (for profiling it)")
     args = ap.parse_args()
@@ -561,6 +605,14 @@ def main():
         step()
     torch.cuda.synchronize(dev)
     assert C.cosa_get_status(stream) == 0
+    if args.decode_only:
+        res = decode_leg(C, torch, x, shape, wl, order, count, dev, stream, args.eps, hbm,
+                         reps=args.steps)
+        if rank == 0:
+            print(json.dumps({"decode": res, "workload": args.workload}), flush=True)
+        if world > 1:
+            dist.destroy_process_group()
+        return 0
 
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
     clocks = ClockSampler(torch.cuda.current_device())
@@ -840,46 +892,9 @@ def main():
     except Exception as exc:  # an extra leg: report the failure, keep the line
         line["preskip"] = {"error": repr(exc)}
 
-    # ---- decode (the pages' future work): the last token of every head with the list
-    # KAP wrote for its q-block, against the same kernel visiting every page
-    def decode_leg():
-        t = N - 1
-        P_ = wl.page_size
-        qdec = x["q"][:, :, t].contiguous()
-        pos = torch.full((B,), t, dtype=torch.int32, device=dev)
-        o_dec, c_dec = order[:, :, -1].contiguous(), count[:, :, -1].contiguous()
-        n_all = t // P_ + 1
-        o_full = torch.full((B, Hq, wl.num_pages), -1, dtype=torch.int32, device=dev)
-        o_full[:, :, :n_all] = torch.arange(n_all, dtype=torch.int32, device=dev)
-        c_full = torch.full((B, Hq), n_all, dtype=torch.int32, device=dev)
-        outd = torch.empty(B, Hq, D, dtype=torch.bfloat16, device=dev)
-        compd = torch.empty(B, Hq, dtype=torch.int32, device=dev)
-        wsd = torch.empty(C.cosa_osk_decode_workspace_size(shape, wl.num_pages), dtype=torch.uint8,
-                          device=dev)
-        page_bytes = P_ * D * 2
-        res = []
-        for label, o, c, eps in (("KAP list", o_dec, c_dec, args.eps), ("KAP list", o_dec, c_dec, 0.0),
-                                 ("every page", o_full, c_full, 0.0)):
-            od = C.OskParams(eps=eps)
-            ms = _timed(lambda: C.cosa_osk_decode(shape, od, qdec, x["k_pool"], x["v_pool"],
-                                                  x["page_table"], pos, o, c, outd, wsd,
-                                                  computed=compd, stream=stream), 20, stream, warm=3)
-            if C.cosa_get_status(stream) != 0:
-                raise RuntimeError("in-kernel error status in decode")
-            listed = int(c.to(torch.int64).sum().item())
-            kept = int(compd.to(torch.int64).sum().item())
-            byts = (listed + kept) * page_bytes  # K of every listed page, V of every kept one
-            res.append({"list": label, "eps": eps, "us": ms * 1e3, "listed_pages": listed,
-                        "computed_pages": kept, "bytes": byts,
-                        "gbs": byts / (ms * 1e-3) / 1e9, "frac_vs_hbm": byts / (ms * 1e-3) / 1e9 / hbm})
-        for r in res:
-            r["speedup_vs_every_page"] = res[-1]["us"] / r["us"]
-        return {"position": t, "heads": B * Hq, "points": res,
-                "note": "bytes: K of the listed pages + V of the kept pages, read by each head "
-                        "(the G heads of a KV head share pages through L2)"}
-
     try:
-        line["decode"] = decode_leg()
+        line["decode"] = decode_leg(C, torch, x, shape, wl, order, count, dev, stream, args.eps,
+                                    hbm)
     except Exception as exc:  # an extra leg: report the failure, keep the line
         line["decode"] = {"error": repr(exc)}
 
