@@ -294,7 +294,7 @@ struct KapPageMax {
 constexpr int ORDER_MAX_ROWS = 64;  // representative rows read by one CTA (G * R in group mode)
 
 template <bool FROM_A, bool GROUP>
-__global__ void __launch_bounds__(ORDER_THREADS) kap_order_kernel(
+__global__ void __launch_bounds__(ORDER_THREADS, 3) kap_order_kernel(
     const float* __restrict__ scores, const uint8_t* __restrict__ hrm, KapPageMax pm,
     float* __restrict__ scores_out, uint8_t* __restrict__ hrm_out, int32_t* __restrict__ order,
     int32_t* __restrict__ count, int num_q_heads, int num_q_blocks, int num_pages, int q_block,
@@ -351,14 +351,23 @@ __global__ void __launch_bounds__(ORDER_THREADS) kap_order_kernel(
       int flag;
       if (FROM_A) {
         // MaxNorm: S[p] = mean_r exp(a[r][p] - m_r); HRM: p is some row's first
-        // maximum (group mode: the largest head score, any head's flag)
+        // maximum (group mode: the largest head score, any head's flag).  A head's
+        // R <= 8 page maxima are loaded together, then summed in row order.
         sv = 0.f;
         flag = 0;
         for (int g = 0; g < n_heads; ++g) {
+          float av[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            av[i] = i < pm.R ? arow[(long long)(g * pm.R + i) * n_b + p] : 0.f;
           float sg = 0.f;
-          for (int r = g * pm.R; r < (g + 1) * pm.R; ++r) {
-            sg += expf(arow[(long long)r * n_b + p] - m_s[r]);
-            flag |= (arg_s[r] == p);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            if (i < pm.R) {
+              const int r = g * pm.R + i;
+              sg += expf(av[i] - m_s[r]);
+              flag |= (arg_s[r] == p);
+            }
           }
           sv = fmaxf(sv, sg * invR);
         }
@@ -465,50 +474,62 @@ __global__ void __launch_bounds__(ORDER_THREADS) kap_order_kernel(
     for (int p = beg; p < beg + per && p < n_b; ++p)
       if (selected(p)) orow[pos++] = p;
   } else {
-    // kept keys only, then a bitonic sort (descending) of those
+    // kept keys only, then a sort (descending) of those
     unsigned long long* kept = keys + npow2;
     int m = 1;
     while (m < total) m <<= 1;
     for (int p = beg; p < beg + per && p < n_b; ++p)
       if (selected(p)) kept[pos++] = keys[p];
-    const int mw = m < 32 ? 32 : m;  // whole warps take part in the register stages
-    for (int i = total + threadIdx.x; i < mw; i += blockDim.x) kept[i] = 0ull;  // below every key
-    __syncthreads();
-    // Bitonic sort, descending.  Stages pairing elements 32 or more apart go through
-    // shared memory; the others pair lanes of one warp and run in registers (element i
-    // is held by lane i % 32 of its warp; the partner of i is i ^ j).
-    auto warp_stages = [&](int k_lo, int k_hi) {
-      for (int i0 = 0; i0 < mw; i0 += blockDim.x) {
-        const int i = i0 + (int)threadIdx.x;
-        if (i >= mw) continue;  // whole warps: mw and blockDim are multiples of 32
-        unsigned long long x = kept[i];
-        for (int kk = k_lo; kk <= k_hi; kk <<= 1)
-          for (int j = (kk >> 1) < 16 ? (kk >> 1) : 16; j > 0; j >>= 1) {
-            const unsigned long long y = __shfl_xor_sync(0xffffffffu, x, j);
-            const bool keep_max = ((i & j) == 0) == ((i & kk) == 0);
-            x = keep_max ? (x > y ? x : y) : (x < y ? x : y);
-          }
-        kept[i] = x;
-      }
+    if (total <= (int)blockDim.x) {
+      // up to one key per thread: a key's place is the number of larger keys (the
+      // keys are distinct: the page is in the low bits), read by broadcast
       __syncthreads();
-    };
-    if (m >= 2) warp_stages(2, m < 32 ? m : 32);  // every size up to 32 at once
-    for (int kk = 64; kk <= m; kk <<= 1) {
-      for (int j = kk >> 1; j >= 32; j >>= 1) {
-        for (int i = threadIdx.x; i < m; i += blockDim.x) {
-          const int ixj = i ^ j;
-          if (ixj > i) {
-            const unsigned long long x = kept[i], y = kept[ixj];
-            const bool desc = (i & kk) == 0;
-            if (desc ? (x < y) : (x > y)) { kept[i] = y; kept[ixj] = x; }
-          }
+      if ((int)threadIdx.x < total) {
+        const unsigned long long mine = kept[threadIdx.x];
+        int rank = 0;
+        for (int k = 0; k < total; ++k) rank += kept[k] > mine;
+        orow[rank] = 0x7fffffff - (int)(mine & 0x7fffffffull);
+      }
+    } else {
+      const int mw = m < 32 ? 32 : m;  // whole warps take part in the register stages
+      for (int i = total + threadIdx.x; i < mw; i += blockDim.x) kept[i] = 0ull;  // below every key
+      __syncthreads();
+      // Bitonic sort, descending.  Stages pairing elements 32 or more apart go through
+      // shared memory; the others pair lanes of one warp and run in registers (element i
+      // is held by lane i % 32 of its warp; the partner of i is i ^ j).
+      auto warp_stages = [&](int k_lo, int k_hi) {
+        for (int i0 = 0; i0 < mw; i0 += blockDim.x) {
+          const int i = i0 + (int)threadIdx.x;
+          if (i >= mw) continue;  // whole warps: mw and blockDim are multiples of 32
+          unsigned long long x = kept[i];
+          for (int kk = k_lo; kk <= k_hi; kk <<= 1)
+            for (int j = (kk >> 1) < 16 ? (kk >> 1) : 16; j > 0; j >>= 1) {
+              const unsigned long long y = __shfl_xor_sync(0xffffffffu, x, j);
+              const bool keep_max = ((i & j) == 0) == ((i & kk) == 0);
+              x = keep_max ? (x > y ? x : y) : (x < y ? x : y);
+            }
+          kept[i] = x;
         }
         __syncthreads();
+      };
+      if (m >= 2) warp_stages(2, m < 32 ? m : 32);  // every size up to 32 at once
+      for (int kk = 64; kk <= m; kk <<= 1) {
+        for (int j = kk >> 1; j >= 32; j >>= 1) {
+          for (int i = threadIdx.x; i < m; i += blockDim.x) {
+            const int ixj = i ^ j;
+            if (ixj > i) {
+              const unsigned long long x = kept[i], y = kept[ixj];
+              const bool desc = (i & kk) == 0;
+              if (desc ? (x < y) : (x > y)) { kept[i] = y; kept[ixj] = x; }
+            }
+          }
+          __syncthreads();
+        }
+        warp_stages(kk, kk);
       }
-      warp_stages(kk, kk);
+      for (int i = threadIdx.x; i < total; i += blockDim.x)
+        orow[i] = 0x7fffffff - (int)(kept[i] & 0x7fffffffull);
     }
-    for (int i = threadIdx.x; i < total; i += blockDim.x)
-      orow[i] = 0x7fffffff - (int)(kept[i] & 0x7fffffffull);
   }
   for (int j = total + threadIdx.x; j < k_cap; j += blockDim.x) orow[j] = -1;
   if (threadIdx.x == 0) {
