@@ -553,35 +553,17 @@ __global__ void __launch_bounds__(TcCfg<D, P>::NT, 1)
     bool ok = true;     // OSK: collective within the warpgroup
     bool fail = false;  // this warp missed a wait after the vote; reported at the next vote
     // Page ids of list entries [fb, fb + 32) (lane l: entry fb + l) in pid_l and, in the
-    // leading warp, their TMA coordinates in cz_l.  The next block's ids and coordinates
-    // (pid_1, cz_1) and the ids of the block after it (pid_2) are loaded ahead, so that
-    // moving on to a new block waits on no global load.
-    int fb = -1, pid_l = 0, cz_l = 0, pid_1 = 0, cz_1 = 0, pid_2 = 0;
-    auto ids_of = [&](int base) {
-      const int jl = base + lane;
-      return jl < n_list ? page_at(jl) : 0;
-    };
-    auto coords_of = [&](int base, int pid) {
-      const int jl = base + lane;
-      return (lead_warp && jl < n_list) ? coord_of(pid) : 0;
-    };
+    // leading warp, their TMA coordinates in cz_l, loaded when the list reaches a new
+    // block of 32 (loading the next block ahead was measured 4 % slower)
+    int fb = -1, pid_l = 0, cz_l = 0;
     // page id (and, in the leading warp, TMA coordinate) of list entry j; j only grows
     auto fetch = [&](int j, int& cz) -> int {
       const int base = j & ~31;
       if (base != fb) {
-        if (base == fb + 32) {  // the block loaded ahead
-          pid_l = pid_1;
-          cz_l = cz_1;
-          pid_1 = pid_2;
-          cz_1 = coords_of(base + 32, pid_1);
-        } else {  // first block: loaded here
-          pid_l = ids_of(base);
-          cz_l = coords_of(base, pid_l);
-          pid_1 = ids_of(base + 32);
-          cz_1 = coords_of(base + 32, pid_1);
-        }
-        pid_2 = ids_of(base + 64);
         fb = base;
+        const int jl = base + lane;
+        pid_l = jl < n_list ? page_at(jl) : 0;
+        if (lead_warp) cz_l = jl < n_list ? coord_of(pid_l) : 0;
       }
       cz = __shfl_sync(0xffffffffu, cz_l, j & 31);
       return __shfl_sync(0xffffffffu, pid_l, j & 31);
