@@ -368,7 +368,7 @@ TcParams make_params(const cosa_shape_t* s, void* out, float* lse, const int32_t
 // Workspace of cosa_osk_decode: the listed pages' logits and local maxima, and the
 // per-chunk partial sums.
 struct DecodeLayout {
-  size_t logits, mloc, po, pl, pn, total;
+  size_t logits, mloc, po, pl, pn, arr, total;
   int n_chunks;
 };
 
@@ -387,6 +387,8 @@ DecodeLayout decode_layout(const cosa_shape_t* s, int k_cap) {
   off = align256(off + bh * L.n_chunks * sizeof(float));
   L.pn = off;
   off = align256(off + bh * L.n_chunks * sizeof(int));
+  L.arr = off;
+  off = align256(off + bh * sizeof(int));
   L.total = off;
   return L;
 }
@@ -397,8 +399,6 @@ cosa_status_t launch_decode_t(const DecodeParams& prm, int bh, cudaStream_t st) 
   decode_qk_kernel<D, P><<<grid, DEC_THREADS, 0, st>>>(prm);
   if (last_launch() != COSA_OK) return COSA_ERR_CUDA;
   decode_pv_kernel<D, P><<<grid, DEC_THREADS, 0, st>>>(prm);
-  if (last_launch() != COSA_OK) return COSA_ERR_CUDA;
-  decode_combine_kernel<D><<<bh, 128, 0, st>>>(prm);
   return last_launch();
 }
 
@@ -921,6 +921,7 @@ cosa_status_t cosa_osk_decode(const cosa_shape_t* shape, const cosa_osk_params_t
   prm.part_o = reinterpret_cast<float*>(ws + L.po);
   prm.part_l = reinterpret_cast<float*>(ws + L.pl);
   prm.part_n = reinterpret_cast<int*>(ws + L.pn);
+  prm.arrived = reinterpret_cast<int*>(ws + L.arr);
   prm.num_q_heads = shape->num_q_heads;
   prm.num_kv_heads = shape->num_kv_heads;
   prm.group = shape->num_q_heads / shape->num_kv_heads;

@@ -11,8 +11,9 @@
 //                      in, log2 units, keys past the query masked) into the
 //                      workspace, and the page's local max
 //   decode_pv_kernel   per chunk of the list: the decisions, then the kept pages'
-//                      exp2(s - M) V and row sum against M, the list's final max
-//   decode_combine_kernel   the chunks' partial sums to O / l, LSE, counts
+//                      exp2(s - M) V and row sum against M, the list's final max;
+//                      the chunk that finishes last for its head adds the chunks'
+//                      partial sums to O / l, the LSE and the computed count
 // For eps <= 1 a skipped page's local max lies below the running max, so the
 // running max before list position j is the max of the local maxima of all pages
 // listed before j: every decision is known from the local maxima alone, and M, the
@@ -42,6 +43,7 @@ struct DecodeParams {
   float* part_o;                // workspace [B H_q][n_chunks][D]
   float* part_l;                // workspace [B H_q][n_chunks]
   int* part_n;                  // workspace [B H_q][n_chunks]
+  int* arrived;                 // workspace [B H_q]: chunks of the head done (reset by the logits pass)
   int num_q_heads, num_kv_heads, group, seq_len, pages_per_seq, k_cap, n_chunks;
   float scale_log2, log2_eps;
 };
@@ -72,11 +74,23 @@ __global__ void __launch_bounds__(DEC_THREADS) decode_qk_kernel(const DecodePara
   const int b = (int)(bh / p.num_q_heads), h = (int)(bh % p.num_q_heads);
   const int hk = h / p.group;
   const int t = __ldg(p.positions + b);
-  if (t < 0 || t >= p.seq_len) {
-    if (threadIdx.x == 0 && blockIdx.x == 0) set_status(COSA_ERR_INVALID_ARG);
-    return;
+  const bool t_ok = t >= 0 && t < p.seq_len;
+  const int n = t_ok ? min(max(__ldg(p.count + bh), 0), p.k_cap) : 0;
+  if (blockIdx.x == 0) {
+    // the P V pass counts this head's chunks in; a head with nothing to visit (an
+    // empty list, or a position out of range: reported) gets its outputs here
+    if (threadIdx.x == 0) {
+      p.arrived[bh] = 0;
+      if (!t_ok) set_status(COSA_ERR_INVALID_ARG);
+      if (n == 0) {
+        if (p.lse) p.lse[bh] = -INFINITY;
+        if (p.computed) p.computed[bh] = 0;
+      }
+    }
+    if (n == 0)
+      for (int d = threadIdx.x; d < D; d += DEC_THREADS) p.out[bh * D + d] = __float2bfloat16_rn(0.f);
   }
-  const int n = min(max(__ldg(p.count + bh), 0), p.k_cap);
+  if (n == 0) return;
   // this lane's 8 query dims (scale and log2 e folded in)
   float qv[8];
   {
@@ -247,6 +261,7 @@ __global__ void __launch_bounds__(DEC_THREADS) decode_pv_kernel(const DecodePara
     for (int w = 0; w < DEC_WARPS; ++w) v += o_s[w][d];
     p.part_o[pc * D + d] = v;
   }
+  __shared__ int last_s;
   if (threadIdx.x == 0) {
     float l = 0.f;
     int kept = 0;
@@ -256,35 +271,37 @@ __global__ void __launch_bounds__(DEC_THREADS) decode_pv_kernel(const DecodePara
     p.part_l[pc] = l;
     p.part_n[pc] = kept;
   }
-}
-
-template <int D>
-__global__ void __launch_bounds__(128) decode_combine_kernel(const DecodeParams p) {
-  const long long bh = blockIdx.x;
-  const int b = (int)(bh / p.num_q_heads);
-  const int t = __ldg(p.positions + b);
-  const bool ok = t >= 0 && t < p.seq_len;
-  const int n = ok ? min(max(__ldg(p.count + bh), 0), p.k_cap) : 0;
-  const int nc = (n + DEC_CHUNK - 1) / DEC_CHUNK;
-  float l = 0.f;
-  int kept = 0;
-  for (int c = 0; c < nc; ++c) {
-    l += p.part_l[bh * p.n_chunks + c];
-    kept += p.part_n[bh * p.n_chunks + c];
-  }
-  const float inv = l > 0.f ? 1.f / l : 0.f;
-  for (int d = threadIdx.x; d < D; d += blockDim.x) {
-    float o = 0.f;
-    for (int c = 0; c < nc; ++c) o += p.part_o[(bh * p.n_chunks + c) * D + d];
-    p.out[bh * D + d] = __float2bfloat16_rn(o * inv);
-  }
+  // the chunk that finishes last for this head combines (every chunk's partial sums
+  // are made visible before it counts itself in)
+  __syncthreads();
   if (threadIdx.x == 0) {
-    if (p.computed) p.computed[bh] = kept;
-    if (p.lse) {
-      float m = -INFINITY;
-      for (int j = 0; j < n; ++j) m = fmaxf(m, p.mloc[bh * p.k_cap + j]);
-      p.lse[bh] = l > 0.f ? (m + log2f(l)) * 0.69314718055994531f : -INFINITY;
+    __threadfence();
+    const int nc = (n + DEC_CHUNK - 1) / DEC_CHUNK;
+    last_s = atomicAdd(p.arrived + bh, 1) == nc - 1;
+    if (last_s) __threadfence();
+  }
+  __syncthreads();
+  if (!last_s) return;
+  const int nc = (n + DEC_CHUNK - 1) / DEC_CHUNK;
+  const long long pc0 = bh * p.n_chunks;
+  __shared__ float l_tot;
+  if (threadIdx.x == 0) {
+    float l = 0.f;
+    int kept = 0;
+    for (int c = 0; c < nc; ++c) {
+      l += ((volatile float*)p.part_l)[pc0 + c];
+      kept += ((volatile int*)p.part_n)[pc0 + c];
     }
+    l_tot = l;
+    if (p.computed) p.computed[bh] = kept;
+    if (p.lse) p.lse[bh] = l > 0.f ? (ma + log2f(l)) * 0.69314718055994531f : -INFINITY;
+  }
+  __syncthreads();
+  const float inv = l_tot > 0.f ? 1.f / l_tot : 0.f;
+  for (int d = threadIdx.x; d < D; d += DEC_THREADS) {
+    float o = 0.f;
+    for (int c = 0; c < nc; ++c) o += ((volatile float*)p.part_o)[(pc0 + c) * D + d];
+    p.out[bh * D + d] = __float2bfloat16_rn(o * inv);
   }
 }
 
