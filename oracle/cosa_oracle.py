@@ -368,8 +368,9 @@ def expand_group_order(order_g: np.ndarray, count_g: np.ndarray, num_q_heads: in
 # its K load and QK^T.  This variant applies the same kind of test one stage
 # earlier, on the proxy's page maxima a[r][p] (kap_block_scores) and the proxy's
 # own running max along the ordered list, and removes the pages it rejects from
-# the list, so the kernel never visits them.  Reading (the plainest one the
-# spec example allows): along the list L = (p_0, p_1, ...),
+# the list, so the kernel never visits them.  Reading (a proxy-estimated logit
+# compared with a running max, in its plainest form): along the list
+# L = (p_0, p_1, ...),
 #   ahat_r(j) = max over positions j' < j of a[r][p_j'];
 #   representative r keeps position j iff a[r][p_j] > -inf and (ahat_r(j) = -inf
 #     or a[r][p_j] + margin - ahat_r(j) >= ln(eps));
