@@ -22,7 +22,7 @@ LSE_ABS = 2e-3
 # Skip decisions: the kernel decides in fp32 (log2 domain), the oracle in
 # float64 (natural log).  A tile whose float64 margin |max_i d_i - ln eps| is
 # below this many nats may legitimately go either way.
-SKIP_MARGIN = 2e-3
+SKIP_MARGIN = 1e-3
 
 
 def shape_of(wl: W.Workload, x: dict) -> C.Shape:
