@@ -41,8 +41,8 @@ TRAFFIC = {
     "osk": {"workload": "gqa-128k", "bytes": 1652753920 + 1035382784,
             "source_sha256_16": "58ec01c35dcc6e5a",
             "files": ("attn_tc.cuh", "tc_ptx.cuh", "common.cuh")},
-    "kap_pool": {"workload": "gqa-128k", "bytes": 1342216192 + 183949568,
-                 "source_sha256_16": "6c846c1eb0b2207e",
+    "kap_pool": {"workload": "gqa-128k", "bytes": 1342215168 + 184500224,
+                 "source_sha256_16": "db13d4d202b518c7",
                  "files": ("kap.cuh", "common.cuh")},
 }
 

@@ -204,7 +204,8 @@ cosa_status_t launch_pool(const cosa_shape_t* s, const cosa_kap_params_t* k, con
       reinterpret_cast<const __nv_bfloat16*>(q), reinterpret_cast<const __nv_bfloat16*>(k_pool),
       page_table, reinterpret_cast<float*>(ws + L.q_hi), reinterpret_cast<float*>(ws + L.q_lo),
       reinterpret_cast<float*>(ws + L.k_hi), reinterpret_cast<float*>(ws + L.k_lo), n_qvec,
-      k->q_sub, n_kvec, k->k_sub, Hq, Hk, G, R, nQB, P, nP, s->pages_per_seq, T);
+      k->q_sub, n_kvec, k->k_sub, Hq, Hk, G, R, nQB, P, nP, s->pages_per_seq,
+      s->num_phys_pages, T);
   return last_launch();
 }
 
@@ -679,7 +680,7 @@ cosa_status_t cosa_prefill_write(const cosa_shape_t* shape, const cosa_kap_param
         static_cast<const bf*>(q_tok), static_cast<const bf*>(k_tok), static_cast<const bf*>(v_tok),
         page_table, static_cast<bf*>(q), static_cast<bf*>(k_pool), static_cast<bf*>(v_pool), f[0],
         f[1], f[2], f[3], n_qvec, kap->q_sub, n_kvec, kap->k_sub, Hq, Hk, G, R, nQB, P, nP,
-        shape->pages_per_seq, T, N);
+        shape->pages_per_seq, shape->num_phys_pages, T, N);
   };
   if (shape->head_dim == 128) args(prefill_write_kernel<128>);
   else args(prefill_write_kernel<64>);
@@ -927,6 +928,7 @@ cosa_status_t cosa_osk_decode(const cosa_shape_t* shape, const cosa_osk_params_t
   prm.group = shape->num_q_heads / shape->num_kv_heads;
   prm.seq_len = shape->seq_len;
   prm.pages_per_seq = shape->pages_per_seq;
+  prm.num_phys_pages = shape->num_phys_pages;
   prm.k_cap = k_cap;
   prm.n_chunks = L.n_chunks;
   prm.scale_log2 = shape->softmax_scale * 1.4426950408889634f;
@@ -988,6 +990,12 @@ cosa_status_t cosa_attention_host(const cosa_shape_t* shape, const cosa_kap_para
     return COSA_ERR_INVALID_ARG;
   if (!workspace || workspace_bytes < L.total || reinterpret_cast<uintptr_t>(workspace) % 256)
     return COSA_ERR_WORKSPACE;
+  // the page table is on the host here, so its entries are checked before anything is queued
+  for (int b = 0; b < shape->batch; ++b)
+    for (int p = 0; p < shape->seq_len / shape->page_size; ++p) {
+      const int32_t v = page_table_host[static_cast<size_t>(b) * shape->pages_per_seq + p];
+      if (v < 0 || v >= shape->num_phys_pages) return COSA_ERR_INVALID_ARG;
+    }
   const int B = shape->batch, Hq = shape->num_q_heads, Hkv = shape->num_kv_heads, G = Hq / Hkv;
   const size_t head_bytes = static_cast<size_t>(shape->seq_len) * shape->head_dim * 2;  // one (b, h)
   const size_t page_bytes = static_cast<size_t>(shape->page_size) * shape->head_dim * 2;

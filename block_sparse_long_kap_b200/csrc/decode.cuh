@@ -44,7 +44,7 @@ struct DecodeParams {
   float* part_l;                // workspace [B H_q][n_chunks]
   int* part_n;                  // workspace [B H_q][n_chunks]
   int* arrived;                 // workspace [B H_q]: chunks of the head done (reset by the logits pass)
-  int num_q_heads, num_kv_heads, group, seq_len, pages_per_seq, k_cap, n_chunks;
+  int num_q_heads, num_kv_heads, group, seq_len, pages_per_seq, num_phys_pages, k_cap, n_chunks;
   float scale_log2, log2_eps;
 };
 
@@ -111,6 +111,13 @@ __global__ void __launch_bounds__(DEC_THREADS) decode_qk_kernel(const DecodePara
       continue;
     }
     const int phys = __ldg(p.page_table + (long long)b * p.pages_per_seq + pg);
+    if (phys < 0 || phys >= p.num_phys_pages) {  // outside the pool: reported, not read
+      if (lane == 0) {
+        set_status(COSA_ERR_INVALID_ARG);
+        p.mloc[bh * p.k_cap + j] = -INFINITY;
+      }
+      continue;
+    }
     const uint4* kp = reinterpret_cast<const uint4*>(
         p.k_pool + ((long long)phys * p.num_kv_heads + hk) * P * D);
     float* lrow = p.logits + (bh * p.k_cap + j) * P;
@@ -216,6 +223,7 @@ __global__ void __launch_bounds__(DEC_THREADS) decode_pv_kernel(const DecodePara
     const int pg = __ldg(p.order + bh * p.k_cap + j);
     if (pg < 0 || pg > t / P) continue;  // an invalid entry (reported by the logits pass)
     const int phys = __ldg(p.page_table + (long long)b * p.pages_per_seq + pg);
+    if (phys < 0 || phys >= p.num_phys_pages) continue;  // reported by the logits pass
     const uint4* vp = reinterpret_cast<const uint4*>(
         p.v_pool + ((long long)phys * p.num_kv_heads + hk) * P * D);
     const float* lrow = p.logits + (bh * p.k_cap + j) * P;

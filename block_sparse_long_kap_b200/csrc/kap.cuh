@@ -56,7 +56,8 @@ __global__ void __launch_bounds__(256) kap_pool_kernel(
     const int32_t* __restrict__ page_table, float* __restrict__ q_hi, float* __restrict__ q_lo,
     float* __restrict__ k_hi, float* __restrict__ k_lo, long long n_qvec, int q_sub,
     long long n_kvec, int k_sub, int num_q_heads, int num_kv_heads, int group, int R,
-    int num_q_blocks, int page_size, int num_pages, int pages_per_seq, int T) {
+    int num_q_blocks, int page_size, int num_pages, int pages_per_seq, int num_phys_pages,
+    int T) {
   constexpr int LPR = D / 8;     // lanes per row: each lane loads 8 bf16 (16 B)
   constexpr int RPI = 32 / LPR;  // rows covered per warp-wide load
   const int lane = threadIdx.x & 31;
@@ -64,7 +65,7 @@ __global__ void __launch_bounds__(256) kap_pool_kernel(
   const __nv_bfloat16* src;
   long long drow;
   float *dhi, *dlo;
-  int rows;
+  int rows, n_read;
   if (w < n_qvec) {
     src = q + w * (long long)q_sub * D;
     const int r = (int)(w % R);
@@ -77,7 +78,7 @@ __global__ void __launch_bounds__(256) kap_pool_kernel(
     drow = ((long long)(b * num_kv_heads + hk) * num_q_blocks + qb) * (group * R) + g * R + r;
     dhi = q_hi;
     dlo = q_lo;
-    rows = q_sub;
+    n_read = rows = q_sub;
   } else {
     const long long kv = w - n_qvec;
     if (kv >= n_kvec) return;
@@ -88,18 +89,24 @@ __global__ void __launch_bounds__(256) kap_pool_kernel(
     const int hk = (int)(r % num_kv_heads);
     const int b = (int)(r / num_kv_heads);
     const int phys = page_table[(long long)b * pages_per_seq + p];
-    src = k_pool + (((long long)phys * num_kv_heads + hk) * page_size + (long long)t * k_sub) * D;
+    n_read = rows = k_sub;
+    if (phys < 0 || phys >= num_phys_pages) {  // outside the pool: reported, not read
+      if (lane == 0) set_status(COSA_ERR_INVALID_ARG);
+      n_read = 0;  // the pooled vector is written as zero
+      src = k_pool;
+    } else {
+      src = k_pool + (((long long)phys * num_kv_heads + hk) * page_size + (long long)t * k_sub) * D;
+    }
     drow = kv;
     dhi = k_hi;
     dlo = k_lo;
-    rows = k_sub;
   }
   const int c = lane % LPR;
   float acc[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) acc[i] = 0.f;
 #pragma unroll 4
-  for (int r = lane / LPR; r < rows; r += RPI) {
+  for (int r = lane / LPR; r < n_read; r += RPI) {
     uint4 v = __ldg(reinterpret_cast<const uint4*>(src + (long long)r * D) + c);
     const __nv_bfloat162* hh = reinterpret_cast<const __nv_bfloat162*>(&v);
 #pragma unroll
@@ -152,7 +159,8 @@ __global__ void __launch_bounds__(256) prefill_write_kernel(
     __nv_bfloat16* __restrict__ v_pool, float* __restrict__ q_hi, float* __restrict__ q_lo,
     float* __restrict__ k_hi, float* __restrict__ k_lo, long long n_qvec, int q_sub,
     long long n_kvec, int k_sub, int num_q_heads, int num_kv_heads, int group, int R,
-    int num_q_blocks, int page_size, int num_pages, int pages_per_seq, int T, int seq_len) {
+    int num_q_blocks, int page_size, int num_pages, int pages_per_seq, int num_phys_pages,
+    int T, int seq_len) {
   constexpr int LPR = D / 8;     // lanes per row: each lane moves 8 bf16 (16 B)
   constexpr int RPI = 32 / LPR;  // rows covered per warp-wide load
   const int lane = threadIdx.x & 31;
@@ -196,9 +204,15 @@ __global__ void __launch_bounds__(256) prefill_write_kernel(
     src = k_tok + off_src;
     vsrc = v_tok + off_src;
     src_stride = (long long)num_kv_heads * D;
-    const long long off_dst = (((long long)phys * num_kv_heads + hk) * page_size + (long long)t * k_sub) * D;
-    dst = k_pool + off_dst;
-    vdst = v_pool + off_dst;
+    if (phys < 0 || phys >= num_phys_pages) {  // outside the pool: reported, not written
+      if (lane == 0) set_status(COSA_ERR_INVALID_ARG);
+      dst = nullptr;  // the pooled vector still comes from the rows read
+    } else {
+      const long long off_dst =
+          (((long long)phys * num_kv_heads + hk) * page_size + (long long)t * k_sub) * D;
+      dst = k_pool + off_dst;
+      vdst = v_pool + off_dst;
+    }
     drow = kv;
     dhi = k_hi;
     dlo = k_lo;
@@ -211,8 +225,8 @@ __global__ void __launch_bounds__(256) prefill_write_kernel(
 #pragma unroll 4
   for (int r = lane / LPR; r < rows; r += RPI) {
     const uint4 v = __ldg(reinterpret_cast<const uint4*>(src + (long long)r * src_stride) + c);
-    reinterpret_cast<uint4*>(dst + (long long)r * D)[c] = v;
-    if (vsrc) {
+    if (dst) reinterpret_cast<uint4*>(dst + (long long)r * D)[c] = v;
+    if (vdst) {
       const uint4 vv = __ldg(reinterpret_cast<const uint4*>(vsrc + (long long)r * src_stride) + c);
       reinterpret_cast<uint4*>(vdst + (long long)r * D)[c] = vv;
     }

@@ -43,8 +43,14 @@
  *   - Supported shapes (COSA_ERR_UNSUPPORTED otherwise): D = 128 (all kernels)
  *     or D = 64 (KAP and the attention kernels); P in {64, 128};
  *     Bq in {64, 128}; N a multiple of P and of Bq; H_q a multiple of H_kv;
- *     page_table entries in [0, num_phys_pages) (not checked: the caller's
- *     contract, as for any index buffer).
+ *     page_table entries in [0, num_phys_pages).  The kernels that address
+ *     pages with plain loads and stores (KAP's pooling, cosa_prefill_write,
+ *     cosa_osk_decode) check every entry they use: one outside the pool is
+ *     recorded as COSA_ERR_INVALID_ARG in the status word and that page is
+ *     neither read nor written (its pooled key vectors are zero; decode treats
+ *     the list entry as invalid).  The TMA kernels (OSK, dense) read such a
+ *     page as zeros, and cosa_attention_host checks its host page table before
+ *     anything is queued.
  */
 #ifndef COSA_H_
 #define COSA_H_
@@ -312,8 +318,10 @@ cosa_status_t cosa_osk_decode_workspace_size(const cosa_shape_t* shape, int32_t 
  * otherwise).  out bf16 [B][H_q][D]; lse fp32 [B][H_q], computed int32 [B][H_q]
  * and skip_log uint8 [B][H_q][k_cap] may be NULL.  workspace: at least
  * cosa_osk_decode_workspace_size(shape, k_cap) bytes, 256-byte aligned.  A list
- * entry past the query's page, or a position out of range, is never read: it is
- * recorded as COSA_ERR_INVALID_ARG in the status word. */
+ * entry past the query's page or naming a physical page outside the pool, or a
+ * position out of range, is never read: it is recorded as COSA_ERR_INVALID_ARG
+ * in the status word (an empty list, or a position out of range, gives a zero
+ * output, lse -inf and 0 computed). */
 cosa_status_t cosa_osk_decode(const cosa_shape_t* shape, const cosa_osk_params_t* osk,
                               const void* q, const void* k_pool, const void* v_pool,
                               const int32_t* page_table, const int32_t* positions,
@@ -349,7 +357,8 @@ cosa_status_t cosa_attention_host_workspace_size(const cosa_shape_t* shape,
  * The host buffers must stay valid and unmodified until `stream` reaches the end
  * of this call's work.  workspace: device buffer of at least
  * cosa_attention_host_workspace_size bytes, 256-byte aligned.  Argument errors
- * return before anything is queued; a failed CUDA call returns COSA_ERR_CUDA
+ * (a page_table_host entry outside [0, num_phys_pages) among them:
+ * COSA_ERR_INVALID_ARG) return before anything is queued; a failed CUDA call returns COSA_ERR_CUDA
  * with the work queued so far still joined to `stream`; in-kernel errors go to
  * the status word as for the stage calls. */
 cosa_status_t cosa_attention_host(const cosa_shape_t* shape, const cosa_kap_params_t* kap,

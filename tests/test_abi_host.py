@@ -215,3 +215,27 @@ def test_prefill_write_argument_checks_on_host():
     # a workspace smaller than cosa_kap_workspace_size
     assert lib.cosa_prefill_write(ctypes.byref(s), ctypes.byref(k), 16, 16, 16, 16, 16, 16, 16,
                                   256, 16, None) == 5
+
+
+def test_host_pipeline_checks_its_host_page_table():
+    """cosa_attention_host reads its page table on the host: an entry outside
+    [0, num_phys_pages) returns COSA_ERR_INVALID_ARG before any CUDA call."""
+    import numpy as np
+    lib = C.lib()
+    shp = C.Shape(2, 4, 2, 1024, 128, 64, 128)
+    kap = C.KapParams(budget=0.25, q_sub=32, k_sub=16)
+    ws = C.cosa_attention_host_workspace_size(shp, kap)
+    s, k, o = shp.c(), kap.c(shp), C._Osk(1e-4)
+    for bad in (-1, s.num_phys_pages):
+        pt = np.arange(2 * 16, dtype=np.int32).reshape(2, 16)
+        pt[1, 9] = bad
+        assert lib.cosa_attention_host(ctypes.byref(s), ctypes.byref(k), ctypes.byref(o), 16, 16,
+                                       16, pt.ctypes.data, 16, 256, ws, None) == 1
+    # padded rows (stride 20 for 16 pages): the bad entry sits where only the
+    # row stride, not the page count, reaches it
+    s2 = C.Shape(2, 4, 2, 1024, 128, 64, 128, pages_per_seq=20).c()
+    pt = np.zeros((2, 20), dtype=np.int32)
+    pt[:, :16] = np.arange(32, dtype=np.int32).reshape(2, 16)
+    pt[1, 14] = 99
+    assert lib.cosa_attention_host(ctypes.byref(s2), ctypes.byref(k), ctypes.byref(o), 16, 16, 16,
+                                   pt.ctypes.data, 16, 256, 1 << 40, None) == 1

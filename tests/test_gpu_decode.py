@@ -158,3 +158,92 @@ def test_decode_list_entry_past_the_query_is_reported_not_read():
         C.cosa_osk_decode(shape, C.OskParams(2.0), x["q"][:, :, t].contiguous().cuda(), xd["k_pool"],
                           xd["v_pool"], xd["page_table"], torch.tensor([t], dtype=torch.int32).cuda(),
                           order.cuda(), count.cuda(), out, ws)
+
+
+def test_decode_empty_list_and_position_out_of_range():
+    """A head with an empty list gets a zero output, LSE -inf and 0 computed; a
+    sequence whose position lies outside the cache is reported (status word) and its
+    heads get the same empty result, while the other sequence decodes normally."""
+    wl = W.small_workload("narrow-kv-64k", 4096, 7, 1, batch=2)
+    x = W.make_inputs(wl, seed=75)
+    xd = to_dev(x)
+    shape = shape_of(wl, x)
+    B, Hq, P = 2, 7, 64
+    positions = [3000, 5000]  # the second lies past the 4096-token cache
+    order = torch.full((B, Hq, 64), -1, dtype=torch.int32)
+    count = torch.zeros((B, Hq), dtype=torch.int32)
+    n = positions[0] // P + 1
+    order[0, :, :n] = torch.arange(n, dtype=torch.int32)
+    count[0, :] = n
+    count[0, 3] = 0  # an empty list
+    order[1, :, :5] = torch.arange(5, dtype=torch.int32)
+    count[1, :] = 5
+    qdec = torch.stack([x["q"][0, :, positions[0]], x["q"][1, :, 100]]).contiguous()
+    out = torch.full((B, Hq, 128), float("nan"), dtype=torch.bfloat16, device="cuda")
+    lse = torch.full((B, Hq), float("nan"), device="cuda")
+    comp = torch.full((B, Hq), -7, dtype=torch.int32, device="cuda")
+    ws = torch.empty(C.cosa_osk_decode_workspace_size(shape, 64), dtype=torch.uint8, device="cuda")
+    C.cosa_osk_decode(shape, C.OskParams(1e-4), qdec.cuda(), xd["k_pool"], xd["v_pool"],
+                      xd["page_table"], torch.tensor(positions, dtype=torch.int32).cuda(),
+                      order.cuda(), count.cuda(), out, ws, lse=lse, computed=comp)
+    torch.cuda.synchronize()
+    assert C.cosa_get_status() == 1  # the position out of range, reported
+    o, l, c = out.float().cpu(), lse.cpu(), comp.cpu()
+    for b, h in [(0, 3)] + [(1, h) for h in range(Hq)]:
+        assert torch.all(o[b, h] == 0) and l[b, h] == -math.inf and c[b, h] == 0
+    ref = O.osk_decode(np64(qdec[:1]), np64(x["k_pool"]), np64(x["v_pool"]),
+                       x["page_table"][:1].numpy(), positions[:1], order[:1].numpy(),
+                       count[:1].numpy(), num_kv_heads=1, page_size=P, eps=1e-4,
+                       scale=1 / math.sqrt(128))
+    heads = [h for h in range(Hq) if h != 3]
+    assert_out_close(o[0, heads].double().numpy(), ref["out"][0, heads], "decode batch row 0")
+
+
+def test_decode_page_outside_the_pool_is_reported_not_read():
+    """A list entry whose page-table entry lies outside the pool is reported and
+    treated as an invalid entry: the result equals the oracle's on the list without
+    it (a local max of -inf moves no running max and the entry is skipped)."""
+    wl = W.small_workload("gqa-32k", 4096, 4, 2, shuffle_pages=True)
+    x = W.make_inputs(wl, seed=76)
+    xd = to_dev(x)
+    shape = shape_of(wl, x)
+    t, bad_page, eps = 3500, 17, 1e-4
+    pt = xd["page_table"].clone()
+    pt[0, bad_page] = wl.num_pages + 5
+    n_all = t // 64 + 1
+    rng = np.random.default_rng(76)
+    order = np.full((1, 4, 64), -1, dtype=np.int32)
+    count = np.zeros((1, 4), dtype=np.int32)
+    for h in range(4):
+        lst = [p for p in rng.permutation(n_all) if p != bad_page][:30]
+        lst.insert(3 + h, bad_page)  # never first
+        order[0, h, :len(lst)] = lst
+        count[0, h] = len(lst)
+    qdec = x["q"][:, :, t].contiguous()
+    out = torch.full((1, 4, 128), float("nan"), dtype=torch.bfloat16, device="cuda")
+    lse = torch.full((1, 4), float("nan"), device="cuda")
+    comp = torch.full((1, 4), -7, dtype=torch.int32, device="cuda")
+    skip = torch.full((1, 4, 64), 7, dtype=torch.uint8, device="cuda")
+    ws = torch.empty(C.cosa_osk_decode_workspace_size(shape, 64), dtype=torch.uint8, device="cuda")
+    C.cosa_osk_decode(shape, C.OskParams(eps), qdec.cuda(), xd["k_pool"], xd["v_pool"], pt,
+                      torch.tensor([t], dtype=torch.int32).cuda(), torch.from_numpy(order).cuda(),
+                      torch.from_numpy(count).cuda(), out, ws, lse=lse, computed=comp,
+                      skip_log=skip)
+    torch.cuda.synchronize()
+    assert C.cosa_get_status() == 1
+    sk = skip.cpu().numpy()
+    order2 = np.full_like(order, -1)
+    count2 = count - 1
+    for h in range(4):
+        assert sk[0, h, 3 + h] == 1  # the entry is skipped
+        order2[0, h, :count2[0, h]] = [p for p in order[0, h, :count[0, h]] if p != bad_page]
+    ref = O.osk_decode(np64(qdec), np64(x["k_pool"]), np64(x["v_pool"]), x["page_table"].numpy(),
+                       [t], order2, count2, num_kv_heads=2, page_size=64, eps=eps,
+                       scale=1 / math.sqrt(128))
+    for h in range(4):
+        n = int(count[0, h])
+        mine = np.delete(sk[0, h, :n], 3 + h)
+        amb = np.abs(ref["margin"][0, h, :n - 1]) <= SKIP_MARGIN
+        assert np.all((mine == ref["skip"][0, h, :n - 1]) | amb)
+    assert_out_close(np64(out), ref["out"], "decode without the bad page")
+    assert_lse_close(lse.cpu().numpy(), ref["lse"], "decode without the bad page")

@@ -140,3 +140,24 @@ def test_preskip_128k_long_lists():
         n = int(c0[0, 0, qb])
         keep = o0[0, 0, qb, :n][lg[0, 0, qb, :n] == 0]
         assert int(c1[0, 0, qb]) == len(keep) and o1[0, 0, qb, :len(keep)].tolist() == keep.tolist()
+
+
+def test_preskip_invalid_list_is_reported_and_left():
+    wl = W.small_workload("gqa-32k", 2048, 2, 1)
+    x = W.make_inputs(wl, seed=64)
+    xd, shape, kap, order, count, ws = _gpu_lists(wl, x, 0.5)
+    assert int(count[0, 0, 5]) >= 2
+    order[0, 0, 5, 1] = 40  # q-block 5 sees pages 0..11 only
+    o0, c0 = order.clone(), count.clone()
+    C.cosa_kap_preskip(shape, kap, 1e-2, 0.0, order, count, ws)
+    torch.cuda.synchronize()
+    assert C.cosa_get_status() == 1  # COSA_ERR_INVALID_ARG
+    assert torch.equal(order[0, 0, 5], o0[0, 0, 5]) and count[0, 0, 5] == c0[0, 0, 5]
+    # the other lists were filtered: each is a subsequence of its input that keeps its
+    # first page
+    for (b, h, qb) in [(0, 0, 4), (0, 1, 10), (0, 1, 15)]:
+        n0, n = int(c0[b, h, qb]), int(count[b, h, qb])
+        src, got = o0[b, h, qb, :n0].tolist(), order[b, h, qb, :n].tolist()
+        assert got[0] == src[0] and 1 <= n <= n0
+        it = iter(src)
+        assert all(pg in it for pg in got)
