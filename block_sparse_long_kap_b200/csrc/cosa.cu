@@ -483,37 +483,46 @@ cosa_status_t noalloc_scratch_address(void** out) {
 size_t al256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
 struct HostLayout {
-  cosa_shape_t sub;  // one KV head: H_q = G, H_kv = 1
+  cosa_shape_t sub;  // one query head with its KV head: H_q = 1, H_kv = 1
   int32_t k_cap;
-  size_t q, kv, ord, cnt, pt, kapws;       // bytes: one head's Q (or O), K (or V) pool, lists
-  size_t set_k, set_v, set_o, set_bytes;   // offsets inside one buffer set (Q at 0)
-  size_t off_set[2], off_ord, off_cnt, off_kapws, total;  // page table at 0
+  size_t q, kv, ord, cnt, pt, kapws;  // bytes: one query head's Q (or O) over the batch, one
+                                      // KV head's K (or V) pool column, lists, page table
+  size_t off_kv[2][2];                // [set][K, V]
+  size_t off_q[3], off_o[3];          // query-head slots
+  size_t off_ord, off_cnt, off_kapws, total;  // page table at 0
 };
+constexpr int kHostQSlots = 3;
 
 cosa_status_t host_layout(const cosa_shape_t* s, const cosa_kap_params_t* kap, HostLayout* L) {
   cosa_status_t e = check_shape(s);
   if (e != COSA_OK) return e;
   if ((e = check_kap(s, kap)) != COSA_OK) return e;
   L->sub = *s;
-  L->sub.num_q_heads = s->num_q_heads / s->num_kv_heads;
+  L->sub.num_q_heads = 1;
   L->sub.num_kv_heads = 1;
   const cosa_shape_t* u = &L->sub;
   L->k_cap = kcap_of(u, kap);
   const size_t nqb = static_cast<size_t>(u->seq_len / u->q_block);
-  const size_t bh = static_cast<size_t>(u->batch) * u->num_q_heads;
+  const size_t bh = static_cast<size_t>(u->batch);
   L->q = bh * u->seq_len * u->head_dim * 2;
   L->kv = static_cast<size_t>(u->num_phys_pages) * u->page_size * u->head_dim * 2;
   L->ord = bh * nqb * L->k_cap * 4;
   L->cnt = bh * nqb * 4;
   L->pt = static_cast<size_t>(s->batch) * s->pages_per_seq * 4;
   L->kapws = kap_layout(u, kap).total;
-  L->set_k = al256(L->q);
-  L->set_v = L->set_k + al256(L->kv);
-  L->set_o = L->set_v + al256(L->kv);
-  L->set_bytes = L->set_o + al256(L->q);
-  L->off_set[0] = al256(L->pt);
-  L->off_set[1] = L->off_set[0] + L->set_bytes;
-  L->off_ord = L->off_set[1] + L->set_bytes;
+  size_t off = al256(L->pt);
+  for (int x = 0; x < 2; ++x)
+    for (int t = 0; t < 2; ++t) {
+      L->off_kv[x][t] = off;
+      off += al256(L->kv);
+    }
+  for (int y = 0; y < kHostQSlots; ++y) {
+    L->off_q[y] = off;
+    off += al256(L->q);
+    L->off_o[y] = off;
+    off += al256(L->q);
+  }
+  L->off_ord = off;
   L->off_cnt = L->off_ord + al256(L->ord);
   L->off_kapws = L->off_cnt + al256(L->cnt);
   L->total = L->off_kapws + al256(L->kapws);
@@ -525,26 +534,31 @@ cosa_status_t host_layout(const cosa_shape_t* s, const cosa_kap_params_t* kap, H
 struct HostPipe {
   cudaStream_t in = nullptr, out = nullptr;
   cudaEvent_t start = nullptr, fin_in = nullptr, fin_out = nullptr;
-  cudaEvent_t loaded[2] = {}, used[2] = {}, drained[2] = {};
+  cudaEvent_t kv_loaded[2] = {}, kv_used[2] = {};
+  cudaEvent_t q_loaded[kHostQSlots] = {}, q_used[kHostQSlots] = {}, o_drained[kHostQSlots] = {};
+  cudaEvent_t* all(int i) {
+    cudaEvent_t* evs[] = {&start, &fin_in, &fin_out, &kv_loaded[0], &kv_loaded[1], &kv_used[0],
+                          &kv_used[1], &q_loaded[0], &q_loaded[1], &q_loaded[2], &q_used[0],
+                          &q_used[1], &q_used[2], &o_drained[0], &o_drained[1], &o_drained[2]};
+    return evs[i];
+  }
+  static constexpr int kEvents = 16;
   bool create() {
     if (cudaStreamCreateWithFlags(&in, cudaStreamNonBlocking) != cudaSuccess ||
         cudaStreamCreateWithFlags(&out, cudaStreamNonBlocking) != cudaSuccess)
       return false;
-    cudaEvent_t* evs[] = {&start, &fin_in, &fin_out, &loaded[0], &loaded[1],
-                          &used[0], &used[1], &drained[0], &drained[1]};
-    for (cudaEvent_t* e : evs)
-      if (cudaEventCreateWithFlags(e, cudaEventDisableTiming) != cudaSuccess) return false;
+    for (int i = 0; i < kEvents; ++i)
+      if (cudaEventCreateWithFlags(all(i), cudaEventDisableTiming) != cudaSuccess) return false;
     return true;
   }
   ~HostPipe() {
-    cudaEvent_t evs[] = {start, fin_in, fin_out, loaded[0], loaded[1],
-                         used[0], used[1], drained[0], drained[1]};
-    for (cudaEvent_t e : evs)
-      if (e) cudaEventDestroy(e);
+    for (int i = 0; i < kEvents; ++i)
+      if (*all(i)) cudaEventDestroy(*all(i));
     if (in) cudaStreamDestroy(in);
     if (out) cudaStreamDestroy(out);
   }
 };
+static_assert(kHostQSlots == 3, "the event list above names three slots");
 
 }  // namespace
 
@@ -1018,43 +1032,56 @@ cosa_status_t cosa_attention_host(const cosa_shape_t* shape, const cosa_kap_para
             cudaMemcpyAsync(pt_d, page_table_host, L.pt, cudaMemcpyHostToDevice, pp.in) ==
                 cudaSuccess;
   e = ok ? COSA_OK : COSA_ERR_CUDA;
+  // One query head at a time (unit u = c * G + g: KV head c, its query head g), so
+  // the last unit's kernels and read-back, which no copy-in overlaps, are short.
+  // KV head c's pool columns go into set c % 2, reloaded once the kernels of its
+  // last query head are done; query head u's Q and O use slot u % 3, Q reloaded once
+  // the unit's kernels are done and O rewritten once its read-back is done.
   for (int c = 0; e == COSA_OK && c < Hkv; ++c) {
     const int x = c & 1;
-    uint8_t* set = ws + L.off_set[x];
-    uint8_t *q_d = set, *k_d = set + L.set_k, *v_d = set + L.set_v, *o_d = set + L.set_o;
-    // KV head c in: its G query heads of every sequence, its column of the page pools
-    // (one page-sized row per physical page), once the kernels of head c - 2 are done
-    // with this buffer set
-    ok = c < 2 || cudaStreamWaitEvent(pp.in, pp.used[x], 0) == cudaSuccess;
-    for (int b = 0; ok && b < B; ++b)
-      ok = cudaMemcpyAsync(q_d + static_cast<size_t>(b) * G * head_bytes,
-                           qh + (static_cast<size_t>(b) * Hq + static_cast<size_t>(c) * G) * head_bytes,
-                           G * head_bytes, cudaMemcpyHostToDevice, pp.in) == cudaSuccess;
-    ok = ok &&
+    uint8_t* k_d = ws + L.off_kv[x][0];
+    uint8_t* v_d = ws + L.off_kv[x][1];
+    // KV head c's column of the page pools (one page-sized row per physical page)
+    ok = (c < 2 || cudaStreamWaitEvent(pp.in, pp.kv_used[x], 0) == cudaSuccess) &&
          cudaMemcpy2DAsync(k_d, page_bytes, kh + c * page_bytes, Hkv * page_bytes, page_bytes,
                            shape->num_phys_pages, cudaMemcpyHostToDevice, pp.in) == cudaSuccess &&
          cudaMemcpy2DAsync(v_d, page_bytes, vh + c * page_bytes, Hkv * page_bytes, page_bytes,
                            shape->num_phys_pages, cudaMemcpyHostToDevice, pp.in) == cudaSuccess &&
-         cudaEventRecord(pp.loaded[x], pp.in) == cudaSuccess &&
-         // the kernels wait for the inputs and for the read-back of head c - 2's output
-         cudaStreamWaitEvent(st, pp.loaded[x], 0) == cudaSuccess &&
-         (c < 2 || cudaStreamWaitEvent(st, pp.drained[x], 0) == cudaSuccess);
+         cudaEventRecord(pp.kv_loaded[x], pp.in) == cudaSuccess &&
+         cudaStreamWaitEvent(st, pp.kv_loaded[x], 0) == cudaSuccess;
     if (!ok) { e = COSA_ERR_CUDA; break; }
-    e = cosa_kap_select(&L.sub, kap, q_d, k_d, pt_d, ord_d, cnt_d, nullptr, nullptr, kapws_d,
-                        L.kapws, stream);
-    if (e != COSA_OK) break;
-    e = cosa_osk_attention(&L.sub, osk, q_d, k_d, v_d, pt_d, ord_d, cnt_d, L.k_cap, o_d, nullptr,
-                           nullptr, nullptr, stream);
-    if (e != COSA_OK) break;
-    // head c's output back to its place in out_host
-    ok = cudaEventRecord(pp.used[x], st) == cudaSuccess &&
-         cudaStreamWaitEvent(pp.out, pp.used[x], 0) == cudaSuccess;
-    for (int b = 0; ok && b < B; ++b)
-      ok = cudaMemcpyAsync(oh + (static_cast<size_t>(b) * Hq + static_cast<size_t>(c) * G) * head_bytes,
-                           o_d + static_cast<size_t>(b) * G * head_bytes, G * head_bytes,
-                           cudaMemcpyDeviceToHost, pp.out) == cudaSuccess;
-    ok = ok && cudaEventRecord(pp.drained[x], pp.out) == cudaSuccess;
-    if (!ok) e = COSA_ERR_CUDA;
+    for (int g = 0; g < G; ++g) {
+      const int unit = c * G + g, y = unit % kHostQSlots;
+      const int h = c * G + g;
+      uint8_t* q_d = ws + L.off_q[y];
+      uint8_t* o_d = ws + L.off_o[y];
+      // query head h of every sequence in
+      ok = unit < kHostQSlots || cudaStreamWaitEvent(pp.in, pp.q_used[y], 0) == cudaSuccess;
+      for (int b = 0; ok && b < B; ++b)
+        ok = cudaMemcpyAsync(q_d + static_cast<size_t>(b) * head_bytes,
+                             qh + (static_cast<size_t>(b) * Hq + h) * head_bytes, head_bytes,
+                             cudaMemcpyHostToDevice, pp.in) == cudaSuccess;
+      ok = ok && cudaEventRecord(pp.q_loaded[y], pp.in) == cudaSuccess &&
+           cudaStreamWaitEvent(st, pp.q_loaded[y], 0) == cudaSuccess &&
+           (unit < kHostQSlots || cudaStreamWaitEvent(st, pp.o_drained[y], 0) == cudaSuccess);
+      if (!ok) { e = COSA_ERR_CUDA; break; }
+      e = cosa_kap_select(&L.sub, kap, q_d, k_d, pt_d, ord_d, cnt_d, nullptr, nullptr, kapws_d,
+                          L.kapws, stream);
+      if (e != COSA_OK) break;
+      e = cosa_osk_attention(&L.sub, osk, q_d, k_d, v_d, pt_d, ord_d, cnt_d, L.k_cap, o_d,
+                             nullptr, nullptr, nullptr, stream);
+      if (e != COSA_OK) break;
+      ok = cudaEventRecord(pp.q_used[y], st) == cudaSuccess &&
+           (g < G - 1 || cudaEventRecord(pp.kv_used[x], st) == cudaSuccess) &&
+           cudaStreamWaitEvent(pp.out, pp.q_used[y], 0) == cudaSuccess;
+      // its output back to its place in out_host
+      for (int b = 0; ok && b < B; ++b)
+        ok = cudaMemcpyAsync(oh + (static_cast<size_t>(b) * Hq + h) * head_bytes,
+                             o_d + static_cast<size_t>(b) * head_bytes, head_bytes,
+                             cudaMemcpyDeviceToHost, pp.out) == cudaSuccess;
+      ok = ok && cudaEventRecord(pp.o_drained[y], pp.out) == cudaSuccess;
+      if (!ok) { e = COSA_ERR_CUDA; break; }
+    }
   }
   // the caller's stream holds until everything queued above (copies included) is done
   const bool joined = cudaEventRecord(pp.fin_in, pp.in) == cudaSuccess &&

@@ -342,15 +342,15 @@ cosa_status_t cosa_dense_attention(const cosa_shape_t* shape, const void* q, con
 cosa_status_t cosa_attention_host_workspace_size(const cosa_shape_t* shape,
                                                  const cosa_kap_params_t* kap, size_t* bytes);
 
-/* Both stages end to end from host memory: for every KV head, copy its G query
- * heads of Q (every sequence) and its column of the K and V page pools to the
- * device, run cosa_kap_select and cosa_osk_attention on that head alone (shape
- * with H_q = G, H_kv = 1: heads are independent in both stages, so the result
- * equals the whole-layer calls), and copy its output back to its place in
- * out_host.  The copies of the next KV head and the read-back of the previous
- * one run on two streams of the call's own, overlapping the kernels, which run
- * on `stream`; `stream` waits for all of it, so synchronising `stream` means the
- * output is in out_host.  q_host bf16 [B][H_q][N][D], k_pool_host / v_pool_host
+/* Both stages end to end from host memory: for every KV head, copy its column of
+ * the K and V page pools to the device, and for each of its G query heads in turn
+ * copy that head's Q (every sequence), run cosa_kap_select and cosa_osk_attention on
+ * that query head alone (shape with H_q = 1, H_kv = 1: heads are independent in both
+ * stages, so the result equals the whole-layer calls) and copy its output back to
+ * its place in out_host.  The copies in and the read-backs run on two streams of
+ * the call's own, overlapping the kernels, which run on `stream`; `stream` waits for
+ * all of it, so synchronising `stream` means the output is in out_host.  q_host
+ * bf16 [B][H_q][N][D], k_pool_host / v_pool_host
  * bf16 [num_phys_pages][H_kv][P][D], page_table_host int32 [B][pages_per_seq]
  * and out_host bf16 [B][H_q][N][D] are host memory; page-locked memory lets the
  * copies overlap the kernels (pageable memory works but the copies serialise).

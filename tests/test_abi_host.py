@@ -144,17 +144,19 @@ def test_group_entry_points_reject_bad_arguments_before_launch():
 
 
 def test_host_pipeline_workspace_and_argument_checks():
-    """cosa_attention_host: the workspace holds two sets of one KV head's inputs and
-    output plus that head's lists and KAP workspace; bad arguments return before
-    anything is queued (no CUDA call is made on these paths)."""
+    """cosa_attention_host: the workspace holds two sets of one KV head's K and V pool
+    columns, three slots of one query head's Q and O (over the batch), and one query
+    head's lists and KAP workspace; bad arguments return before anything is queued
+    (no CUDA call is made on these paths)."""
     lib = C.lib()
     shp = C.Shape(2, 8, 2, 2048, 128, 64, 128)
     kap = C.KapParams(budget=0.25, q_sub=32, k_sub=16)
     ws = C.cosa_attention_host_workspace_size(shp, kap)
-    sub = C.Shape(2, 4, 1, 2048, 128, 64, 128)
-    q_head = 2 * 4 * 2048 * 128 * 2
+    sub = C.Shape(2, 1, 1, 2048, 128, 64, 128, num_phys_pages=shp.c().num_phys_pages)
+    q_head = 2 * 1 * 2048 * 128 * 2
     kv_head = shp.c().num_phys_pages * 64 * 128 * 2
-    assert ws >= 2 * (2 * q_head + 2 * kv_head) + C.cosa_kap_workspace_size(sub, kap)
+    need = 2 * 2 * kv_head + 3 * 2 * q_head + C.cosa_kap_workspace_size(sub, kap)
+    assert need <= ws <= need + 64 * 1024 + 2 * 2 * 1024 * C.cosa_kap_kcap(sub, kap) * 4
     s, k, o = shp.c(), kap.c(shp), C._Osk(1e-4)
     # null host buffer, negative eps, missing / small / misaligned workspace
     assert lib.cosa_attention_host(ctypes.byref(s), ctypes.byref(k), ctypes.byref(o), None, 16, 16,
