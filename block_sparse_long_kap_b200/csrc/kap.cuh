@@ -298,6 +298,42 @@ __device__ __forceinline__ int block_excl_scan(int v, int* warp_sums, int* total
   return before;
 }
 
+// Descending bitonic sort of 32 E 64-bit keys held by one warp: element e = 32 i + lane
+// in x[i].  Pairs 32 or more apart sit in one lane's registers; the others are exchanged
+// between lanes.  Fully unrolled, so every register index is a constant.
+template <int E>
+__device__ __forceinline__ void warp_sort_desc(unsigned long long (&x)[E]) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int kk = 2; kk <= 32 * E; kk <<= 1) {
+#pragma unroll
+    for (int j = kk >> 1; j > 0; j >>= 1) {
+      if (j >= 32) {
+        const int jj = j >> 5;
+#pragma unroll
+        for (int i = 0; i < E; ++i) {
+          if ((i ^ jj) > i) {
+            const int e = 32 * i + lane;
+            const unsigned long long a = x[i], b = x[i ^ jj];
+            const bool desc = (e & kk) == 0;  // larger first in this block
+            const bool sw = desc ? (a < b) : (a > b);
+            x[i] = sw ? b : a;
+            x[i ^ jj] = sw ? a : b;
+          }
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < E; ++i) {
+          const int e = 32 * i + lane;
+          const unsigned long long y = __shfl_xor_sync(0xffffffffu, x[i], j);
+          const bool keep_max = ((e & j) == 0) == ((e & kk) == 0);
+          x[i] = keep_max ? (x[i] > y ? x[i] : y) : (x[i] < y ? x[i] : y);
+        }
+      }
+    }
+  }
+}
+
 struct KapPageMax {
   const float* a;       // triangular page maxima (see kap_tc.cuh)
   const float* row_max; // [B * H_kv * nQB * G * R]
@@ -494,14 +530,36 @@ __global__ void __launch_bounds__(ORDER_THREADS, 3) kap_order_kernel(
     while (m < total) m <<= 1;
     for (int p = beg; p < beg + per && p < n_b; ++p)
       if (selected(p)) kept[pos++] = keys[p];
-    if (total <= (int)blockDim.x) {
-      // up to one key per thread: a key's place is the number of larger keys (the
-      // keys are distinct: the page is in the low bits), read by broadcast
+    if (total <= 32 * (int)(blockDim.x >> 5)) {
+      // up to one run of 32 keys per warp: each warp sorts its run in registers, then
+      // each key's place is its place in its run plus, for every other run, the
+      // number of that run's keys above it (a binary search: runs are descending, and
+      // the zero keys that pad the last run lie below every key)
+      const int lane = (int)threadIdx.x & 31, warp = (int)threadIdx.x >> 5;
+      const int runs = (total + 31) >> 5;
+      __syncthreads();
+      if (warp < runs) {
+        const int e = 32 * warp + lane;
+        unsigned long long x[1] = {e < total ? kept[e] : 0ull};
+        warp_sort_desc<1>(x);
+        kept[e] = x[0];
+      }
       __syncthreads();
       if ((int)threadIdx.x < total) {
-        const unsigned long long mine = kept[threadIdx.x];
-        int rank = 0;
-        for (int k = 0; k < total; ++k) rank += kept[k] > mine;
+        const int t = (int)threadIdx.x, own = t >> 5;
+        const unsigned long long mine = kept[t];
+        int rank = t & 31;
+        for (int r = 0; r < runs; ++r) {
+          if (r == own) continue;
+          const unsigned long long* run = kept + 32 * r;
+          int lo = 0, hi = 32;  // first index whose key is not above mine
+          while (lo < hi) {
+            const int mid = (lo + hi) >> 1;
+            if (run[mid] > mine) lo = mid + 1;
+            else hi = mid;
+          }
+          rank += lo;
+        }
         orow[rank] = 0x7fffffff - (int)(mine & 0x7fffffffull);
       }
     } else {
