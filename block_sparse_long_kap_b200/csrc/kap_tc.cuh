@@ -217,17 +217,35 @@ __global__ void __launch_bounds__(192, 1)
         tmem_ld32(t_row + buf * C::BN + c * 32, raw);
         const int s0 = ct * C::BN + c * 32;  // sub-key of column 0 (a multiple of T)
         const int pg0 = s0 / T;
+        constexpr int NPG = 32 / T;          // pages of this chunk
+        float v[NPG];
 #pragma unroll
-        for (int k = 0; k < 32 / T; ++k) {
+        for (int k = 0; k < NPG; ++k) {
           const int pg = pg0 + k;
-          float v = -INFINITY;
+          v[k] = -INFINITY;
 #pragma unroll
           for (int t = 0; t < T; ++t) {
-            if (pg * P + t * ksub <= rep_last) v = fmaxf(v, __uint_as_float(raw[k * T + t]) * scale);
+            if (pg * P + t * ksub <= rep_last) v[k] = fmaxf(v[k], __uint_as_float(raw[k * T + t]) * scale);
           }
-          if (valid && pg < n_b) {
-            arow[pg] = v;
-            if (v > m) { m = v; arg = pg; }
+          if (valid && pg < n_b && v[k] > m) { m = v[k]; arg = pg; }
+        }
+        // the chunk's page maxima with the widest stores the row's alignment allows
+        // (one row per thread: scalar stores send a request per page and row)
+        if (valid && pg0 < n_b) {
+          float* dst = arow + pg0;
+          const uintptr_t ad = reinterpret_cast<uintptr_t>(dst);
+          if (pg0 + NPG <= n_b && NPG % 4 == 0 && (ad & 15) == 0) {
+#pragma unroll
+            for (int k = 0; k < NPG; k += 4)
+              *reinterpret_cast<float4*>(dst + k) = make_float4(v[k], v[k + 1], v[k + 2], v[k + 3]);
+          } else if (pg0 + NPG <= n_b && NPG % 2 == 0 && (ad & 7) == 0) {
+#pragma unroll
+            for (int k = 0; k < NPG; k += 2)
+              *reinterpret_cast<float2*>(dst + k) = make_float2(v[k], v[k + 1]);
+          } else {
+#pragma unroll
+            for (int k = 0; k < NPG; ++k)
+              if (pg0 + k < n_b) dst[k] = v[k];
           }
         }
       }
