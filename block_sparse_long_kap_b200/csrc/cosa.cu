@@ -5,6 +5,7 @@
 #include <cstdio>
 #include <cstring>
 #include <mutex>
+#include <type_traits>
 
 #include <cudaTypedefs.h>
 
@@ -176,8 +177,15 @@ cosa_status_t launch_order(const cosa_shape_t* s, const cosa_kap_params_t* k, bo
   const size_t smem = (size_t)(npow2 + (npow2 < 32 ? 32 : npow2)) * 8;
   if (smem > 200 * 1024) return COSA_ERR_UNSUPPORTED;
   if (from_a && (group ? pm.group : 1) * pm.R > ORDER_MAX_ROWS) return COSA_ERR_UNSUPPORTED;
-  auto kern = !from_a ? kap_order_kernel<false, false>
-                      : (group ? kap_order_kernel<true, true> : kap_order_kernel<true, false>);
+  const int R = s->q_block / k->q_sub;  // a power of two up to 8 (check_kap)
+  auto pick = [&](auto g) {
+    constexpr bool G = decltype(g)::value;
+    return R == 1 ? kap_order_kernel<true, G, 1>
+         : R == 2 ? kap_order_kernel<true, G, 2>
+         : R == 4 ? kap_order_kernel<true, G, 4> : kap_order_kernel<true, G, 8>;
+  };
+  auto kern = !from_a ? kap_order_kernel<false, false, 0>
+                      : (group ? pick(std::true_type()) : pick(std::false_type()));
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
       cudaSuccess)
     return COSA_ERR_CUDA;

@@ -343,7 +343,9 @@ struct KapPageMax {
 
 constexpr int ORDER_MAX_ROWS = 64;  // representative rows read by one CTA (G * R in group mode)
 
-template <bool FROM_A, bool GROUP>
+// RT: representatives per q-block and head (q_block / q_sub) fixed at compile time, so the
+// per-page loop over them carries no dead iterations; 0 where the scores come given
+template <bool FROM_A, bool GROUP, int RT>
 __global__ void __launch_bounds__(ORDER_THREADS, 3) kap_order_kernel(
     const float* __restrict__ scores, const uint8_t* __restrict__ hrm, KapPageMax pm,
     float* __restrict__ scores_out, uint8_t* __restrict__ hrm_out, int32_t* __restrict__ order,
@@ -391,6 +393,15 @@ __global__ void __launch_bounds__(ORDER_THREADS, 3) kap_order_kernel(
     }
     __syncthreads();
   }
+  // (one head's row maxima and first maximal pages, in registers)
+  constexpr int RM = RT > 0 ? RT : 1;
+  float m_r[RM];
+  int arg_r[RM];
+#pragma unroll
+  for (int i = 0; i < RM; ++i) {
+    m_r[i] = FROM_A && !GROUP ? m_s[i] : 0.f;
+    arg_r[i] = FROM_A && !GROUP ? arg_s[i] : -1;
+  }
   const float* srow = FROM_A ? nullptr : scores + row * num_pages;
   const uint8_t* hrow = FROM_A ? nullptr : hrm + row * num_pages;
   const float invR = FROM_A ? 1.0f / (float)pm.R : 0.f;  // R is a power of two
@@ -406,18 +417,15 @@ __global__ void __launch_bounds__(ORDER_THREADS, 3) kap_order_kernel(
         sv = 0.f;
         flag = 0;
         for (int g = 0; g < n_heads; ++g) {
-          float av[8];
+          float av[RM];
 #pragma unroll
-          for (int i = 0; i < 8; ++i)
-            av[i] = i < pm.R ? arow[(long long)(g * pm.R + i) * n_b + p] : 0.f;
+          for (int i = 0; i < RM; ++i) av[i] = arow[(long long)(g * RM + i) * n_b + p];
           float sg = 0.f;
 #pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            if (i < pm.R) {
-              const int r = g * pm.R + i;
-              sg += expf(av[i] - m_s[r]);
-              flag |= (arg_s[r] == p);
-            }
+          for (int i = 0; i < RM; ++i) {
+            const int r = g * RM + i;
+            sg += expf(av[i] - (GROUP ? m_s[r] : m_r[i]));
+            flag |= ((GROUP ? arg_s[r] : arg_r[i]) == p);
           }
           sv = fmaxf(sv, sg * invR);
         }
