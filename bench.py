@@ -38,8 +38,8 @@ WORKLOAD = "gqa-128k"
 # of these kernels.  Each figure describes the kernel source the capture ran,
 # identified by a hash of the files below; any other source reports null.
 TRAFFIC = {
-    "osk": {"workload": "gqa-128k", "bytes": 1653753600 + 1038393856,
-            "source_sha256_16": "f772f35140ec898d",
+    "osk": {"workload": "gqa-128k", "bytes": 1652753920 + 1035382784,
+            "source_sha256_16": "58ec01c35dcc6e5a",
             "files": ("attn_tc.cuh", "tc_ptx.cuh", "common.cuh")},
     "kap_pool": {"workload": "gqa-128k", "bytes": 1342215168 + 184500224,
                  "source_sha256_16": "db13d4d202b518c7",
@@ -488,6 +488,8 @@ def main():
                     help="run only the first K KV heads of the layer (a smaller case of the "
                          "same layer, for profiling; one GPU)")
     ap.add_argument("--no-extras", action="store_true", help="skip dense/sweep/e2e/cpu legs")
+    ap.add_argument("--no-sweep", action="store_true",
+                    help="skip the per-budget sweep leg (the same fixed layers whatever --workload)")
     ap.add_argument("--sweep-only", action="store_true",
                     help="run only the per-budget sweep and print it")
     ap.add_argument("--decode-only", action="store_true",
@@ -956,10 +958,11 @@ def main():
     torch.cuda.empty_cache()
 
     # ---- speedup per budget on the other long-context layers ----------------
-    try:
-        line["budget_sweep"] = budget_sweep(C, W, dev, stream, burst)
-    except Exception as exc:  # an extra leg: report the failure, keep the line
-        line["budget_sweep"] = {"error": repr(exc)}
+    if not args.no_sweep:
+        try:
+            line["budget_sweep"] = budget_sweep(C, W, dev, stream, burst)
+        except Exception as exc:  # an extra leg: report the failure, keep the line
+            line["budget_sweep"] = {"error": repr(exc)}
 
     # ---- CPU oracle on a bounded sample of the same workload ----------------
     xh = {"q": x["q"][:, :1].cpu(), "k_pool": x["k_pool"][:, :1].cpu(),

@@ -175,16 +175,11 @@ __global__ void __launch_bounds__(384, 1)
   auto wait = [&](uint32_t bar_addr, uint32_t parity) -> bool {
     if (mbar_try_wait(bar_addr, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
-    uint32_t n = 0;
     while (!mbar_try_wait(bar_addr, parity)) {
-      // (the status word is a global load: read it now and then, not on every turn,
-      // or its latency delays the wake-up when the phase completes)
-      if ((++n & 31u) == 0) {
-        if (*abort_flag) return false;
-        if (timed_out(t0)) {
-          give_up();
-          return false;
-        }
+      if (*abort_flag) return false;
+      if (timed_out(t0)) {
+        give_up();
+        return false;
       }
     }
     return true;
