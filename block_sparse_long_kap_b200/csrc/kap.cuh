@@ -20,6 +20,8 @@
 //                     scores (cosa_kap_order).
 #pragma once
 
+#include <type_traits>
+
 #include "common.cuh"
 
 namespace cosa {
@@ -222,22 +224,30 @@ __global__ void __launch_bounds__(256) prefill_write_kernel(
   float acc[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+  // one loop per case (Q rows; K and V rows; K rows of a page outside the pool, pooled
+  // only), so no loop carries a branch per row
+  auto rows_loop = [&](auto copy_k, auto copy_v) {
+    constexpr bool CK = decltype(copy_k)::value, CV = decltype(copy_v)::value;
 #pragma unroll 4
-  for (int r = lane / LPR; r < rows; r += RPI) {
-    const uint4 v = __ldg(reinterpret_cast<const uint4*>(src + (long long)r * src_stride) + c);
-    if (dst) reinterpret_cast<uint4*>(dst + (long long)r * D)[c] = v;
-    if (vdst) {
-      const uint4 vv = __ldg(reinterpret_cast<const uint4*>(vsrc + (long long)r * src_stride) + c);
-      reinterpret_cast<uint4*>(vdst + (long long)r * D)[c] = vv;
-    }
-    const __nv_bfloat162* hh = reinterpret_cast<const __nv_bfloat162*>(&v);
+    for (int r = lane / LPR; r < rows; r += RPI) {
+      const uint4 v = __ldg(reinterpret_cast<const uint4*>(src + (long long)r * src_stride) + c);
+      if (CK) reinterpret_cast<uint4*>(dst + (long long)r * D)[c] = v;
+      if (CV) {
+        const uint4 vv = __ldg(reinterpret_cast<const uint4*>(vsrc + (long long)r * src_stride) + c);
+        reinterpret_cast<uint4*>(vdst + (long long)r * D)[c] = vv;
+      }
+      const __nv_bfloat162* hh = reinterpret_cast<const __nv_bfloat162*>(&v);
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      float2 f = __bfloat1622float2(hh[i]);
-      acc[2 * i] += f.x;
-      acc[2 * i + 1] += f.y;
+      for (int i = 0; i < 4; ++i) {
+        float2 f = __bfloat1622float2(hh[i]);
+        acc[2 * i] += f.x;
+        acc[2 * i + 1] += f.y;
+      }
     }
-  }
+  };
+  if (vdst) rows_loop(std::true_type(), std::true_type());
+  else if (dst) rows_loop(std::true_type(), std::false_type());
+  else rows_loop(std::false_type(), std::false_type());
   if (!pool) return;
 #pragma unroll
   for (int off = LPR; off < 32; off <<= 1) {
